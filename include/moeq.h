@@ -1,0 +1,196 @@
+/*
+ * moeq.h -- C ABI of libmoeq.so: the decode-time quantized Mixture-of-Experts
+ * FFN step on NVIDIA B200 (sm_100a).
+ *
+ * One token (or a small batch of tokens) passes through one MoE layer:
+ *   1. router GEMV, logits = W_r x, then softmax and top-K over E experts;
+ *   2. for each selected expert and for the always-on shared expert, the
+ *      gate and up projections as group-affine low-bit dequant mat-vecs,
+ *      w = q*scale + bias per group of G consecutive inputs, evaluated in the
+ *      rearranged form fma(q, scale*x, bias*x) summed per group;
+ *   3. SwiGLU, h = silu(gate) * up;
+ *   4. the down projection, a dequant mat-vec of h;
+ *   5. the weighted combine with the shared expert and the residual, with an
+ *      optional RMSNorm'd bf16 copy for the next layer.
+ *
+ * Sources, cited by page title and section:
+ *   "Flash-MoE - Chay mo hinh 397 ty tham so tren laptop"
+ *   (vi.news.hada.io/topic?id=27758):
+ *     "Kien truc mo hinh"           512 experts, K=4 active, hidden 4096;
+ *     "SSD Expert Streaming"        about 6.75 MB per 4-bit expert;
+ *     "Kernel dequant toi uu FMA"   (nibble*scale+bias)*x as
+ *                                   fma(nibble, scale*x, bias*x);
+ *     "Metal Compute Shaders"       4-bit/2-bit dequant mat-vec, SwiGLU,
+ *                                   RMS norm, MoE combine + residual + gate;
+ *     "Deferred GPU Expert Compute" combine + norm + residual on the GPU,
+ *                                   handed straight to the next layer.
+ *   "LOOM" (alessandroviola.dev/it/research/loom/): expert-major storage.
+ *
+ * Conventions for every call:
+ *   - Pointers named *_bf16 hold IEEE bfloat16 values; all buffers except the
+ *     moe_layer_q struct itself are DEVICE memory owned by the caller. The
+ *     library never allocates or frees device memory.
+ *   - Device pointers must be 16-byte aligned (MOE_ERR_ALIGN otherwise).
+ *   - Calls are asynchronous on `stream` (a cudaStream_t; NULL = legacy
+ *     default stream) and never synchronise, except moe_get_device_error.
+ *   - Argument errors are found on the host before any launch and returned
+ *     as a status; nothing is launched then.
+ *   - Errors found on the device (an expert index outside [0, E), a code
+ *     that does not fit its bit width) set an error word in the workspace
+ *     and the affected output is written as zero; kernels never trap.
+ *     Read it with moe_get_device_error.
+ *   - A workspace is caller-allocated device memory of at least
+ *     moe_workspace_bytes(...) bytes, zeroed once with moe_workspace_init
+ *     before first use. Calls that share a workspace must be ordered on one
+ *     stream; distinct workspaces make calls independent.
+ */
+#ifndef MOEQ_H
+#define MOEQ_H
+
+#include <stddef.h>
+#include <stdint.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+#define MOEQ_ABI_VERSION 1
+#define MOEQ_MAX_K 8      /* largest routed top-K */
+#define MOEQ_MAX_B 64     /* largest token batch per call */
+
+typedef enum moe_status {
+  MOE_OK = 0,
+  MOE_ERR_INVALID_ARG = 1, /* null pointer, bad size or shape */
+  MOE_ERR_ALIGN = 2,       /* a device pointer is not 16-byte aligned */
+  MOE_ERR_UNSUPPORTED = 3, /* bits/group/shape outside the supported set */
+  MOE_ERR_CUDA = 4,        /* a CUDA launch or copy failed */
+  MOE_ERR_INDEX = 5,       /* device: an expert index was outside [0, E) */
+  MOE_ERR_TIMEOUT = 6,     /* device: a bounded wait gave up */
+  MOE_ERR_WORKSPACE = 7,   /* workspace missing or smaller than required */
+  MOE_ERR_RANGE = 8        /* device: a code did not fit in its bit width */
+} moe_status;
+
+/*
+ * One MoE layer's resident weights (all pointers are device memory).
+ *
+ * Expert record (expert-major: each expert is one contiguous block, as in
+ * LOOM's layout), for `bits` in {2, 4} and group size `group`:
+ *   [gate codes  I x H][up codes  I x H][down codes  H x I]
+ *   [gate table  I x H/group][up table  I x H/group][down table  H x I/group]
+ * A code matrix [rows x cols] is row-major; in each row, element c sits in
+ * byte floor(c*bits/8) at bit offset (c*bits) mod 8, lowest bits first.
+ * A table entry is the bf16 pair (scale, bias) of one (row, group), scale
+ * first; the dequantised weight is w = q*scale + bias with q unsigned.
+ * Record size: moe_expert_bytes(H, I, bits, group); byte offsets of the six
+ * parts: moe_expert_offsets. At H=4096, I=1024, 4-bit, group 64 a record is
+ * 7,077,888 bytes (6.75 MiB), the per-expert size the Flash-MoE page gives.
+ */
+typedef struct moe_layer_q {
+  int H;           /* hidden size; H*bits/8 and I*bits/8 multiples of 16 */
+  int I;           /* expert intermediate size */
+  int E;           /* routed experts */
+  int K;           /* routed experts per token, 1..MOEQ_MAX_K, K <= E */
+  int group;       /* 32, 64 or 128; divides H and I */
+  int bits_routed; /* 2 or 4 */
+  int bits_shared; /* 2 or 4 */
+  const void* experts;       /* E routed records, back to back */
+  const void* shared;        /* 1 shared-expert record (bits_shared) */
+  const void* router_w;      /* bf16 [E, H], row-major */
+  const void* shared_gate_w; /* bf16 [H], or NULL: shared expert weight 1 */
+} moe_layer_q;
+
+/* Bytes of one expert record (see moe_layer_q); 0 for unsupported args. */
+size_t moe_expert_bytes(int H, int I, int bits, int group);
+
+/* Byte offsets within one expert record of: off[0] gate codes, off[1] up
+ * codes, off[2] down codes, off[3] gate table, off[4] up table, off[5] down
+ * table. */
+moe_status moe_expert_offsets(int H, int I, int bits, int group, size_t off[6]);
+
+/* Workspace bytes for calls on up to B tokens of this layer shape. */
+size_t moe_workspace_bytes(int B, int K, int H, int I, int E);
+
+/* Zero a workspace (asynchronous cudaMemsetAsync on `stream`). */
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_pack_q -- pack one code matrix into the layout of moe_layer_q.
+ *   codes      u8 [rows, cols], one code per byte, values < 2^bits
+ *   scale_bf16 bf16 [rows, cols/group]
+ *   bias_bf16  bf16 [rows, cols/group]
+ *   packed_out u8 [rows, cols*bits/8]
+ *   sb_out     bf16 [rows, cols/group, 2]  (scale, bias) pairs
+ *   ws         optional workspace (NULL allowed): a code >= 2^bits sets
+ *              MOE_ERR_RANGE there; its low `bits` bits are packed.
+ * bits in {2,4}; group in {32,64,128}; cols % group == 0; cols*bits/8 a
+ * multiple of 16. The layout is the affine form of the Flash-MoE page
+ * ("Kernel dequant toi uu FMA": (nibble*scale+bias)), 4- and 2-bit widths as
+ * in its "Metal Compute Shaders" section.
+ */
+moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* bias_bf16,
+                      int rows, int cols, int bits, int group,
+                      void* packed_out, void* sb_out, void* ws, void* stream);
+
+/*
+ * moe_router_topk -- router GEMV + softmax + top-K for B tokens.
+ *   x_bf16        bf16 [B, H]
+ *   router_w_bf16 bf16 [E, H]
+ *   forced_idx    NULL, or int32 [B, K]: use these experts instead of the
+ *                 top-K (their weights still come from the softmax)
+ *   idx_out       int32 [B, K]: experts by descending logit, ties to the
+ *                 lower index
+ *   w_out         fp32 [B, K]: softmax probability over all E of each pick;
+ *                 divided by their sum when renorm != 0
+ *   logits_out    fp32 [B, E] or NULL
+ * Logits accumulate in fp32 (bf16 products are exact in fp32).
+ * Source: "Kien truc mo hinh" (512 experts, K active per token).
+ */
+moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B, int H, int E, int K,
+                           int renorm, const int32_t* forced_idx, int32_t* idx_out, float* w_out,
+                           float* logits_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_expert_ffn_q -- gate/up dequant mat-vecs, SwiGLU and down dequant
+ * mat-vec for the K routed experts idx[b, :] and the shared expert of each
+ * token, in one call.
+ *   x_bf16 bf16 [B, H]; idx int32 [B, K]
+ *   y_out  fp32 [B, K+1, H]: slot k < K is expert idx[b,k]'s output, slot K
+ *          the shared expert's (unweighted)
+ * Per group of G inputs a row contributes scale*sum(q*x) + bias*sum(x): the
+ * group-summed form of fma(q, scale*x, bias*x) (Flash-MoE page, section
+ * "Kernel dequant toi uu FMA"); products are exact and accumulate in fp32.
+ * The down projection reads h rounded to fp16 under a per-expert power-of-
+ * two scale. An index outside [0,E) sets MOE_ERR_INDEX and zeroes that slot.
+ */
+moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx,
+                            float* y_out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * moe_combine_residual -- out[b] = r[b] + sum_k w[b,k] y[b,k] + gamma_b y[b,K]
+ *   y fp32 [B, K+1, H]; w fp32 [B, K]; x_bf16 bf16 [B, H]
+ *   resid_in   fp32 [B, H], or NULL: r = x (bf16 widened)
+ *   gamma_b    1 when L->shared_gate_w is NULL, else sigmoid(w_sg . x[b])
+ *   resid_out  fp32 [B, H] (may alias resid_in)
+ *   xnorm_bf16_out  bf16 [B, H] or NULL: RMSNorm(out[b]) with unit weight
+ *              and epsilon eps, rounded to nearest-even bf16
+ * Source: "Metal Compute Shaders" (MoE combine + residual + gate, RMS norm)
+ * and "Deferred GPU Expert Compute" (combine + norm + residual feed the next
+ * layer).
+ */
+moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const float* w, const void* x_bf16,
+                                const float* resid_in, int B, float* resid_out, void* xnorm_bf16_out,
+                                float eps, void* stream);
+
+/* Read (and clear) the workspace error word. Synchronises `stream`.
+ * Returns MOE_OK, MOE_ERR_INDEX, MOE_ERR_RANGE, MOE_ERR_TIMEOUT, or
+ * MOE_ERR_CUDA if the copy itself failed. */
+moe_status moe_get_device_error(void* ws, void* stream);
+
+const char* moe_status_str(moe_status s);
+int moe_abi_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOEQ_H */

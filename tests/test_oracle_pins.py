@@ -1,0 +1,339 @@
+"""Pins of the oracle against what the pages and the mathematics fix.
+
+Each test checks one oracle function against something other than itself:
+the pages' numbers (6.75 MB per expert), hand-derived byte images, closed
+forms, special cases that reduce to a textbook or library routine, and brute
+force. A plausible mistake (a dropped bias term, a wrong group index, a
+transposed operand, a swapped gate/up, a reversed sort or tie-break) fails at
+least one of them. All CPU-only.
+"""
+import math
+import os
+
+import numpy as np
+import pytest
+
+GOLDEN = os.path.join(os.path.dirname(os.path.abspath(__file__)), "golden")
+
+
+def _rows(name):
+    with open(os.path.join(GOLDEN, name)) as f:
+        for line in f:
+            line = line.strip()
+            if line and not line.startswith("#"):
+                yield line
+
+
+def _bf16(v):
+    """bf16 bits of a float that is exactly representable in bf16."""
+    b = np.float32(v).view(np.uint32)
+    assert (b & 0xFFFF) == 0, v
+    return np.uint16(b >> 16)
+
+
+def _rand_layer(rng, rows, cols, bits, group):
+    codes = rng.integers(0, 1 << bits, size=(rows, cols), dtype=np.uint8)
+    # scale/bias as bf16 by truncating random fp32 bit patterns
+    s32 = rng.uniform(0.005, 0.02, size=(rows, cols // group)).astype(np.float32).view(np.uint32)
+    b32 = rng.normal(0, 0.01, size=(rows, cols // group)).astype(np.float32).view(np.uint32)
+    scale = (s32 >> 16).astype(np.uint16)
+    bias = (b32 >> 16).astype(np.uint16)
+    return codes, scale, bias
+
+
+def _f64(bits):
+    return (np.asarray(bits, dtype=np.uint16).astype(np.uint32) << 16).view(np.float32).astype(np.float64)
+
+
+# ---- sizes (the page's 6.75 MB per expert) ----------------------------------
+
+def test_expert_bytes_match_page(ref):
+    for line in _rows("expert_bytes.txt"):
+        H, I, bits, group, nbytes = map(int, line.split())
+        assert ref.expert_bytes(H, I, bits, group) == nbytes
+    assert ref.expert_bytes(4096, 1024, 4, 64) == int(6.75 * 2 ** 20)
+
+
+# ---- bf16 conversions -------------------------------------------------------
+
+def test_bf16_widening_exact(ref):
+    assert ref.bf16_to_f64(0x3F80)[0] == 1.0
+    assert ref.bf16_to_f64(0x4049)[0] == 3.140625
+    assert ref.bf16_to_f64(0xC2F7)[0] == -123.5
+    assert ref.bf16_to_f64(0x0001)[0] == 2.0 ** -133
+
+
+def test_bf16_rounding_nearest_even(ref):
+    cases = {
+        1.0 + 2 ** -8: 0x3F80,               # tie, even stays 1.0
+        1.0 + 3 * 2 ** -8: 0x3F82,           # tie, rounds to even 1+2^-6
+        1.0 + 2 ** -8 + 2 ** -20: 0x3F81,    # above the tie
+        -2.0: 0xC000,
+        2.0 ** -133: 0x0001,                 # smallest subnormal
+        1.5 * 2.0 ** -133: 0x0002,           # subnormal tie to even
+        2.0 ** -134: 0x0000,                 # tie to even zero
+        1e39: 0x7F80,                        # overflow
+        0.0: 0x0000,
+    }
+    for v, bits in cases.items():
+        assert int(ref.f64_to_bf16(v)[0]) == bits, (v, hex(bits))
+
+
+# ---- packing ----------------------------------------------------------------
+
+def test_pack_golden_bytes(ref):
+    n = 0
+    for line in _rows("pack_bytes.txt"):
+        bits, group, codes, expect = [t.strip() for t in line.split("|")]
+        bits, group = int(bits), int(group)
+        c = np.array([[int(ch, 16) for ch in codes]], dtype=np.uint8)
+        ng = c.shape[1] // group
+        packed, sb = ref.pack(c, np.full((1, ng), 0x3F80, np.uint16), np.full((1, ng), 0xBF80, np.uint16),
+                              bits, group)
+        assert [int(v) for v in packed[0]] == [int(t, 16) for t in expect.split()]
+        assert sb.shape == (1, ng, 2)
+        assert (sb[..., 0] == 0x3F80).all() and (sb[..., 1] == 0xBF80).all()  # scale first
+        n += 1
+    assert n >= 4
+
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (4, 64), (2, 32), (2, 64), (4, 128)])
+def test_pack_is_little_endian_bitstring(ref, bits, group):
+    """Independent reading of the layout: a packed row is the row's codes
+    written as one little-endian integer, sum_c q_c * 2^(c*bits)."""
+    rng = np.random.default_rng(bits * 1000 + group)
+    codes, scale, bias = _rand_layer(rng, 3, 256, bits, group)
+    packed, sb = ref.pack(codes, scale, bias, bits, group)
+    for r in range(3):
+        big = sum(int(q) << (c * bits) for c, q in enumerate(codes[r]))
+        assert bytes(packed[r]) == big.to_bytes(256 * bits // 8, "little")
+        assert (sb[r, :, 0] == scale[r]).all() and (sb[r, :, 1] == bias[r]).all()
+
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (2, 64)])
+def test_pack_roundtrip_and_range(ref, bits, group):
+    rng = np.random.default_rng(7)
+    codes, scale, bias = _rand_layer(rng, 5, 128, bits, group)
+    packed, sb = ref.pack(codes, scale, bias, bits, group)
+    c2, s2, b2 = ref.unpack(packed, sb, 5, 128, bits, group)
+    assert (c2 == codes).all() and (s2 == scale).all() and (b2 == bias).all()
+    codes[2, 3] = 1 << bits
+    with pytest.raises(ValueError):
+        ref.pack(codes, scale, bias, bits, group)
+
+
+# ---- dequant mat-vec --------------------------------------------------------
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (4, 64), (2, 64)])
+def test_gemv_fma_rearrangement_identity(ref, bits, group):
+    """The Flash-MoE page's identity: (q*s+b)*x == fma(q, s*x, b*x), and its
+    per-group sum s*sum(qx) + b*sum(x): three forms agree to 1e-12."""
+    rng = np.random.default_rng(11)
+    codes, scale, bias = _rand_layer(rng, 64, 512, bits, group)
+    x = rng.normal(size=512)
+    y0 = ref.dequant_gemv(codes, scale, bias, group, x)
+    y1 = ref.dequant_gemv_fma(codes, scale, bias, group, x)
+    y2 = ref.dequant_gemv_grouped(codes, scale, bias, group, x)
+    tol = 1e-12 * np.abs(y0).max()
+    assert np.abs(y1 - y0).max() <= tol and np.abs(y2 - y0).max() <= tol
+
+
+def test_gemv_constant_codes_closed_form(ref):
+    """All codes c, per-row constant scale and bias: y_r = (c*s_r + b_r) * sum(x)."""
+    rows, cols, group = 6, 256, 64
+    rng = np.random.default_rng(3)
+    x = rng.normal(size=cols)
+    svals = [0.0078125, 0.015625, 0.01171875, 0.009765625, 0.005859375, 0.0185546875]
+    bvals = [0.25, -0.5, 0.0, 0.125, -0.0625, 1.0]
+    for c in (0, 5, 15):
+        codes = np.full((rows, cols), c, np.uint8)
+        scale = np.array([[_bf16(s)] * (cols // group) for s in svals], np.uint16)
+        bias = np.array([[_bf16(b)] * (cols // group) for b in bvals], np.uint16)
+        y = ref.dequant_gemv(codes, scale, bias, group, x)
+        expect = np.array([(c * s + b) for s, b in zip(svals, bvals)]) * math.fsum(x)
+        assert np.allclose(y, expect, rtol=1e-12, atol=1e-12)
+
+
+def test_gemv_zero_codes_leave_bias_term(ref):
+    """q = 0: y_r = sum_g b_{r,g} * sum_{j in g} x_j (catches a dropped or
+    misindexed bias term)."""
+    rng = np.random.default_rng(5)
+    codes, scale, bias = _rand_layer(rng, 8, 256, 4, 32)
+    codes[:] = 0
+    x = rng.normal(size=256)
+    y = ref.dequant_gemv(codes, scale, bias, 32, x)
+    expect = (_f64(bias) * x.reshape(8, 32).sum(axis=1)[None, :]).sum(axis=1)
+    assert np.allclose(y, expect, rtol=1e-12, atol=1e-14)
+
+
+@pytest.mark.parametrize("bits,group", [(4, 32), (2, 64)])
+def test_gemv_one_hot_recovers_dequantised_column(ref, bits, group):
+    """x = e_j gives column j dequantised, q[r,j]*s[r,j//G] + b[r,j//G], exactly
+    (catches a transposed operand or a wrong group index)."""
+    rng = np.random.default_rng(9)
+    rows, cols = 16, 256
+    codes, scale, bias = _rand_layer(rng, rows, cols, bits, group)
+    for j in (0, 1, group - 1, group, cols - 1, 77):
+        x = np.zeros(cols)
+        x[j] = 1.0
+        y = ref.dequant_gemv(codes, scale, bias, group, x)
+        expect = codes[:, j].astype(np.float64) * _f64(scale[:, j // group]) + _f64(bias[:, j // group])
+        assert (y == expect).all()
+
+
+def test_gemv_matches_dense_library_matmul(ref):
+    """Against numpy's dense float64 mat-vec of the explicitly dequantised matrix."""
+    rng = np.random.default_rng(13)
+    codes, scale, bias = _rand_layer(rng, 40, 320, 4, 32)
+    x = rng.normal(size=320)
+    W = codes.astype(np.float64) * np.repeat(_f64(scale), 32, axis=1) + np.repeat(_f64(bias), 32, axis=1)
+    assert np.allclose(ref.dequant_gemv(codes, scale, bias, 32, x), W @ x, rtol=1e-12, atol=1e-12)
+
+
+# ---- router -----------------------------------------------------------------
+
+def test_router_one_hot_rows(ref):
+    """W_r row e = c_e * unit vector at pi(e): logit_e = c_e * x[pi(e)] exactly."""
+    E, H = 8, 64
+    rng = np.random.default_rng(1)
+    x = np.array([_bf16(v) for v in (rng.integers(-64, 64, size=H) / 8.0)], np.uint16)
+    perm = rng.permutation(H)[:E]
+    cs = [0.5, -1.0, 2.0, 0.25, 1.5, -0.75, 3.0, 1.0]
+    W = np.zeros((E, H), np.uint16)
+    for e in range(E):
+        W[e, perm[e]] = _bf16(cs[e])
+    logits = ref.router_logits(x, W)
+    assert (logits == np.array([cs[e] * _f64(x[perm[e]]) for e in range(E)])).all()
+
+
+def _brute_topk(logits, K):
+    order = sorted(range(len(logits)), key=lambda e: (-logits[e], e))
+    return order[:K]
+
+
+def _softmax_closed(logits):
+    m = max(logits)
+    ex = [math.exp(v - m) for v in logits]
+    z = math.fsum(ex)
+    return [v / z for v in ex]
+
+
+@pytest.mark.parametrize("E,K", [(8, 2), (512, 4), (64, 8)])
+def test_topk_matches_brute_force_sort(ref, E, K):
+    rng = np.random.default_rng(E + K)
+    for trial in range(20):
+        logits = rng.normal(scale=1.28, size=E)
+        if trial % 3 == 0:  # exact ties must go to the lower index
+            logits[rng.integers(E)] = logits.max()
+            logits[rng.integers(E)] = logits.max()
+        idx, w = ref.topk(logits, K)
+        assert list(idx) == _brute_topk(list(logits), K)
+        p = _softmax_closed(list(logits))
+        assert np.allclose(w, [p[i] for i in idx], rtol=1e-12)
+        idx_r, w_r = ref.topk(logits, K, renorm=True)
+        assert list(idx_r) == list(idx)
+        assert np.allclose(w_r, np.array([p[i] for i in idx]) / math.fsum(p[i] for i in idx), rtol=1e-12)
+
+
+def test_topk_ties_prefer_lower_index(ref):
+    logits = np.array([1.0, 3.0, 3.0, 0.5, 3.0, 2.0])
+    idx, _ = ref.topk(logits, 4)
+    assert list(idx) == [1, 2, 4, 5]
+
+
+def test_topk_forced_indices(ref):
+    logits = np.array([0.1, 0.4, -0.3, 2.0, 1.0])
+    idx, w = ref.topk(logits, 2, forced=np.array([2, 0], np.int32))
+    p = _softmax_closed(list(logits))
+    assert list(idx) == [2, 0] and np.allclose(w, [p[2], p[0]], rtol=1e-14)
+    with pytest.raises(ValueError):
+        ref.topk(logits, 2, forced=np.array([5, 0], np.int32))
+
+
+def test_softmax_two_expert_closed_form(ref):
+    for a, b in ((0.0, 0.0), (1.0, -2.0), (30.0, 29.5), (-5.0, 3.0)):
+        p = ref.softmax(np.array([a, b]))
+        assert abs(p[0] - 1.0 / (1.0 + math.exp(b - a))) < 1e-15
+        assert abs(p.sum() - 1.0) < 1e-15
+
+
+# ---- SwiGLU -----------------------------------------------------------------
+
+def test_silu_closed_forms(ref):
+    e = math.e
+    assert ref.silu(0.0) == 0.0
+    assert abs(ref.silu(1.0) - e / (e + 1.0)) < 1e-15
+    assert abs(ref.silu(-1.0) - (-1.0 / (e + 1.0))) < 1e-15
+    assert abs(ref.silu(2.0) - 2.0 * e * e / (e * e + 1.0)) < 1e-15
+    for z in (-7.5, -0.3, 0.7, 4.0, 12.0):  # z*sigmoid(z) == z*(1+tanh(z/2))/2
+        assert abs(ref.silu(z) - z * (1.0 + math.tanh(z / 2.0)) / 2.0) < 1e-14 * max(1.0, abs(z))
+    assert abs(ref.silu(40.0) - 40.0) < 1e-12 and abs(ref.silu(-40.0)) < 1e-15
+
+
+def test_swiglu_gate_is_the_silu_operand(ref):
+    h = ref.swiglu(np.array([1.0, 2.0]), np.array([2.0, 1.0]))
+    e = math.e
+    assert abs(h[0] - 2.0 * e / (e + 1.0)) < 1e-15      # silu(g=1) * u=2
+    assert abs(h[1] - 2.0 * e * e / (e * e + 1.0)) < 1e-15
+
+
+# ---- expert FFN --------------------------------------------------------------
+
+def test_expert_ffn_constant_closed_form(ref):
+    """Constant codes/scales per matrix: g_i = (cg*s+b)*sum(x), u_i =
+    (cu*s+b)*sum(x), h_i = silu(g)*u, y = (cd*s+b)*I*h. Distinct gate and up
+    constants catch a swap of the two."""
+    H, I, G = 128, 64, 32
+    rng = np.random.default_rng(2)
+    x = rng.normal(size=H) / 8.0
+    s, b = 0.0078125, 0.015625
+
+    def mat(rows, cols, c, bb):
+        return (np.full((rows, cols), c, np.uint8), np.full((rows, cols // G), _bf16(s), np.uint16),
+                np.full((rows, cols // G), _bf16(bb), np.uint16))
+
+    gate, up, down = mat(I, H, 3, b), mat(I, H, 11, -b), mat(H, I, 6, b)
+    y = ref.expert_ffn(H, I, G, gate, up, down, x)
+    sx = math.fsum(x)
+    g = (3 * s + b) * sx
+    u = (11 * s - b) * sx
+    hval = g * (1.0 + math.tanh(g / 2.0)) / 2.0 * u
+    expect = (6 * s + b) * I * hval
+    assert np.allclose(y, expect, rtol=1e-12)
+
+
+# ---- combine, gate, norm ----------------------------------------------------
+
+def test_combine_one_hot_weight_selects_expert(ref):
+    rng = np.random.default_rng(4)
+    K, H = 4, 32
+    y = rng.normal(size=(K + 1, H))
+    for k in range(K):
+        w = np.zeros(K)
+        w[k] = 1.0
+        assert (ref.combine(y, w, 0.0, np.zeros(H)) == y[k]).all()
+    assert (ref.combine(y, np.zeros(K), 1.0, np.zeros(H)) == y[K]).all()
+    r = rng.normal(size=H)
+    assert (ref.combine(np.zeros((K + 1, H)), np.ones(K), 1.0, r) == r).all()
+
+
+def test_shared_gate_is_sigmoid(ref):
+    H = 16
+    x = np.array([_bf16(1.0)] * H, np.uint16)
+    assert ref.shared_gate(np.zeros(H, np.uint16), x) == 0.5
+    wsg = np.zeros(H, np.uint16)
+    wsg[3] = _bf16(2.0)
+    assert abs(ref.shared_gate(wsg, x) - 1.0 / (1.0 + math.exp(-2.0))) < 1e-15
+
+
+def test_rmsnorm_closed_forms(ref):
+    out = ref.rmsnorm(np.array([3.0, 4.0]), 0.0)
+    assert np.allclose(out, [3.0 / math.sqrt(12.5), 4.0 / math.sqrt(12.5)], rtol=1e-15)
+    c, eps = -0.5, 1e-6
+    out = ref.rmsnorm(np.full(64, c), eps)
+    assert np.allclose(out, c / math.sqrt(c * c + eps), rtol=1e-15)
+    xb = ref.rmsnorm_bf16(np.array([3.0, -4.0, 0.0, 5.0]), 0.0)
+    # rms = sqrt(50/4); 3/3.5355 = 0.8485 -> bf16 0x3F59, etc.
+    assert [int(v) for v in xb] == [int(ref.f64_to_bf16(v)[0]) for v in (3 / math.sqrt(12.5), -4 / math.sqrt(12.5),
+                                                                          0.0, 5 / math.sqrt(12.5))]
+    assert int(xb[2]) == 0 and int(xb[1]) & 0x8000
