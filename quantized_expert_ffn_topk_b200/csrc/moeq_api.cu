@@ -1,0 +1,312 @@
+// moeq_api.cu -- host side of libmoeq.so: argument checks, launch shapes and
+// the extern "C" entry points declared in include/moeq.h.
+#include <cuda_runtime.h>
+
+#include <algorithm>
+#include <cstring>
+
+#include "combine.cuh"
+#include "common.cuh"
+#include "ffn.cuh"
+#include "pack.cuh"
+#include "router.cuh"
+
+namespace moeq {
+namespace {
+
+inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+inline bool bits_ok(int bits) { return bits == 2 || bits == 4; }
+inline bool group_ok(int g) { return g == 32 || g == 64 || g == 128; }
+
+// A row of `cols` codes must be whole 16-byte chunks and whole groups.
+inline bool cols_ok(int cols, int bits, int group) {
+  return cols > 0 && cols % group == 0 && ((int64_t)cols * bits) % 128 == 0;
+}
+
+inline moe_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? MOE_OK : MOE_ERR_CUDA;
+}
+
+int g_num_sms = 0;
+inline int num_sms() {
+  if (g_num_sms == 0) {
+    int dev = 0, n = 0;
+    if (cudaGetDevice(&dev) != cudaSuccess || cudaDeviceGetAttribute(&n, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess)
+      n = 148;
+    g_num_sms = n > 0 ? n : 148;
+  }
+  return g_num_sms;
+}
+
+// Launch with programmatic dependent launch allowed, so a kernel's prologue
+// may overlap the tail of the previous kernel on the stream.
+template <typename... KArgs, typename... Args>
+moe_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t s, Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = s;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  cudaError_t e = cudaLaunchKernelEx(&cfg, kern, std::forward<Args>(args)...);
+  if (e != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+template <typename K>
+moe_status ensure_smem(K kern, size_t bytes) {
+  if (bytes <= 48 * 1024) return MOE_OK;
+  if (bytes > 227 * 1024) return MOE_ERR_UNSUPPORTED;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+// Workspace layout: [control 256 B][logits B*E fp32][h B*(K+1)*I fp32]
+struct WsLayout {
+  size_t logits, h, total;
+};
+inline WsLayout ws_layout(int B, int K, int H, int I, int E) {
+  (void)H;
+  WsLayout l{};
+  size_t o = sizeof(WsCtrl);
+  l.logits = o;
+  o += align_up((size_t)B * E * sizeof(float));
+  l.h = o;
+  o += align_up((size_t)B * (K + 1) * I * sizeof(float));
+  l.total = o;
+  return l;
+}
+
+inline void expert_offsets(int H, int I, int bits, int group, size_t off[6]) {
+  const size_t hi = (size_t)H * I;
+  const size_t cb = hi * bits / 8;          // one matrix of codes
+  const size_t tb = hi / group * 4;         // one (scale, bias) table
+  off[0] = 0;
+  off[1] = cb;
+  off[2] = 2 * cb;
+  off[3] = 3 * cb;
+  off[4] = 3 * cb + tb;
+  off[5] = 3 * cb + 2 * tb;
+}
+
+moe_status check_layer(const moe_layer_q* L) {
+  if (!L) return MOE_ERR_INVALID_ARG;
+  if (L->H <= 0 || L->I <= 0 || L->E <= 0 || L->K <= 0) return MOE_ERR_INVALID_ARG;
+  if (L->K > MOEQ_MAX_K || L->K > L->E) return MOE_ERR_INVALID_ARG;
+  if (!bits_ok(L->bits_routed) || !bits_ok(L->bits_shared) || !group_ok(L->group)) return MOE_ERR_UNSUPPORTED;
+  for (int bits : {L->bits_routed, L->bits_shared})
+    if (!cols_ok(L->H, bits, L->group) || !cols_ok(L->I, bits, L->group)) return MOE_ERR_UNSUPPORTED;
+  if (!L->experts || !L->shared || !L->router_w) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(L->experts) || !aligned16(L->shared) || !aligned16(L->router_w)) return MOE_ERR_ALIGN;
+  if (L->shared_gate_w && !aligned16(L->shared_gate_w)) return MOE_ERR_ALIGN;
+  return MOE_OK;
+}
+
+}  // namespace
+}  // namespace moeq
+
+using namespace moeq;
+
+extern "C" {
+
+int moe_abi_version(void) { return MOEQ_ABI_VERSION; }
+
+const char* moe_status_str(moe_status s) {
+  switch (s) {
+    case MOE_OK: return "ok";
+    case MOE_ERR_INVALID_ARG: return "invalid argument";
+    case MOE_ERR_ALIGN: return "device pointer not 16-byte aligned";
+    case MOE_ERR_UNSUPPORTED: return "unsupported bits/group/shape";
+    case MOE_ERR_CUDA: return "CUDA error";
+    case MOE_ERR_INDEX: return "expert index out of range (device)";
+    case MOE_ERR_TIMEOUT: return "bounded wait timed out (device)";
+    case MOE_ERR_WORKSPACE: return "workspace missing or too small";
+    case MOE_ERR_RANGE: return "code does not fit its bit width (device)";
+  }
+  return "unknown status";
+}
+
+size_t moe_expert_bytes(int H, int I, int bits, int group) {
+  if (H <= 0 || I <= 0 || !bits_ok(bits) || !group_ok(group)) return 0;
+  if (!cols_ok(H, bits, group) || !cols_ok(I, bits, group)) return 0;
+  const size_t hi = 3 * (size_t)H * I;
+  return hi * bits / 8 + hi / group * 4;
+}
+
+moe_status moe_expert_offsets(int H, int I, int bits, int group, size_t off[6]) {
+  if (!off) return MOE_ERR_INVALID_ARG;
+  if (moe_expert_bytes(H, I, bits, group) == 0) return MOE_ERR_UNSUPPORTED;
+  expert_offsets(H, I, bits, group, off);
+  return MOE_OK;
+}
+
+size_t moe_workspace_bytes(int B, int K, int H, int I, int E) {
+  if (B <= 0 || K <= 0 || H <= 0 || I <= 0 || E <= 0) return 0;
+  return ws_layout(B, K, H, I, E).total;
+}
+
+moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
+  if (!ws || ws_bytes < sizeof(WsCtrl)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_ALIGN;
+  if (cudaMemsetAsync(ws, 0, ws_bytes, (cudaStream_t)stream) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}
+
+moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* bias_bf16, int rows, int cols,
+                      int bits, int group, void* packed_out, void* sb_out, void* ws, void* stream) {
+  if (!codes || !scale_bf16 || !bias_bf16 || !packed_out || !sb_out) return MOE_ERR_INVALID_ARG;
+  if (rows < 0) return MOE_ERR_INVALID_ARG;
+  if (!bits_ok(bits) || !group_ok(group) || !cols_ok(cols, bits, group)) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(codes) || !aligned16(packed_out) || !aligned16(sb_out) || !aligned16(scale_bf16) ||
+      !aligned16(bias_bf16) || (ws && !aligned16(ws)))
+    return MOE_ERR_ALIGN;
+  if (rows == 0) return MOE_OK;
+  cudaStream_t s = (cudaStream_t)stream;
+  const int64_t nchunks = (int64_t)rows * cols * bits / 128;
+  const int64_t nsb = (int64_t)rows * (cols / group);
+  const unsigned maxg = (unsigned)num_sms() * 8;
+  unsigned g1 = (unsigned)std::min<int64_t>((nchunks + 255) / 256, maxg);
+  unsigned g2 = (unsigned)std::min<int64_t>((nsb + 255) / 256, maxg);
+  WsCtrl* ctrl = reinterpret_cast<WsCtrl*>(ws);
+  if (bits == 4)
+    k_pack_codes<4><<<g1, 256, 0, s>>>(codes, nchunks, reinterpret_cast<uint8_t*>(packed_out), ctrl);
+  else
+    k_pack_codes<2><<<g1, 256, 0, s>>>(codes, nchunks, reinterpret_cast<uint8_t*>(packed_out), ctrl);
+  k_pack_sb<<<g2, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(scale_bf16), reinterpret_cast<const uint16_t*>(bias_bf16),
+                               nsb, reinterpret_cast<uint32_t*>(sb_out));
+  return launch_status();
+}
+
+moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B, int H, int E, int K, int renorm,
+                           const int32_t* forced_idx, int32_t* idx_out, float* w_out, float* logits_out, void* ws,
+                           size_t ws_bytes, void* stream) {
+  if (!x_bf16 || !router_w_bf16 || !idx_out || !w_out) return MOE_ERR_INVALID_ARG;
+  if (B <= 0 || B > MOEQ_MAX_B || H <= 0 || E <= 0 || K <= 0 || K > MOEQ_MAX_K || K > E) return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_workspace_bytes(B, K, H, 32, E)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(x_bf16) || !aligned16(router_w_bf16) || !aligned16(ws)) return MOE_ERR_ALIGN;
+  const size_t smem = (size_t)std::min(B, kRouterTokTile) * H * 2;
+  if (ensure_smem(k_router_topk, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;
+  RouterParams p{};
+  p.x = reinterpret_cast<const uint16_t*>(x_bf16);
+  p.wr = reinterpret_cast<const uint16_t*>(router_w_bf16);
+  p.forced = forced_idx;
+  p.idx = idx_out;
+  p.w = w_out;
+  WsLayout wl = ws_layout(B, K, H, 32, E);
+  p.logits = logits_out ? logits_out : reinterpret_cast<float*>((char*)ws + wl.logits);
+  p.ctrl = reinterpret_cast<WsCtrl*>(ws);
+  p.B = B;
+  p.H = H;
+  p.E = E;
+  p.K = K;
+  p.renorm = renorm;
+  const int ctas = (E + kRouterWarps - 1) / kRouterWarps;
+  return launch_pdl(k_router_topk, dim3(ctas), dim3(kRouterWarps * 32), smem, (cudaStream_t)stream, p);
+}
+
+moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx, float* y_out,
+                            void* ws, size_t ws_bytes, void* stream) {
+  moe_status st = check_layer(L);
+  if (st != MOE_OK) return st;
+  if (!x_bf16 || !idx || !y_out) return MOE_ERR_INVALID_ARG;
+  if (B <= 0 || B > MOEQ_MAX_B) return MOE_ERR_INVALID_ARG;
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_workspace_bytes(B, L->K, L->H, L->I, L->E)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(x_bf16) || !aligned16(y_out) || !aligned16(ws) || !aligned16(idx)) return MOE_ERR_ALIGN;
+  FfnParams p{};
+  p.experts = reinterpret_cast<const uint8_t*>(L->experts);
+  p.shared = reinterpret_cast<const uint8_t*>(L->shared);
+  p.rec_r = moe_expert_bytes(L->H, L->I, L->bits_routed, L->group);
+  p.rec_s = moe_expert_bytes(L->H, L->I, L->bits_shared, L->group);
+  expert_offsets(L->H, L->I, L->bits_routed, L->group, p.off_r);
+  expert_offsets(L->H, L->I, L->bits_shared, L->group, p.off_s);
+  p.x = reinterpret_cast<const uint16_t*>(x_bf16);
+  p.idx = idx;
+  WsLayout wl = ws_layout(B, L->K, L->H, L->I, L->E);
+  p.h = reinterpret_cast<float*>((char*)ws + wl.h);
+  p.y = y_out;
+  p.ctrl = reinterpret_cast<WsCtrl*>(ws);
+  p.H = L->H;
+  p.I = L->I;
+  p.E = L->E;
+  p.K = L->K;
+  p.G = L->group;
+  p.bits_r = L->bits_routed;
+  p.bits_s = L->bits_shared;
+  p.B = B;
+  const bool need4 = p.bits_r == 4 || p.bits_s == 4, need2 = p.bits_r == 2 || p.bits_s == 2;
+  const GuSmem gs = gu_smem_plan(p.H, need4, need2);
+  const DnSmem ds = dn_smem_plan(p.I, p.K);
+  if (ensure_smem(k_gate_up, gs.bytes) != MOE_OK || ensure_smem(k_down, ds.bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
+
+  const int gu_units = (p.K + 1) * p.I, dn_units = (p.K + 1) * p.H;
+  p.units_per_cta_gu = kFfnWarps;
+  p.units_per_cta_dn = kFfnWarps * 4;
+  const int gu_ctas = (gu_units + p.units_per_cta_gu - 1) / p.units_per_cta_gu;
+  const int dn_ctas = (dn_units + p.units_per_cta_dn - 1) / p.units_per_cta_dn;
+  cudaStream_t s = (cudaStream_t)stream;
+  st = launch_pdl(k_gate_up, dim3(gu_ctas, B), dim3(kFfnWarps * 32), gs.bytes, s, p);
+  if (st != MOE_OK) return st;
+  return launch_pdl(k_down, dim3(dn_ctas, B), dim3(kFfnWarps * 32), ds.bytes, s, p);
+}
+
+moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const float* w, const void* x_bf16,
+                                const float* resid_in, int B, float* resid_out, void* xnorm_bf16_out, float eps,
+                                void* stream) {
+  if (!L || !y || !w || !x_bf16 || !resid_out) return MOE_ERR_INVALID_ARG;
+  if (L->H <= 0 || L->K <= 0 || L->K > MOEQ_MAX_K || B <= 0 || B > MOEQ_MAX_B) return MOE_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(y) || !aligned16(x_bf16) || !aligned16(resid_out) || (resid_in && !aligned16(resid_in)) ||
+      (xnorm_bf16_out && !aligned16(xnorm_bf16_out)) || (L->shared_gate_w && !aligned16(L->shared_gate_w)))
+    return MOE_ERR_ALIGN;
+  CombineParams p{};
+  p.y = y;
+  p.w = w;
+  p.x = reinterpret_cast<const uint16_t*>(x_bf16);
+  p.resid_in = resid_in;
+  p.gate_w = reinterpret_cast<const uint16_t*>(L->shared_gate_w);
+  p.resid_out = resid_out;
+  p.xnorm = reinterpret_cast<uint16_t*>(xnorm_bf16_out);
+  p.B = B;
+  p.H = L->H;
+  p.K = L->K;
+  p.eps = eps;
+  return launch_pdl(k_combine, dim3(B), dim3(kCombineThreads), 0, (cudaStream_t)stream, p);
+}
+
+moe_status moe_get_device_error(void* ws, void* stream) {
+  if (!ws) return MOE_ERR_WORKSPACE;
+  cudaStream_t s = (cudaStream_t)stream;
+  int err = 0;
+  if (cudaMemcpyAsync(&err, ws, sizeof(int), cudaMemcpyDeviceToHost, s) != cudaSuccess ||
+      cudaStreamSynchronize(s) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  if (err != 0) {
+    if (cudaMemsetAsync(ws, 0, sizeof(int), s) != cudaSuccess || cudaStreamSynchronize(s) != cudaSuccess) {
+      (void)cudaGetLastError();
+      return MOE_ERR_CUDA;
+    }
+  }
+  return (moe_status)err;
+}
+
+}  // extern "C"

@@ -1,0 +1,149 @@
+// router.cuh -- moe_router_topk: router GEMV (bf16 weights and input, fp32
+// accumulation), then softmax and top-K done by the last CTA to finish.
+#pragma once
+
+#include "common.cuh"
+
+namespace moeq {
+
+constexpr int kRouterWarps = 4;     // warps per CTA, one expert row per warp at a time
+constexpr int kRouterTokTile = 8;   // tokens whose x is staged in shared memory at once
+
+struct RouterParams {
+  const uint16_t* x;       // [B, H] bf16
+  const uint16_t* wr;      // [E, H] bf16
+  const int32_t* forced;   // [B, K] or null
+  int32_t* idx;            // [B, K]
+  float* w;                // [B, K]
+  float* logits;           // [B, E] (workspace or caller buffer)
+  WsCtrl* ctrl;
+  int B, H, E, K, renorm;
+};
+
+// Eight bf16 (one 16-byte word) against eight staged x values.
+__device__ __forceinline__ float dot8_bf16(uint4 wv, const uint4 xv, float acc) {
+  const uint32_t ww[4] = {wv.x, wv.y, wv.z, wv.w};
+  const uint32_t xx[4] = {xv.x, xv.y, xv.z, xv.w};
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    acc = fmaf(__uint_as_float(ww[i] << 16), __uint_as_float(xx[i] << 16), acc);
+    acc = fmaf(__uint_as_float(ww[i] & 0xFFFF0000u), __uint_as_float(xx[i] & 0xFFFF0000u), acc);
+  }
+  return acc;
+}
+
+// Top-K of one token's logits by one warp: K rounds of a warp arg-max with
+// ties to the lower index, then softmax weights at the picks.
+__device__ void topk_one_token(const float* lg, int E, int K, int renorm, const int32_t* forced, int32_t* idx_out,
+                               float* w_out, WsCtrl* ctrl) {
+  const int lane = threadIdx.x & 31;
+  int picked[MOEQ_MAX_K];
+  float mx = -INFINITY;
+  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, __ldcg(lg + e));
+  mx = warp_max(mx);
+  float z = 0.f;
+  for (int e = lane; e < E; e += 32) z += expf(__ldcg(lg + e) - mx);
+  z = warp_sum(z);
+  if (forced) {
+    for (int k = 0; k < K; ++k) {
+      int e = forced[k];
+      if (e < 0 || e >= E) {
+        if (lane == 0) set_error(ctrl, MOE_ERR_INDEX);
+        e = -1;
+      }
+      picked[k] = e;
+    }
+  } else {
+    for (int k = 0; k < K; ++k) {
+      float best = -INFINITY;
+      int bi = 0x7FFFFFFF;
+      for (int e = lane; e < E; e += 32) {
+        bool taken = false;
+        for (int j = 0; j < k; ++j) taken |= (picked[j] == e);
+        float v = __ldcg(lg + e);
+        if (!taken && (v > best || (v == best && e < bi))) {
+          best = v;
+          bi = e;
+        }
+      }
+#pragma unroll
+      for (int o = 16; o > 0; o >>= 1) {
+        float ov = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (ov > best || (ov == best && oi < bi)) {
+          best = ov;
+          bi = oi;
+        }
+      }
+      picked[k] = bi;
+    }
+  }
+  float p[MOEQ_MAX_K];
+  float tot = 0.f;
+  for (int k = 0; k < K; ++k) {
+    p[k] = picked[k] >= 0 ? expf(__ldcg(lg + picked[k]) - mx) / z : 0.f;
+    tot += p[k];
+  }
+  if (lane == 0) {
+    for (int k = 0; k < K; ++k) {
+      idx_out[k] = forced ? forced[k] : picked[k];
+      w_out[k] = (renorm && tot > 0.f) ? p[k] / tot : p[k];
+    }
+  }
+}
+
+__global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(RouterParams p) {
+  extern __shared__ __align__(16) unsigned char smem_raw[];
+  uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [tok_tile, H]
+  __shared__ int s_last;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  const int gwarp = blockIdx.x * kRouterWarps + warp, nwarps = gridDim.x * kRouterWarps;
+  const int nvec = p.H / 8;  // 16-byte words per row
+
+  pdl_wait();
+  for (int b0 = 0; b0 < p.B; b0 += kRouterTokTile) {
+    const int tb = min(kRouterTokTile, p.B - b0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < tb * nvec; i += blockDim.x)
+      reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x + (size_t)b0 * p.H)[i];
+    __syncthreads();
+    for (int e = gwarp; e < p.E; e += nwarps) {
+      const uint16_t* row = p.wr + (size_t)e * p.H;
+      float acc[kRouterTokTile];
+#pragma unroll
+      for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
+      for (int v = lane; v < nvec; v += 32) {
+        uint4 wv = ld_stream16(row + (size_t)v * 8);
+#pragma unroll
+        for (int t = 0; t < kRouterTokTile; ++t)
+          if (t < tb) acc[t] = dot8_bf16(wv, reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
+      }
+#pragma unroll
+      for (int t = 0; t < kRouterTokTile; ++t) {
+        if (t < tb) {
+          float s = warp_sum(acc[t]);
+          if (lane == 0) p.logits[(size_t)(b0 + t) * p.E + e] = s;
+        }
+      }
+    }
+  }
+  pdl_trigger();
+
+  // The last CTA to arrive selects for every token.
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    __threadfence();
+    unsigned t = atomicAdd(&p.ctrl->router_ticket, 1u);
+    s_last = (t == gridDim.x - 1);
+  }
+  __syncthreads();
+  if (!s_last) return;
+  __threadfence();
+  for (int b = warp; b < p.B; b += kRouterWarps)
+    topk_one_token(p.logits + (size_t)b * p.E, p.E, p.K, p.renorm, p.forced ? p.forced + (size_t)b * p.K : nullptr,
+                   p.idx + (size_t)b * p.K, p.w + (size_t)b * p.K, p.ctrl);
+  __syncthreads();
+  if (threadIdx.x == 0) p.ctrl->router_ticket = 0u;
+}
+
+}  // namespace moeq

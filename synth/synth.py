@@ -314,3 +314,11 @@ def zipf_routing(E: int, K: int, B: int, steps: int, s: float = 1.1, seed: int =
                 out[st, b, k] = perm[r]
                 wgt[r] = 0.0
     return out
+
+
+def fill_matrix_dev(w: Workload, layer: int, expert: int, matrix: int, codes_ptr: int, scale_ptr: int,
+                    bias_ptr: int, stream: int = 0) -> None:
+    """Write one matrix's codes and bf16 scale/bias into device buffers."""
+    codes_dev(w, layer, expert, matrix, codes_ptr, stream)
+    scale_dev(w, layer, expert, matrix, scale_ptr, stream)
+    bias_dev(w, layer, expert, matrix, bias_ptr, stream)

@@ -1,0 +1,291 @@
+"""GPU parity: every call of libmoeq.so against the oracle, through the C ABI.
+
+Bars: packed bytes and router indices bit-exact (indices compared where the
+oracle's ranking is decided by more than twice the observed logit error, else
+checked to be the exact top-K of the GPU's own logits); router weights within
+1e-5; expert and layer outputs within max|err| <= 2e-3 * ||y_oracle||_inf;
+combine within 1e-6 relative.
+"""
+import numpy as np
+import pytest
+
+from synth import synth
+from tests import harness as hz
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import quantized_expert_ffn_topk_b200 as moeq  # noqa: E402
+from oracle import layer as ref_layer  # noqa: E402
+from oracle import oracle as ref  # noqa: E402
+
+FFN_TOL = 2e-3
+W_TOL = 1e-5
+
+_layers = {}
+
+
+def get_layer(name, layer=0, shared_gate=False, **over):
+    w = synth.WORKLOADS[name].with_(**over) if over else synth.WORKLOADS[name]
+    key = (w, layer, shared_gate)
+    if key not in _layers:
+        if len(_layers) >= 2:  # keep at most two multi-GB arenas alive
+            _layers.clear()
+            torch.cuda.empty_cache()
+        _layers[key] = hz.build_layer(w, layer, shared_gate)
+    return w, _layers[key]
+
+
+def run_layer(w, L, x, forced=None, renorm=False, resid=None, eps=None):
+    B = x.shape[0]
+    ws = moeq.Workspace(B, w.K, w.H, w.I, w.E)
+    out = L.alloc_outputs(B)
+    fi = None if forced is None else torch.as_tensor(np.ascontiguousarray(forced, np.int32), device="cuda")
+    L.forward(x, ws, out, resid_in=resid, renorm=renorm, forced_idx=fi, eps=eps)
+    torch.cuda.synchronize()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    return out
+
+
+def oracle_token(w, layer, x_bits, forced=None, renorm=False, resid=None, shared_gate_bits=None, eps=None):
+    experts = hz.oracle_experts(w, layer)
+    return ref_layer.layer_token(w.H, w.I, w.E, w.K, w.group, x_bits, synth.router_host(w, layer), experts,
+                                 experts(w.E), renorm=renorm, forced=forced, resid=resid,
+                                 shared_gate_w=shared_gate_bits, eps=eps)
+
+
+# ---- generator: the device copy writes the host copy's bytes --------------
+
+def test_device_generator_matches_host():
+    w = synth.WORKLOADS["tiny"]
+    for (layer, e, m) in ((0, 0, synth.GATE), (3, 8, synth.DOWN), (1, 5, synth.UP)):
+        rows, cols = synth.matrix_shape(w, m)
+        c = torch.empty(rows * cols, dtype=torch.uint8, device="cuda")
+        s = torch.empty(rows * cols // w.group, dtype=torch.bfloat16, device="cuda")
+        b = torch.empty_like(s)
+        synth.fill_matrix_dev(w, layer, e, m, c.data_ptr(), s.data_ptr(), b.data_ptr())
+        torch.cuda.synchronize()
+        assert (c.cpu().numpy().reshape(rows, cols) == synth.codes_host(w, layer, e, m)).all()
+        assert (hz.bf16_bits(s).reshape(rows, -1) == synth.scale_host(w, layer, e, m)).all()
+        assert (hz.bf16_bits(b).reshape(rows, -1) == synth.bias_host(w, layer, e, m)).all()
+    x = hz.x_device(w, 7, 3)
+    assert (hz.bf16_bits(x) == synth.x_host(w, 7, 3)).all()
+
+
+# ---- A0 pack: byte-exact -----------------------------------------------------
+
+@pytest.mark.parametrize("rows,cols,bits,group", [(1, 32, 4, 32), (5, 64, 2, 32), (37, 320, 4, 64), (129, 256, 2, 64),
+                                                  (3, 512, 4, 128), (1024, 4096, 4, 64), (4096, 1024, 2, 64)])
+def test_pack_byte_exact(rows, cols, bits, group):
+    rng = np.random.default_rng(rows * 7 + cols + bits)
+    codes = rng.integers(0, 1 << bits, size=(rows, cols), dtype=np.uint8)
+    scale = rng.integers(0, 1 << 16, size=(rows, cols // group), dtype=np.uint16)
+    bias = rng.integers(0, 1 << 16, size=(rows, cols // group), dtype=np.uint16)
+    dc = torch.from_numpy(codes).cuda()
+    ds = torch.from_numpy(scale.view(np.int16)).cuda()
+    db = torch.from_numpy(bias.view(np.int16)).cuda()
+    packed = torch.full((rows, cols * bits // 8), 0xAB, dtype=torch.uint8, device="cuda")
+    sb = torch.full((rows, cols // group, 2), 0x5A5A, dtype=torch.int16, device="cuda")
+    ws = moeq.Workspace(1, 1, 32, 32, 1)
+    moeq.moe_pack_q(dc, ds, db, rows, cols, bits, group, packed, sb, ws.buf)
+    torch.cuda.synchronize()
+    rp, rsb = ref.pack(codes, scale, bias, bits, group)
+    assert (packed.cpu().numpy() == rp).all()
+    assert (sb.cpu().numpy().view(np.uint16) == rsb).all()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+
+
+def test_pack_flags_out_of_range_code():
+    rows, cols, bits, group = 4, 64, 4, 32
+    codes = np.zeros((rows, cols), np.uint8)
+    codes[2, 5] = 16
+    ws = moeq.Workspace(1, 1, 32, 32, 1)
+    packed = torch.empty((rows, cols // 2), dtype=torch.uint8, device="cuda")
+    sb = torch.empty((rows, 2, 2), dtype=torch.int16, device="cuda")
+    z = torch.zeros((rows, 2), dtype=torch.int16, device="cuda")
+    moeq.moe_pack_q(torch.from_numpy(codes).cuda(), z, z, rows, cols, bits, group, packed, sb, ws.buf)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_ERR_RANGE
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK  # read clears it
+
+
+def test_packed_arena_matches_oracle_pack():
+    w, L = get_layer("tiny")
+    rec = L.experts.cpu().numpy()
+    for e in (0, 5):
+        base = e * L.rec_r
+        g, u, d = synth.expert_host(w, 0, e)
+        for m, (codes, scale, bias) in enumerate((g, u, d)):
+            rp, rsb = ref.pack(codes, scale, bias, w.bits_routed, w.group)
+            got = rec[base + L.off_r[m]: base + L.off_r[m] + rp.size]
+            assert (got == rp.ravel()).all()
+            gsb = rec[base + L.off_r[3 + m]: base + L.off_r[3 + m] + rsb.size * 2].view(np.uint16)
+            assert (gsb == rsb.ravel()).all()
+
+
+# ---- A1+A2 router ------------------------------------------------------------
+
+@pytest.mark.parametrize("name,B,renorm", [("tiny", 1, False), ("tiny", 3, True), ("layer4", 1, False),
+                                           ("layer4", 5, True), ("layer4", 32, False)])
+def test_router_topk(name, B, renorm):
+    w, L = get_layer(name)
+    x = hz.x_device(w, 100, B)
+    ws = moeq.Workspace(B, w.K, w.H, w.I, w.E)
+    idx = torch.empty((B, w.K), dtype=torch.int32, device="cuda")
+    wt = torch.empty((B, w.K), dtype=torch.float32, device="cuda")
+    lg = torch.empty((B, w.E), dtype=torch.float32, device="cuda")
+    moeq.moe_router_topk(x, L.router_w, B, w.H, w.E, w.K, renorm, None, idx, wt, lg, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    wr = synth.router_host(w, 0)
+    xb = synth.x_host(w, 100, B)
+    exact = 0
+    for b in range(B):
+        rl = ref.router_logits(xb[b], wr)
+        tol = 1e-5 * float(np.abs(ref.bf16_to_f64(wr) * hz.bf16_to_f64(xb[b])[None, :]).sum(axis=1).max())
+        exact += hz.check_topk(idx[b].cpu().numpy(), lg[b].cpu().numpy(), rl, w.K, tol)
+        ri, rw = ref.topk(rl, w.K, renorm=renorm, forced=idx[b].cpu().numpy())
+        assert np.abs(wt[b].cpu().numpy() - rw).max() <= W_TOL
+    assert exact >= B - 1  # near ties are rare; never all of them
+
+
+def test_router_forced_and_bad_index():
+    w, L = get_layer("tiny")
+    B = 2
+    x = hz.x_device(w, 3, B)
+    ws = moeq.Workspace(B, w.K, w.H, w.I, w.E)
+    forced = torch.tensor([[3, 1], [0, 7]], dtype=torch.int32, device="cuda")
+    idx = torch.empty((B, w.K), dtype=torch.int32, device="cuda")
+    wt = torch.empty((B, w.K), dtype=torch.float32, device="cuda")
+    moeq.moe_router_topk(x, L.router_w, B, w.H, w.E, w.K, False, forced, idx, wt, None, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert (idx == forced).all()
+    wr = synth.router_host(w, 0)
+    xb = synth.x_host(w, 3, B)
+    for b in range(B):
+        _, rw = ref.topk(ref.router_logits(xb[b], wr), w.K, forced=forced[b].cpu().numpy())
+        assert np.abs(wt[b].cpu().numpy() - rw).max() <= W_TOL
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    bad = torch.tensor([[3, 8], [0, -1]], dtype=torch.int32, device="cuda")
+    moeq.moe_router_topk(x, L.router_w, B, w.H, w.E, w.K, False, bad, idx, wt, None, ws.buf, ws.nbytes)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_ERR_INDEX
+
+
+# ---- A3..A5 expert FFN ---------------------------------------------------------
+
+@pytest.mark.parametrize("name", ["tiny", "layer4", "layer2"])
+def test_expert_ffn(name):
+    w, L = get_layer(name)
+    B = 2
+    x = hz.x_device(w, 11, B)
+    rng = np.random.default_rng(5)
+    idx_np = np.stack([rng.choice(w.E, size=w.K, replace=False) for _ in range(B)]).astype(np.int32)
+    idx = torch.from_numpy(idx_np).cuda()
+    ws = moeq.Workspace(B, w.K, w.H, w.I, w.E)
+    y = torch.empty((B, w.K + 1, w.H), dtype=torch.float32, device="cuda")
+    moeq.moe_expert_ffn_q(L.struct, x, B, idx, y, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    experts = hz.oracle_experts(w, 0)
+    xb = synth.x_host(w, 11, B)
+    yg = y.cpu().numpy()
+    for b in range(B):
+        xd = hz.bf16_to_f64(xb[b])
+        for k, e in enumerate(list(idx_np[b]) + [w.E]):
+            g, u, d = experts(int(e))
+            yr = ref.expert_ffn(w.H, w.I, w.group, g, u, d, xd)
+            assert hz.max_rel_err(yg[b, k], yr) <= FFN_TOL, (b, k, e, hz.max_rel_err(yg[b, k], yr))
+
+
+def test_expert_ffn_bad_index_zeroes_slot():
+    w, L = get_layer("tiny")
+    x = hz.x_device(w, 1, 1)
+    idx = torch.tensor([[1, 99]], dtype=torch.int32, device="cuda")
+    ws = moeq.Workspace(1, w.K, w.H, w.I, w.E)
+    y = torch.full((1, w.K + 1, w.H), 7.0, dtype=torch.float32, device="cuda")
+    moeq.moe_expert_ffn_q(L.struct, x, 1, idx, y, ws.buf, ws.nbytes)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_ERR_INDEX
+    assert (y[0, 1] == 0).all() and (y[0, 0] != 0).any() and (y[0, 2] != 0).any()
+
+
+# ---- A6 combine ------------------------------------------------------------------
+
+@pytest.mark.parametrize("with_gate,with_resid", [(False, False), (True, True)])
+def test_combine_residual(with_gate, with_resid):
+    w, L = get_layer("tiny", shared_gate=with_gate)
+    B = 3
+    rng = np.random.default_rng(9)
+    y = torch.from_numpy(rng.normal(size=(B, w.K + 1, w.H)).astype(np.float32)).cuda()
+    wt = torch.from_numpy(rng.uniform(size=(B, w.K)).astype(np.float32)).cuda()
+    x = hz.x_device(w, 40, B)
+    resid = torch.from_numpy(synth.resid_host(w, 40, B)).cuda() if with_resid else None
+    out = torch.empty((B, w.H), dtype=torch.float32, device="cuda")
+    xn = torch.empty((B, w.H), dtype=torch.bfloat16, device="cuda")
+    moeq.moe_combine_residual(L.struct, y, wt, x, resid, B, out, xn, 1e-6)
+    torch.cuda.synchronize()
+    xb = synth.x_host(w, 40, B)
+    gw = synth.shared_gate_host(w, 0) if with_gate else None
+    for b in range(B):
+        gamma = ref.shared_gate(gw, xb[b]) if with_gate else 1.0
+        r = resid[b].cpu().numpy().astype(np.float64) if with_resid else hz.bf16_to_f64(xb[b])
+        ro = ref.combine(y[b].cpu().numpy().astype(np.float64), wt[b].cpu().numpy().astype(np.float64), gamma, r)
+        assert hz.max_rel_err(out[b].cpu().numpy(), ro) <= 1e-6
+        rn = ref.rmsnorm(ro, 1e-6)
+        xg = hz.bf16_to_f64(hz.bf16_bits(xn[b]))
+        # one bf16 rounding apart at most
+        assert (np.abs(xg - rn) <= np.abs(rn) * 2.0 ** -8 + 1e-30).all()
+
+
+# ---- A1..A6 whole layer -----------------------------------------------------------
+
+@pytest.mark.parametrize("name,B", [("tiny", 1), ("tiny", 4), ("layer4", 1), ("layer2", 1)])
+def test_layer_end_to_end(name, B):
+    w, L = get_layer(name)
+    x = hz.x_device(w, 500, B)
+    out = run_layer(w, L, x, eps=1e-6)
+    xb = synth.x_host(w, 500, B)
+    for b in range(B):
+        ro = oracle_token(w, 0, xb[b], eps=1e-6)
+        got_idx = out["idx"][b].cpu().numpy()
+        if list(got_idx) != list(ro["idx"]):  # a near tie: evaluate the oracle on the GPU's picks
+            hz.check_topk(got_idx, out["logits"][b].cpu().numpy(), ro["logits"], w.K, 1e-3)
+            ro = oracle_token(w, 0, xb[b], forced=got_idx, eps=1e-6)
+        assert np.abs(out["w"][b].cpu().numpy() - ro["w"]).max() <= W_TOL
+        yg = out["y"][b].cpu().numpy()
+        for k in range(w.K + 1):
+            assert hz.max_rel_err(yg[k], ro["y"][k]) <= FFN_TOL
+        assert hz.max_rel_err(out["resid"][b].cpu().numpy(), ro["out"]) <= FFN_TOL
+
+
+def test_batched_zipf_routing_layer():
+    w, L = get_layer("batch32")
+    routing = synth.zipf_routing(w.E, w.K, w.B, 1, w.zipf_s, w.seed)[0]
+    x = hz.x_device(w, 900, w.B)
+    out = run_layer(w, L, x, forced=routing)
+    xb = synth.x_host(w, 900, w.B)
+    for b in range(0, w.B, 7):
+        ro = oracle_token(w, 0, xb[b], forced=routing[b])
+        assert (out["idx"][b].cpu().numpy() == routing[b]).all()
+        assert np.abs(out["w"][b].cpu().numpy() - ro["w"]).max() <= W_TOL
+        assert hz.max_rel_err(out["resid"][b].cpu().numpy(), ro["out"]) <= FFN_TOL
+
+
+@pytest.mark.parametrize("over", [dict(H=320, I=96, E=5, K=1, group=32), dict(H=512, I=192, E=9, K=8, group=64),
+                                  dict(H=384, I=128, E=6, K=3, group=128, bits_routed=2),
+                                  dict(H=256, I=64, E=4, K=4, group=32, bits_routed=2, bits_shared=2)])
+def test_ragged_and_edge_shapes(over):
+    w = synth.WORKLOADS["tiny"].with_(**over)
+    L = hz.build_layer(w, 2)
+    B = 3
+    x = hz.x_device(w, 77, B)
+    out = run_layer(w, L, x, eps=1e-6)
+    xb = synth.x_host(w, 77, B)
+    for b in range(B):
+        got_idx = out["idx"][b].cpu().numpy()
+        ro = oracle_token(w, 2, xb[b], forced=got_idx, eps=1e-6)
+        if w.K < w.E:
+            hz.check_topk(got_idx, out["logits"][b].cpu().numpy(), ro["logits"], w.K, 1e-3)
+        assert hz.max_rel_err(out["resid"][b].cpu().numpy(), ro["out"]) <= FFN_TOL
+        for k in range(w.K + 1):
+            assert hz.max_rel_err(out["y"][b, k].cpu().numpy(), ro["y"][k]) <= FFN_TOL
