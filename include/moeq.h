@@ -181,6 +181,33 @@ moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const floa
                                 const float* resid_in, int B, float* resid_out, void* xnorm_bf16_out,
                                 float eps, void* stream);
 
+/*
+ * moe_decode_layers -- one token (batch 1) through n_layers MoE layers of the
+ * same shape in ONE persistent launch: for each layer l the router, softmax
+ * and top-K, the gate/up dequant mat-vecs with SwiGLU, the down dequant
+ * mat-vec, the combine with the shared expert and the residual, then the
+ * next layer's input x_{l+1} = bf16(RMSNorm(r_{l+1})), as the Flash-MoE page
+ * chains them ("Deferred GPU Expert Compute": combine + norm + residual stay
+ * on the GPU and feed the next layer). Results equal chaining
+ * moe_router_topk, moe_expert_ffn_q and moe_combine_residual per layer.
+ *   layers      host array of n_layers (1..64) layer descriptors
+ *   x_bf16      bf16 [H]: input of layer 0
+ *   resid_in    fp32 [H] residual of layer 0, or NULL: r_0 = x (widened)
+ *   forced_idx  int32 [n_layers, K] or NULL (as in moe_router_topk)
+ *   idx_out, w_out  int32 / fp32 [n_layers, K] or NULL: picks and weights
+ *   resid_out   fp32 [H]: r_n
+ *   xnorm_bf16_out  bf16 [H] or NULL: bf16(RMSNorm(r_n))
+ * Needs one CTA per SM for the whole launch (co-resident; cooperative
+ * launch), E <= 1024, (H/group) % 4 == 0, and a shared-memory plan that fits
+ * one SM (MOE_ERR_UNSUPPORTED otherwise; use the per-call path). A wait that
+ * exceeds about one second ends the kernel with MOE_ERR_TIMEOUT in the
+ * workspace, which must then be re-initialised with moe_workspace_init.
+ */
+moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers, const void* x_bf16, const float* resid_in,
+                             int renorm, const int32_t* forced_idx, int32_t* idx_out, float* w_out,
+                             float* resid_out, void* xnorm_bf16_out, float eps, void* ws, size_t ws_bytes,
+                             void* stream);
+
 /* Read (and clear) the workspace error word. Synchronises `stream`.
  * Returns MOE_OK, MOE_ERR_INDEX, MOE_ERR_RANGE, MOE_ERR_TIMEOUT, or
  * MOE_ERR_CUDA if the copy itself failed. */

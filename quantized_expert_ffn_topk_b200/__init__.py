@@ -52,6 +52,7 @@ _SIGS = {
     "moe_router_topk": (_INT, [_VP, _VP, _INT, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_expert_ffn_q": (_INT, [_LP, _VP, _INT, _VP, _VP, _VP, _SZ, _VP]),
     "moe_combine_residual": (_INT, [_LP, _VP, _VP, _VP, _VP, _INT, _VP, _VP, _FLT, _VP]),
+    "moe_decode_layers": (_INT, [_LP, _INT, _VP, _VP, _INT, _VP, _VP, _VP, _VP, _VP, _FLT, _VP, _SZ, _VP]),
     "moe_get_device_error": (_INT, [_VP, _VP]),
 }
 
@@ -147,6 +148,16 @@ def moe_combine_residual(layer: moe_layer_q, y, w, x_bf16, resid_in, B: int, res
     _check(lib().moe_combine_residual(ctypes.byref(layer), _ptr(y), _ptr(w), _ptr(x_bf16), _ptr(resid_in), B,
                                       _ptr(resid_out), _ptr(xnorm_bf16_out), float(eps), _stream(stream)),
            "moe_combine_residual")
+
+
+def moe_decode_layers(layers, x_bf16, resid_in, renorm: bool, forced_idx, idx_out, w_out, resid_out, xnorm_bf16_out,
+                      eps: float, ws, ws_bytes: int, stream=None) -> None:
+    """layers: a sequence of moe_layer_q (one token through all of them)."""
+    arr = (moe_layer_q * len(layers))(*layers)
+    _check(lib().moe_decode_layers(arr, len(layers), _ptr(x_bf16), _ptr(resid_in), int(bool(renorm)),
+                                   _ptr(forced_idx), _ptr(idx_out), _ptr(w_out), _ptr(resid_out),
+                                   _ptr(xnorm_bf16_out), float(eps), _ptr(ws), ws_bytes, _stream(stream)),
+           "moe_decode_layers")
 
 
 def moe_get_device_error(ws, stream=None) -> int:

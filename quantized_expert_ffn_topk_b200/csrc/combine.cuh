@@ -41,14 +41,32 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(CombineParams p) {
   for (int k = 0; k < MOEQ_MAX_K; ++k) wk[k] = k < p.K ? p.w[(size_t)b * p.K + k] : 0.f;
   const float* yb = p.y + (size_t)b * (p.K + 1) * p.H;
   float ss = 0.f;
-  for (int j = threadIdx.x; j < p.H; j += blockDim.x) {
-    float acc = p.resid_in ? p.resid_in[(size_t)b * p.H + j] : bf16_bits_to_f32(xb[j]);
+  constexpr int U = 4;  // elements per thread in flight
+  for (int j0 = threadIdx.x; j0 < p.H; j0 += blockDim.x * U) {
+    float acc[U], ys[U][MOEQ_MAX_K + 1];
 #pragma unroll
-    for (int k = 0; k < MOEQ_MAX_K; ++k)
-      if (k < p.K) acc += wk[k] * yb[(size_t)k * p.H + j];
-    acc += gamma * yb[(size_t)p.K * p.H + j];
-    p.resid_out[(size_t)b * p.H + j] = acc;
-    ss += acc * acc;
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * blockDim.x;
+      if (j < p.H) {
+        acc[u] = p.resid_in ? p.resid_in[(size_t)b * p.H + j] : bf16_bits_to_f32(xb[j]);
+#pragma unroll
+        for (int k = 0; k <= MOEQ_MAX_K; ++k)
+          if (k <= p.K) ys[u][k] = yb[(size_t)k * p.H + j];
+      }
+    }
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int j = j0 + u * blockDim.x;
+      if (j < p.H) {
+        float a = acc[u];
+#pragma unroll
+        for (int k = 0; k < MOEQ_MAX_K; ++k)
+          if (k < p.K) a += wk[k] * ys[u][k];
+        a += gamma * ys[u][p.K];
+        p.resid_out[(size_t)b * p.H + j] = a;
+        ss += a * a;
+      }
+    }
   }
   if (p.xnorm) {
     ss = block_sum(ss, red);

@@ -13,7 +13,9 @@ namespace moeq {
 struct WsCtrl {
   int error;                // first device-side moe_status (0 = none)
   unsigned router_ticket;   // last-CTA ticket of the router kernel (back to 0 after each call)
-  unsigned pad[62];
+  unsigned sync_count;      // grid-wide arrival counter of the fused decode kernel (0 between calls)
+  unsigned exit_count;      // CTAs that left the fused decode kernel (0 between calls)
+  unsigned pad[60];
 };
 static_assert(sizeof(WsCtrl) == 256, "control block is 256 bytes");
 
@@ -116,6 +118,84 @@ __device__ __forceinline__ int fp16_scale_exp(float amax) {
   if (!(amax > 0.f) || !isfinite(amax)) return 0;
   int e = 15 - (((int)((__float_as_uint(amax) >> 23) & 0xFF)) - 126);
   return max(-120, min(120, e));
+}
+
+}  // namespace moeq
+
+// ---- mbarriers, bulk async copies, bounded waits (sm_90+/sm_100a) ---------
+namespace moeq {
+
+__device__ __forceinline__ uint32_t smem_u32(const void* p) { return (uint32_t)__cvta_generic_to_shared(p); }
+
+__device__ __forceinline__ void mbar_init(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.init.shared::cta.b64 [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
+__device__ __forceinline__ void fence_mbar_init() { asm volatile("fence.mbarrier_init.release.cluster;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async() { asm volatile("fence.proxy.async.shared::cta;" ::: "memory"); }
+
+__device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t bytes) {
+  asm volatile("mbarrier.arrive.expect_tx.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(bytes) : "memory");
+}
+__device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
+}
+__device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
+  uint32_t ok;
+  asm volatile(
+      "{ .reg .pred p;\n\t mbarrier.try_wait.parity.shared::cta.b64 p, [%1], %2;\n\t selp.u32 %0, 1, 0, p; }"
+      : "=r"(ok)
+      : "r"(smem_u32(bar)), "r"(parity)
+      : "memory");
+  return ok != 0;
+}
+
+// Bulk copy global -> this CTA's shared memory; completion counted in bytes
+// on `bar`. Addresses 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+                   smem_u32(dst)),
+               "l"(src), "r"(bytes), "r"(smem_u32(bar))
+               : "memory");
+}
+
+__device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.acquire.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Wait budget for every spin in the library: ~1 s of SM clock cycles.
+constexpr long long kWaitBudgetCycles = 2000000000LL;
+
+// Bounded wait for an mbarrier phase; false on timeout or when `abort` is set.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) return false;
+  }
+}
+
+// Bounded wait until *counter >= target (gpu-scope acquire).
+__device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned target, const volatile int* abort) {
+  if (ld_acquire_gpu(counter) >= target) return true;
+  const long long t0 = clock64();
+  while (ld_acquire_gpu(counter) < target) {
+    if (*abort) return false;
+    if (clock64() - t0 > kWaitBudgetCycles) return false;
+    __nanosleep(32);
+  }
+  return true;
+}
+
+// Named barriers among a subset of the CTA's warps.
+__device__ __forceinline__ void named_sync(int id, int nthreads) {
+  asm volatile("bar.sync %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
+}
+__device__ __forceinline__ void named_arrive(int id, int nthreads) {
+  asm volatile("bar.arrive %0, %1;" ::"r"(id), "r"(nthreads) : "memory");
 }
 
 }  // namespace moeq

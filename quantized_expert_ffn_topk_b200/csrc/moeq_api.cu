@@ -10,6 +10,7 @@
 #include "ffn.cuh"
 #include "pack.cuh"
 #include "router.cuh"
+#include "stack.cuh"
 
 namespace moeq {
 namespace {
@@ -74,17 +75,21 @@ moe_status ensure_smem(K kern, size_t bytes) {
 }
 
 // Workspace layout: [control 256 B][logits B*E fp32][h B*(K+1)*I fp32]
+//                   [r B*H fp32][ss kStackMaxLayers fp32]
 struct WsLayout {
-  size_t logits, h, total;
+  size_t logits, h, r, ss, total;
 };
 inline WsLayout ws_layout(int B, int K, int H, int I, int E) {
-  (void)H;
   WsLayout l{};
   size_t o = sizeof(WsCtrl);
   l.logits = o;
   o += align_up((size_t)B * E * sizeof(float));
   l.h = o;
   o += align_up((size_t)B * (K + 1) * I * sizeof(float));
+  l.r = o;
+  o += align_up((size_t)B * H * sizeof(float));
+  l.ss = o;
+  o += align_up((size_t)kStackMaxLayers * sizeof(float));
   l.total = o;
   return l;
 }
@@ -201,7 +206,7 @@ moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B,
   if (!ws) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_workspace_bytes(B, K, H, 32, E)) return MOE_ERR_WORKSPACE;
   if (!aligned16(x_bf16) || !aligned16(router_w_bf16) || !aligned16(ws)) return MOE_ERR_ALIGN;
-  const size_t smem = (size_t)std::min(B, kRouterTokTile) * H * 2;
+  const size_t smem = std::max((size_t)std::min(B, kRouterTokTile) * H * 2, (size_t)std::min(B, kRouterTokTile) * E * 4);
   if (ensure_smem(k_router_topk, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;
   RouterParams p{};
   p.x = reinterpret_cast<const uint16_t*>(x_bf16);
@@ -256,11 +261,13 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
   const DnSmem ds = dn_smem_plan(p.I, p.K);
   if (ensure_smem(k_gate_up, gs.bytes) != MOE_OK || ensure_smem(k_down, ds.bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
 
-  const int gu_units = (p.K + 1) * p.I, dn_units = (p.K + 1) * p.H;
-  p.units_per_cta_gu = kFfnWarps;
-  p.units_per_cta_dn = kFfnWarps * 4;
-  const int gu_ctas = (gu_units + p.units_per_cta_gu - 1) / p.units_per_cta_gu;
-  const int dn_ctas = (dn_units + p.units_per_cta_dn - 1) / p.units_per_cta_dn;
+  // persistent grids: about two CTAs per SM in total, spread over the tokens
+  const int gu_units = (p.K + 1) * p.I, dn_units = (p.K + 1) * (p.H / kDownRows);
+  const int per_tok = std::max(1, 2 * num_sms() / B);
+  const int gu_ctas = std::min(per_tok, (gu_units + kFfnWarps - 1) / kFfnWarps);
+  const int dn_ctas = std::min(per_tok, (dn_units + kFfnWarps - 1) / kFfnWarps);
+  p.units_per_cta_gu = (gu_units + gu_ctas - 1) / gu_ctas;
+  p.units_per_cta_dn = (dn_units + dn_ctas - 1) / dn_ctas;
   cudaStream_t s = (cudaStream_t)stream;
   st = launch_pdl(k_gate_up, dim3(gu_ctas, B), dim3(kFfnWarps * 32), gs.bytes, s, p);
   if (st != MOE_OK) return st;
@@ -310,3 +317,126 @@ moe_status moe_get_device_error(void* ws, void* stream) {
 }
 
 }  // extern "C"
+
+namespace moeq {
+namespace {
+
+// Shared-memory plan of the fused decode kernel; false when it does not fit.
+bool stack_plan(StackParams& p, int G) {
+  const int H = p.H, I = p.I, K = p.K;
+  size_t o = 0;
+  auto take = [&](size_t bytes) {
+    const size_t at = o;
+    o += align_up(bytes, 128);
+    return (int)at;
+  };
+  p.need4 = (p.bits_r == 4 || p.bits_s == 4);
+  p.need2 = (p.bits_r == 2 || p.bits_s == 2);
+  p.sm_xs = take((size_t)H * 2);
+  p.sm_img4 = take(p.need4 ? (size_t)H * 2 : 0);
+  p.sm_tab4 = take(p.need4 ? (size_t)(H / Img<4>::HC) * 8 : 0);
+  p.sm_img2 = take(p.need2 ? (size_t)H * 2 : 0);
+  p.sm_tab2 = take(p.need2 ? (size_t)(H / Img<2>::HC) * 8 : 0);
+  p.himg_stride = (int)align_up((size_t)I * 2, 128);
+  p.htab_stride = (int)align_up((size_t)(I / Img<4>::HC) * 8, 128);
+  p.sm_himg = take((size_t)p.himg_stride * (K + 1));
+  p.sm_htab = take((size_t)p.htab_stride * (K + 1));
+  p.nblk_max = strided_count(0, G, H / kDnBlk);
+  const int bmax = std::max(p.bits_r, p.bits_s);
+  p.dblk_bytes = (int)align_up((size_t)kDnBlk * ((size_t)I * bmax / 8 + (size_t)I / p.G * 4), 16);
+  p.sm_regc = take((size_t)p.dblk_bytes * p.nblk_max * (K + 1));
+  const size_t unit = std::max((size_t)H, 2 * ((size_t)H * bmax / 8) + 2 * ((size_t)H / p.G * 4));
+  p.slot_bytes = (int)align_up(unit, 128);
+  const size_t budget = 227 * 1024 - 2048;  // leave room for the static shared memory
+  if (o + (size_t)p.slot_bytes * 2 > budget) return false;
+  p.nslot = (int)std::min<size_t>(kMaxSlots, (budget - o) / p.slot_bytes);
+  p.sm_ring = take((size_t)p.slot_bytes * p.nslot);
+  return o <= budget;
+}
+
+size_t stack_smem_bytes(const StackParams& p) { return (size_t)p.sm_ring + (size_t)p.slot_bytes * p.nslot; }
+
+}  // namespace
+}  // namespace moeq
+
+extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers, const void* x_bf16,
+                                        const float* resid_in, int renorm, const int32_t* forced_idx,
+                                        int32_t* idx_out, float* w_out, float* resid_out, void* xnorm_bf16_out,
+                                        float eps, void* ws, size_t ws_bytes, void* stream) {
+  if (!layers || n_layers <= 0 || n_layers > kStackMaxLayers) return MOE_ERR_INVALID_ARG;
+  const moe_layer_q& L0 = layers[0];
+  for (int l = 0; l < n_layers; ++l) {
+    moe_status st = check_layer(&layers[l]);
+    if (st != MOE_OK) return st;
+    const moe_layer_q& L = layers[l];
+    if (L.H != L0.H || L.I != L0.I || L.E != L0.E || L.K != L0.K || L.group != L0.group ||
+        L.bits_routed != L0.bits_routed || L.bits_shared != L0.bits_shared)
+      return MOE_ERR_INVALID_ARG;
+  }
+  if (!x_bf16 || !resid_out) return MOE_ERR_INVALID_ARG;
+  if (!(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(resid_out) || (resid_in && !aligned16(resid_in)) ||
+      (xnorm_bf16_out && !aligned16(xnorm_bf16_out)) || (ws && !aligned16(ws)))
+    return MOE_ERR_ALIGN;
+  if (!ws) return MOE_ERR_WORKSPACE;
+  if (ws_bytes < moe_workspace_bytes(1, L0.K, L0.H, L0.I, L0.E)) return MOE_ERR_WORKSPACE;
+  const int G = num_sms();
+  if (L0.E > 1024 || strided_count(0, G, L0.E) > kMaxRouterRowsPerCta) return MOE_ERR_UNSUPPORTED;
+  if ((L0.H / L0.group) % 4 != 0 || L0.H % (2 * 16) != 0) return MOE_ERR_UNSUPPORTED;
+
+  StackParams p{};
+  for (int l = 0; l < n_layers; ++l) {
+    p.L[l].experts = reinterpret_cast<const uint8_t*>(layers[l].experts);
+    p.L[l].shared = reinterpret_cast<const uint8_t*>(layers[l].shared);
+    p.L[l].router_w = reinterpret_cast<const uint16_t*>(layers[l].router_w);
+    p.L[l].gate_w = reinterpret_cast<const uint16_t*>(layers[l].shared_gate_w);
+  }
+  p.n_layers = n_layers;
+  p.H = L0.H;
+  p.I = L0.I;
+  p.E = L0.E;
+  p.K = L0.K;
+  p.G = L0.group;
+  p.bits_r = L0.bits_routed;
+  p.bits_s = L0.bits_shared;
+  p.rec_r = moe_expert_bytes(p.H, p.I, p.bits_r, p.G);
+  size_t off[6];
+  expert_offsets(p.H, p.I, p.bits_r, p.G, off);
+  for (int i = 0; i < 6; ++i) p.off_r[i] = (uint32_t)off[i];
+  expert_offsets(p.H, p.I, p.bits_s, p.G, off);
+  for (int i = 0; i < 6; ++i) p.off_s[i] = (uint32_t)off[i];
+  p.x_in = reinterpret_cast<const uint16_t*>(x_bf16);
+  p.resid_in = resid_in;
+  p.forced = forced_idx;
+  p.idx_out = idx_out;
+  p.w_out = w_out;
+  p.resid_out = resid_out;
+  p.xnorm_out = reinterpret_cast<uint16_t*>(xnorm_bf16_out);
+  p.eps = eps;
+  p.renorm = renorm;
+  WsLayout wl = ws_layout(1, p.K, p.H, p.I, p.E);
+  p.ctrl = reinterpret_cast<WsCtrl*>(ws);
+  p.logits = reinterpret_cast<float*>((char*)ws + wl.logits);
+  p.h = reinterpret_cast<float*>((char*)ws + wl.h);
+  p.r = reinterpret_cast<float*>((char*)ws + wl.r);
+  p.ss = reinterpret_cast<float*>((char*)ws + wl.ss);
+  if (!stack_plan(p, G)) return MOE_ERR_UNSUPPORTED;
+  const size_t smem = stack_smem_bytes(p);
+  if (ensure_smem(k_decode_layers, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;
+
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(G);
+  cfg.blockDim = dim3(kStackThreads);
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = (cudaStream_t)stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeCooperative;  // all CTAs co-resident: they wait on one another
+  attr[0].val.cooperative = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  if (cudaLaunchKernelEx(&cfg, k_decode_layers, p) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  return MOE_OK;
+}

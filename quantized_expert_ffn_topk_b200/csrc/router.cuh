@@ -8,6 +8,7 @@ namespace moeq {
 
 constexpr int kRouterWarps = 4;     // warps per CTA, one expert row per warp at a time
 constexpr int kRouterTokTile = 8;   // tokens whose x is staged in shared memory at once
+constexpr int kRouterUnroll = 16;   // 16-byte loads of one row in flight per lane
 
 struct RouterParams {
   const uint16_t* x;       // [B, H] bf16
@@ -39,10 +40,10 @@ __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const 
   const int lane = threadIdx.x & 31;
   int picked[MOEQ_MAX_K];
   float mx = -INFINITY;
-  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, __ldcg(lg + e));
+  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, lg[e]);
   mx = warp_max(mx);
   float z = 0.f;
-  for (int e = lane; e < E; e += 32) z += expf(__ldcg(lg + e) - mx);
+  for (int e = lane; e < E; e += 32) z += expf(lg[e] - mx);
   z = warp_sum(z);
   if (forced) {
     for (int k = 0; k < K; ++k) {
@@ -60,7 +61,7 @@ __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const 
       for (int e = lane; e < E; e += 32) {
         bool taken = false;
         for (int j = 0; j < k; ++j) taken |= (picked[j] == e);
-        float v = __ldcg(lg + e);
+        float v = lg[e];
         if (!taken && (v > best || (v == best && e < bi))) {
           best = v;
           bi = e;
@@ -75,13 +76,17 @@ __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const 
           bi = oi;
         }
       }
+      if (bi < 0 || bi >= E) {  // no finite logit left (NaN input): no expert
+        if (lane == 0) set_error(ctrl, MOE_ERR_INDEX);
+        bi = -1;
+      }
       picked[k] = bi;
     }
   }
   float p[MOEQ_MAX_K];
   float tot = 0.f;
   for (int k = 0; k < K; ++k) {
-    p[k] = picked[k] >= 0 ? expf(__ldcg(lg + picked[k]) - mx) / z : 0.f;
+    p[k] = picked[k] >= 0 ? expf(lg[picked[k]] - mx) / z : 0.f;
     tot += p[k];
   }
   if (lane == 0) {
@@ -112,11 +117,20 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(RouterParams 
       float acc[kRouterTokTile];
 #pragma unroll
       for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
-      for (int v = lane; v < nvec; v += 32) {
-        uint4 wv = ld_stream16(row + (size_t)v * 8);
+      for (int v0 = lane; v0 < nvec; v0 += 32 * kRouterUnroll) {
+        uint4 wv[kRouterUnroll];
 #pragma unroll
-        for (int t = 0; t < kRouterTokTile; ++t)
-          if (t < tb) acc[t] = dot8_bf16(wv, reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
+        for (int u = 0; u < kRouterUnroll; ++u)
+          if (v0 + 32 * u < nvec) wv[u] = ld_stream16(row + (size_t)(v0 + 32 * u) * 8);
+#pragma unroll
+        for (int u = 0; u < kRouterUnroll; ++u) {
+          const int v = v0 + 32 * u;
+          if (v < nvec) {
+#pragma unroll
+            for (int t = 0; t < kRouterTokTile; ++t)
+              if (t < tb) acc[t] = dot8_bf16(wv[u], reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
+          }
+        }
       }
 #pragma unroll
       for (int t = 0; t < kRouterTokTile; ++t) {
@@ -139,9 +153,18 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(RouterParams 
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  for (int b = warp; b < p.B; b += kRouterWarps)
-    topk_one_token(p.logits + (size_t)b * p.E, p.E, p.K, p.renorm, p.forced ? p.forced + (size_t)b * p.K : nullptr,
-                   p.idx + (size_t)b * p.K, p.w + (size_t)b * p.K, p.ctrl);
+  float* lsm = reinterpret_cast<float*>(smem_raw);  // logits of up to kRouterTokTile tokens
+  for (int b0 = 0; b0 < p.B; b0 += kRouterTokTile) {
+    const int tb = min(kRouterTokTile, p.B - b0);
+    __syncthreads();
+    for (int i = threadIdx.x; i < tb * p.E; i += blockDim.x) lsm[i] = __ldcg(p.logits + (size_t)b0 * p.E + i);
+    __syncthreads();
+    for (int t = warp; t < tb; t += kRouterWarps) {
+      const int b = b0 + t;
+      topk_one_token(lsm + (size_t)t * p.E, p.E, p.K, p.renorm, p.forced ? p.forced + (size_t)b * p.K : nullptr,
+                     p.idx + (size_t)b * p.K, p.w + (size_t)b * p.K, p.ctrl);
+    }
+  }
   __syncthreads();
   if (threadIdx.x == 0) p.ctrl->router_ticket = 0u;
 }

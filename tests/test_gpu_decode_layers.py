@@ -1,0 +1,173 @@
+"""GPU parity of the fused persistent decode (moe_decode_layers) against the
+oracle: one layer (router-driven), a chain of layers carried through the
+residual and RMSNorm, forced routing, the device error path and repeat calls
+on one workspace."""
+import numpy as np
+import pytest
+
+from synth import synth
+from tests import harness as hz
+
+pytestmark = pytest.mark.gpu
+
+torch = pytest.importorskip("torch")
+if not torch.cuda.is_available():
+    pytest.skip("needs a CUDA GPU", allow_module_level=True)
+
+import quantized_expert_ffn_topk_b200 as moeq  # noqa: E402
+from oracle import layer as ref_layer  # noqa: E402
+
+FFN_TOL = 2e-3
+W_TOL = 1e-5
+EPS = 1e-6
+
+_cache = {}
+
+
+def layers_for(name, n, **over):
+    w = synth.WORKLOADS[name].with_(**over) if over else synth.WORKLOADS[name]
+    key = (w, n)
+    if key not in _cache:
+        _cache.clear()
+        torch.cuda.empty_cache()
+        _cache[key] = (w, [hz.build_layer(w, l) for l in range(n)])
+    return _cache[key]
+
+
+def run(w, Ls, x, resid=None, forced=None, renorm=False):
+    n = len(Ls)
+    ws = moeq.Workspace(1, w.K, w.H, w.I, w.E)
+    idx = torch.empty((n, w.K), dtype=torch.int32, device="cuda")
+    wt = torch.empty((n, w.K), dtype=torch.float32, device="cuda")
+    out = torch.empty(w.H, dtype=torch.float32, device="cuda")
+    xn = torch.empty(w.H, dtype=torch.bfloat16, device="cuda")
+    fi = None if forced is None else torch.as_tensor(np.ascontiguousarray(forced, np.int32), device="cuda")
+    moeq.moe_decode_layers([L.struct for L in Ls], x, resid, renorm, fi, idx, wt, out, xn, EPS, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    return ws, idx.cpu().numpy(), wt.cpu().numpy(), out.cpu().numpy().astype(np.float64), hz.bf16_bits(xn)
+
+
+def oracle_chain(w, n, x_bits, forced=None, gpu_idx=None):
+    """Chain the oracle over n layers; where the GPU picked differently on a
+    near tie, follow the GPU's picks (checked by the caller)."""
+    x = x_bits
+    r = None
+    res = []
+    for l in range(n):
+        experts = hz.oracle_experts(w, l)
+        f = None if forced is None else forced[l]
+        ro = ref_layer.layer_token(w.H, w.I, w.E, w.K, w.group, x, synth.router_host(w, l), experts, experts(w.E),
+                                   forced=f, resid=r, eps=EPS)
+        if forced is None and gpu_idx is not None and list(ro["idx"]) != list(gpu_idx[l]):
+            ro = ref_layer.layer_token(w.H, w.I, w.E, w.K, w.group, x, synth.router_host(w, l), experts,
+                                       experts(w.E), forced=gpu_idx[l], resid=r, eps=EPS)
+            ro["near_tie"] = True
+        res.append(ro)
+        x, r = ro["xn"], ro["out"]
+    return res
+
+
+@pytest.mark.parametrize("name", ["tiny", "layer4", "layer2"])
+def test_one_layer_matches_oracle(name):
+    w, Ls = layers_for(name, 1)
+    x = hz.x_device(w, 321, 1)[0]
+    ws, idx, wt, out, xn = run(w, Ls, x)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    ro = oracle_chain(w, 1, synth.x_host(w, 321)[0], gpu_idx=idx)[0]
+    assert "near_tie" not in ro, (idx[0], ro["idx"])
+    assert list(idx[0]) == list(ro["idx"])
+    assert np.abs(wt[0] - ro["w"]).max() <= W_TOL
+    assert hz.max_rel_err(out, ro["out"]) <= FFN_TOL
+    xg = hz.bf16_to_f64(xn)
+    rn = ro["out"] / np.sqrt(np.mean(ro["out"] ** 2) + EPS)
+    assert (np.abs(xg - rn) <= np.abs(rn) * 2.0 ** -7 + 1e-6).all()
+
+
+def test_chain_of_layers_router_driven():
+    n = 3
+    w, Ls = layers_for("layer4", n)
+    x = hz.x_device(w, 11, 1)[0]
+    ws, idx, wt, out, xn = run(w, Ls, x)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    res = oracle_chain(w, n, synth.x_host(w, 11)[0], gpu_idx=idx)
+    ties = sum("near_tie" in ro for ro in res)
+    assert ties <= 1
+    for l in range(n):
+        assert np.abs(wt[l] - res[l]["w"]).max() <= W_TOL
+    assert hz.max_rel_err(out, res[-1]["out"]) <= FFN_TOL
+
+
+def test_stack_with_forced_overlap_routing():
+    n = 6
+    w, Ls = layers_for("layer4", n)
+    routing = synth.overlap_routing(w.E, w.K, 2, n, 0.27, seed=0)
+    for t in range(2):
+        x = hz.x_device(w, 1000 + t, 1)[0]
+        ws, idx, wt, out, xn = run(w, Ls, x, forced=routing[t])
+        assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+        assert (idx == routing[t]).all()
+        res = oracle_chain(w, n, synth.x_host(w, 1000 + t)[0], forced=routing[t])
+        for l in range(n):
+            assert np.abs(wt[l] - res[l]["w"]).max() <= W_TOL
+        assert hz.max_rel_err(out, res[-1]["out"]) <= FFN_TOL
+
+
+def test_residual_input_and_renorm():
+    w, Ls = layers_for("tiny", 2)
+    x = hz.x_device(w, 5, 1)[0]
+    resid = torch.from_numpy(synth.resid_host(w, 5)[0]).cuda()
+    ws, idx, wt, out, xn = run(w, Ls, x, resid=resid, renorm=True)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    xb = synth.x_host(w, 5)[0]
+    r = resid.cpu().numpy().astype(np.float64)
+    for l in range(2):
+        experts = hz.oracle_experts(w, l)
+        ro = ref_layer.layer_token(w.H, w.I, w.E, w.K, w.group, xb, synth.router_host(w, l), experts, experts(w.E),
+                                   renorm=True, forced=idx[l], resid=r, eps=EPS)
+        assert np.abs(wt[l] - ro["w"]).max() <= W_TOL
+        xb, r = ro["xn"], ro["out"]
+    assert hz.max_rel_err(out, r) <= FFN_TOL
+
+
+def test_bad_forced_index_and_repeat_calls():
+    w, Ls = layers_for("tiny", 1)
+    x = hz.x_device(w, 9, 1)[0]
+    ws, idx, wt, out, xn = run(w, Ls, x)
+    ws2, idx2, wt2, out2, xn2 = run(w, Ls, x)
+    assert (out == out2).all() and (idx == idx2).all()
+    # the same workspace twice in a row: counters come back to zero
+    n = 1
+    idx_t = torch.empty((n, w.K), dtype=torch.int32, device="cuda")
+    wt_t = torch.empty((n, w.K), dtype=torch.float32, device="cuda")
+    o = torch.empty(w.H, dtype=torch.float32, device="cuda")
+    for _ in range(3):
+        moeq.moe_decode_layers([Ls[0].struct], x, None, False, None, idx_t, wt_t, o, None, EPS, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    assert (o.cpu().numpy() == out.astype(np.float32)).all()
+    bad = torch.tensor([[1, 8]], dtype=torch.int32, device="cuda")
+    moeq.moe_decode_layers([Ls[0].struct], x, None, False, bad, idx_t, wt_t, o, None, EPS, ws.buf, ws.nbytes)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_ERR_INDEX
+
+
+def test_graph_capture_of_decode_layers():
+    w, Ls = layers_for("tiny", 2)
+    x = hz.x_device(w, 4, 1)[0]
+    ws = moeq.Workspace(1, w.K, w.H, w.I, w.E)
+    o = torch.empty(w.H, dtype=torch.float32, device="cuda")
+    xn = torch.empty(w.H, dtype=torch.bfloat16, device="cuda")
+    s = torch.cuda.Stream()
+    with torch.cuda.stream(s):
+        moeq.moe_decode_layers([L.struct for L in Ls], x, None, False, None, None, None, o, xn, EPS, ws.buf, ws.nbytes)
+        s.synchronize()
+        ref_o = o.clone()
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=s):
+            moeq.moe_decode_layers([L.struct for L in Ls], x, None, False, None, None, None, o, xn, EPS, ws.buf,
+                                   ws.nbytes)
+        o.zero_()
+        g.replay()
+        g.replay()
+        s.synchronize()
+    assert (o == ref_o).all()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
