@@ -36,7 +36,7 @@ def parse():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="layer4", choices=["layer4", "layer2"])
-    ap.add_argument("--layers", type=int, default=16, help="resident layers walked by the steps (even)")
+    ap.add_argument("--layers", type=int, default=16, help="resident layers walked by the steps")
     ap.add_argument("--cpu-sample", type=int, default=12, help="tokens in the oracle CPU-baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     return ap.parse_args()
@@ -154,6 +154,81 @@ def run_reference(args, w, rank: int):
 
 # ---- our arm ------------------------------------------------------------------
 
+def build_layers(w, nlayers, dev, s):
+    import quantized_expert_ffn_topk_b200 as moeq
+    from synth import synth
+    layers = []
+    for l in range(nlayers):
+        L = moeq.QuantLayer(w.H, w.I, w.E, w.K, w.group, w.bits_routed, w.bits_shared, device=dev)
+        L.fill(lambda e, m, c, sc, b, l=l: synth.fill_matrix_dev(w, l, e, m, c, sc, b, s), stream=s)
+        synth.router_dev(w, l, L.router_w.data_ptr(), s)
+        layers.append(L)
+    return layers
+
+
+def per_call_path(w, layers, ws, dev, stream, steps):
+    """The four per-token calls (router+top-K, expert FFN, combine) chained
+    like decode, each step one CUDA graph of 4 kernels with PDL; also times
+    the expert-FFN call alone with events around it."""
+    import torch
+
+    import quantized_expert_ffn_topk_b200 as moeq
+    s = stream.cuda_stream
+    nl = len(layers)
+    xbuf = [torch.empty((1, w.H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
+    xbuf[0].normal_()
+    resid = xbuf[0].float().clone()
+    outs = [L.alloc_outputs(1, logits=False, xnorm=False) for L in layers]
+    for o in outs:
+        o["resid"] = resid
+
+    def step(t):
+        l = t % nl
+        o = outs[l]
+        o["xnorm"] = xbuf[(l + 1) % 2]
+        layers[l].forward(xbuf[l % 2], ws, o, resid_in=resid, eps=1e-6, stream=s)
+
+    for l in range(nl):
+        step(l)
+    torch.cuda.synchronize()
+    graphs = []
+    for l in range(nl):
+        g = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g, stream=stream):
+            step(l)
+        graphs.append(g)
+    for t in range(2 * nl):
+        graphs[t % nl].replay()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    torch.cuda.synchronize()
+    a.record(stream)
+    for t in range(steps):
+        graphs[t % nl].replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b)
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nl)]
+    ffn_ms = []
+    for t in range(max(nl, min(steps, 1600))):
+        l = t % nl
+        L, o = layers[l], outs[l]
+        xin = xbuf[l % 2]
+        moeq.moe_router_topk(xin, L.router_w, 1, w.H, w.E, w.K, False, None, o["idx"], o["w"], None, ws.buf,
+                             ws.nbytes, s)
+        e0, e1 = ev[l]
+        e0.record(stream)
+        moeq.moe_expert_ffn_q(L.struct, xin, 1, o["idx"], o["y"], ws.buf, ws.nbytes, s)
+        e1.record(stream)
+        o["xnorm"] = xbuf[(l + 1) % 2]
+        moeq.moe_combine_residual(L.struct, o["y"], o["w"], xin, resid, 1, resid, o["xnorm"], 1e-6, s)
+        if l == nl - 1:
+            torch.cuda.synchronize()
+            ffn_ms += [x.elapsed_time(y) for (x, y) in ev]
+    torch.cuda.synchronize()
+    del graphs
+    return steps / (ms / 1e3), statistics.mean(ffn_ms)
+
+
 def run_ours(args, w, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -164,57 +239,50 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(device=dev)
-    nlayers = args.layers + (args.layers % 2)
+    nlayers = args.layers
+    eps = 1e-6
     with torch.cuda.stream(stream):
         s = stream.cuda_stream
-        layers = []
-        for l in range(nlayers):
-            L = moeq.QuantLayer(w.H, w.I, w.E, w.K, w.group, w.bits_routed, w.bits_shared, device=dev)
-            L.fill(lambda e, m, c, sc, b, l=l: synth.fill_matrix_dev(w, l, e, m, c, sc, b, s), stream=s)
-            synth.router_dev(w, l, L.router_w.data_ptr(), s)
-            layers.append(L)
+        layers = build_layers(w, nlayers, dev, s)
         ws = moeq.Workspace(1, w.K, w.H, w.I, w.E, device=dev, stream=s)
-        xbuf = [torch.empty((1, w.H), dtype=torch.bfloat16, device=dev) for _ in range(2)]
-        synth.x_dev(w, 1000 * rank, 1, xbuf[0].data_ptr(), s)
-        resid = xbuf[0].float().clone()
-        outs = [L.alloc_outputs(1, logits=False, xnorm=False) for L in layers]
-        for o in outs:
-            o["resid"] = resid
+        x = torch.empty(w.H, dtype=torch.bfloat16, device=dev)
+        synth.x_dev(w, 1000 * rank, 1, x.data_ptr(), s)
+        resid = x.float().clone()
+        structs = [L.struct for L in layers]
         torch.cuda.synchronize()
 
-        def step(t):
-            l = t % nlayers
-            L, o = layers[l], outs[l]
-            o["xnorm"] = xbuf[(l + 1) % 2]
-            L.forward(xbuf[l % 2], ws, o, resid_in=resid, eps=1e-6, stream=s)
+        # a step is one layer-token; one launch walks all resident layers
+        # (x <- RMSNorm(r) of the last layer, so passes chain like decode)
+        def launch(n):
+            moeq.moe_decode_layers(structs[:n], x, resid, False, None, None, None, resid, x, eps, ws.buf, ws.nbytes, s)
 
-        # one CUDA graph per layer: the 4 kernels of a step, chained with PDL
-        graphs = []
-        for l in range(nlayers):
-            step(l)  # warm the launch path outside capture
+        launch(nlayers)
         torch.cuda.synchronize()
-        for l in range(nlayers):
-            g = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g, stream=stream):
-                step(l)
-            graphs.append(g)
-        torch.cuda.synchronize()
-        # restart the chain from a clean input
-        synth.x_dev(w, 1000 * rank, 1, xbuf[0].data_ptr(), s)
-        resid.copy_(xbuf[0].float())
         if moeq.moe_get_device_error(ws.buf, s) != moeq.MOE_OK:
-            raise RuntimeError("device error during warm-up")
-
-        for t in range(args.warmup):
-            graphs[t % nlayers].replay()
+            raise RuntimeError("device error in the first launch")
+        full, rem = divmod(args.steps, nlayers)
+        g_full = torch.cuda.CUDAGraph()
+        with torch.cuda.graph(g_full, stream=stream):
+            launch(nlayers)
+        g_rem = None
+        if rem:
+            g_rem = torch.cuda.CUDAGraph()
+            with torch.cuda.graph(g_rem, stream=stream):
+                launch(rem)
+        synth.x_dev(w, 1000 * rank, 1, x.data_ptr(), s)
+        resid.copy_(x.float())
+        for _ in range(max(1, args.warmup // nlayers)):
+            g_full.replay()
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         if world > 1:
             dist.barrier()
         torch.cuda.synchronize()
         with ClockSampler(local_rank) as clk:
             start.record(stream)
-            for t in range(args.steps):
-                graphs[(args.warmup + t) % nlayers].replay()
+            for _ in range(full):
+                g_full.replay()
+            if g_rem is not None:
+                g_rem.replay()
             end.record(stream)
             torch.cuda.synchronize()
         if world > 1:
@@ -227,81 +295,67 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
             tt = torch.tensor([ms], device=dev)
             dist.all_reduce(tt, op=dist.ReduceOp.MAX)
             ms = float(tt.item())
+        launches = full + (1 if rem else 0)
+        del g_full, g_rem
 
-        # dominant call: the expert FFN (gate/up + down kernels), timed per call
-        # with events on the launching stream over the same kind of steps
-        ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nlayers)]
-        ffn_ms = []
-        reps = max(nlayers, min(args.steps, 2000))
-        for t in range(reps):
-            l = t % nlayers
-            L, o = layers[l], outs[l]
-            xin = xbuf[l % 2]
-            moeq.moe_router_topk(xin, L.router_w, 1, w.H, w.E, w.K, False, None, o["idx"], o["w"], None, ws.buf,
-                                 ws.nbytes, s)
-            a, b = ev[l]
-            a.record(stream)
-            moeq.moe_expert_ffn_q(L.struct, xin, 1, o["idx"], o["y"], ws.buf, ws.nbytes, s)
-            b.record(stream)
-            o["xnorm"] = xbuf[(l + 1) % 2]
-            moeq.moe_combine_residual(L.struct, o["y"], o["w"], xin, resid, 1, resid, o["xnorm"], 1e-6, s)
-            if l == nlayers - 1:
-                torch.cuda.synchronize()
-                ffn_ms += [x.elapsed_time(y) for (x, y) in ev]
-        torch.cuda.synchronize()
+        # the per-call path (router_topk, expert_ffn_q, combine_residual)
+        pc_tps, ffn_avg_ms = per_call_path(w, layers, ws, dev, stream, min(args.steps, 4000))
 
-        # end to end through the public calls with host buffers
+        # end to end through the public call with host buffers: per step one
+        # layer-token, x copied in from pinned memory and r copied back out
         e2e = None
         if not args.no_e2e:
-            n_e2e = min(args.steps, 2000)
-            xh = torch.empty((n_e2e, w.H), dtype=torch.bfloat16, pin_memory=True)
+            n_e2e = min(args.steps, 4000)
             tmp = torch.empty((n_e2e, w.H), dtype=torch.bfloat16, device=dev)
             synth.x_dev(w, 50_000, n_e2e, tmp.data_ptr(), s)
             torch.cuda.synchronize()
-            xh.copy_(tmp.cpu())
+            xh = tmp.cpu().pin_memory()
             outh = torch.empty((n_e2e, w.H), dtype=torch.float32, pin_memory=True)
-            xd = torch.empty((1, w.H), dtype=torch.bfloat16, device=dev)
-            e2e_out = outs[0]
+            xd = torch.empty(w.H, dtype=torch.bfloat16, device=dev)
+            rd = torch.empty(w.H, dtype=torch.float32, device=dev)
             torch.cuda.synchronize()
             e0, e1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
             e0.record(stream)
             for t in range(n_e2e):
-                L = layers[t % nlayers]
-                xd.copy_(xh[t:t + 1], non_blocking=True)
-                e2e_out["xnorm"] = xbuf[1]
-                L.forward(xd, ws, e2e_out, resid_in=None, eps=1e-6, stream=s)
-                outh[t:t + 1].copy_(e2e_out["resid"], non_blocking=True)
+                xd.copy_(xh[t], non_blocking=True)
+                moeq.moe_decode_layers(structs[t % nlayers: t % nlayers + 1], xd, None, False, None, None, None, rd,
+                                       None, eps, ws.buf, ws.nbytes, s)
+                outh[t].copy_(rd, non_blocking=True)
             e1.record(stream)
             torch.cuda.synchronize()
             e2e_ms = e0.elapsed_time(e1)
             e2e = {"value": n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": w.H * 2,
-                   "d2h_bytes_per_step": w.H * 4, "steps": n_e2e}
+                   "d2h_bytes_per_step": w.H * 4, "steps": n_e2e,
+                   "path": "moe_decode_layers (1 layer per call) with pinned host input/output copies"}
 
     step_bytes, rec_r, rec_s = algorithmic_bytes(w)
-    ffn_bytes = w.K * rec_r + rec_s
-    ffn_avg_ms = statistics.mean(ffn_ms)
     peak, peak_src = peaks()
-    achieved = ffn_bytes / (ffn_avg_ms / 1e3) / 1e9
     tps = world * args.steps / (ms / 1e3)
+    achieved = step_bytes * args.steps / (ms / 1e3) / 1e9
+    ffn_bytes = w.K * rec_r + rec_s
+    resident = sum(L.nbytes() for L in layers)
     line = {
         "metric": "MoE-layer decode tokens/s", "value": tps, "unit": "tokens/s", "n_gpus": world,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "f32", "data": "synthetic",
         "config": {"workload": "%s: batch-1 MoE layer H%d E%d I%d top-%d + shared, %d-bit routed / %d-bit shared, "
                                "group %d" % (w.name, w.H, w.E, w.I, w.K, w.bits_routed, w.bits_shared, w.group),
-                   "batch": 1, "layers_resident": nlayers,
-                   "resident_bytes": sum(L.nbytes() for L in layers),
-                   "l2": "inputs larger than L2: steps walk %d resident layers (%.1f GB)" %
-                         (nlayers, sum(L.nbytes() for L in layers) / 1e9),
+                   "batch": 1, "layers_resident": nlayers, "resident_bytes": resident,
+                   "l2": "inputs larger than L2: each launch walks %d resident layers (%.1f GB)" %
+                         (nlayers, resident / 1e9),
                    "parallelism": "replicas" if world > 1 else "single GPU",
-                   "launch": "one CUDA graph per layer-step, 4 kernels chained with PDL"},
+                   "launch": "moe_decode_layers: one persistent kernel per %d layer-token steps, CUDA graph" % nlayers},
         "step_bytes": step_bytes,
-        "effective_gbs": step_bytes / (ms / args.steps / 1e3) / 1e9,
-        "frac_of_8tbs": step_bytes / (ms / args.steps / 1e3) / 8e12,
+        "effective_gbs": achieved,
+        "frac_of_8tbs": achieved * 1e9 / 8e12,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
-                     "traffic": None, "kernel": "moe_expert_ffn_q (gate/up + down)",
-                     "bytes_per_launch": ffn_bytes, "avg_launch_us": ffn_avg_ms * 1e3, "peak_source": peak_src},
-        "gpu_launches": 4 * args.steps,
+                     "traffic": None, "kernel": "k_decode_layers",
+                     "bytes_per_launch": step_bytes * nlayers, "avg_launch_us": ms * 1e3 / launches,
+                     "peak_source": peak_src},
+        "per_call": {"value": pc_tps, "unit": "tokens/s",
+                     "path": "moe_router_topk + moe_expert_ffn_q + moe_combine_residual, graph per step",
+                     "ffn_call_us": ffn_avg_ms * 1e3, "ffn_call_gbs": ffn_bytes / (ffn_avg_ms / 1e3) / 1e9},
+        "gpu_launches": launches,
         "clocks": clk.summary(),
     }
     if e2e is not None:

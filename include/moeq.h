@@ -74,16 +74,20 @@ typedef enum moe_status {
  * One MoE layer's resident weights (all pointers are device memory).
  *
  * Expert record (expert-major: each expert is one contiguous block, as in
- * LOOM's layout), for `bits` in {2, 4} and group size `group`:
- *   [gate codes  I x H][up codes  I x H][down codes  H x I]
- *   [gate table  I x H/group][up table  I x H/group][down table  H x I/group]
- * A code matrix [rows x cols] is row-major; in each row, element c sits in
- * byte floor(c*bits/8) at bit offset (c*bits) mod 8, lowest bits first.
- * A table entry is the bf16 pair (scale, bias) of one (row, group), scale
- * first; the dequantised weight is w = q*scale + bias with q unsigned.
- * Record size: moe_expert_bytes(H, I, bits, group); byte offsets of the six
- * parts: moe_expert_offsets. At H=4096, I=1024, 4-bit, group 64 a record is
- * 7,077,888 bytes (6.75 MiB), the per-expert size the Flash-MoE page gives.
+ * LOOM's layout), for `bits` in {2, 4} and group size `group`. A code row
+ * stores element c in byte floor(c*bits/8) at bit offset (c*bits) mod 8,
+ * lowest bits first; a table row stores one bf16 pair (scale, bias) per
+ * group of `group` inputs, scale first; the dequantised weight is
+ * w = q*scale + bias with q unsigned. The record is laid out so that the
+ * rows a kernel needs together are adjacent in memory:
+ *   I gate/up units, unit i (U bytes) =
+ *       [gate code row i][up code row i][gate table row i][up table row i]
+ *   then H/4 down blocks, block b (D bytes) =
+ *       [down code rows 4b..4b+3][down table rows 4b..4b+3]
+ * with gate/up rows of H inputs and down rows of I inputs. moe_expert_layout
+ * gives U, D and the offsets; moe_pack_expert writes a record. At H=4096,
+ * I=1024, 4-bit, group 64 a record is 7,077,888 bytes (6.75 MiB), the
+ * per-expert size the Flash-MoE page gives ("SSD Expert Streaming").
  */
 typedef struct moe_layer_q {
   int H;           /* hidden size; H*bits/8 and I*bits/8 multiples of 16 */
@@ -102,10 +106,14 @@ typedef struct moe_layer_q {
 /* Bytes of one expert record (see moe_layer_q); 0 for unsupported args. */
 size_t moe_expert_bytes(int H, int I, int bits, int group);
 
-/* Byte offsets within one expert record of: off[0] gate codes, off[1] up
- * codes, off[2] down codes, off[3] gate table, off[4] up table, off[5] down
- * table. */
-moe_status moe_expert_offsets(int H, int I, int bits, int group, size_t off[6]);
+/* Layout of one expert record (see moe_layer_q):
+ *   lay[0] U, bytes of one gate/up unit
+ *   lay[1] byte offset of the first down block (= I * U)
+ *   lay[2] D, bytes of one down block
+ *   lay[3] rows per down block (4)
+ *   lay[4] bytes of one gate/up code row (H*bits/8): the up row's offset in a unit
+ *   lay[5] bytes of one down code row (I*bits/8) */
+moe_status moe_expert_layout(int H, int I, int bits, int group, size_t lay[6]);
 
 /* Workspace bytes for calls on up to B tokens of this layer shape. */
 size_t moe_workspace_bytes(int B, int K, int H, int I, int E);
@@ -130,6 +138,17 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* bias_bf16,
                       int rows, int cols, int bits, int group,
                       void* packed_out, void* sb_out, void* ws, void* stream);
+
+/*
+ * moe_pack_expert -- pack the gate [I,H], up [I,H] and down [H,I] code
+ * matrices of one expert (u8 codes, bf16 scale/bias [rows, cols/group]) into
+ * one expert record at record_out (moe_expert_bytes(H, I, bits, group)
+ * bytes), with the same packing as moe_pack_q. ws as in moe_pack_q.
+ */
+moe_status moe_pack_expert(const uint8_t* codes_gate, const void* scale_gate_bf16, const void* bias_gate_bf16,
+                           const uint8_t* codes_up, const void* scale_up_bf16, const void* bias_up_bf16,
+                           const uint8_t* codes_down, const void* scale_down_bf16, const void* bias_down_bf16,
+                           int H, int I, int bits, int group, void* record_out, void* ws, void* stream);
 
 /*
  * moe_router_topk -- router GEMV + softmax + top-K for B tokens.

@@ -45,10 +45,11 @@ _SIGS = {
     "moe_abi_version": (_INT, []),
     "moe_status_str": (ctypes.c_char_p, [_INT]),
     "moe_expert_bytes": (_SZ, [_INT, _INT, _INT, _INT]),
-    "moe_expert_offsets": (_INT, [_INT, _INT, _INT, _INT, ctypes.POINTER(_SZ)]),
+    "moe_expert_layout": (_INT, [_INT, _INT, _INT, _INT, ctypes.POINTER(_SZ)]),
     "moe_workspace_bytes": (_SZ, [_INT, _INT, _INT, _INT, _INT]),
     "moe_workspace_init": (_INT, [_VP, _SZ, _VP]),
     "moe_pack_q": (_INT, [_VP, _VP, _VP, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP]),
+    "moe_pack_expert": (_INT, [_VP] * 9 + [_INT, _INT, _INT, _INT, _VP, _VP, _VP]),
     "moe_router_topk": (_INT, [_VP, _VP, _INT, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_expert_ffn_q": (_INT, [_LP, _VP, _INT, _VP, _VP, _VP, _SZ, _VP]),
     "moe_combine_residual": (_INT, [_LP, _VP, _VP, _VP, _VP, _INT, _VP, _VP, _FLT, _VP]),
@@ -108,10 +109,11 @@ def moe_expert_bytes(H: int, I: int, bits: int, group: int) -> int:
     return int(lib().moe_expert_bytes(H, I, bits, group))
 
 
-def moe_expert_offsets(H: int, I: int, bits: int, group: int):
-    off = (ctypes.c_size_t * 6)()
-    _check(lib().moe_expert_offsets(H, I, bits, group, off), "moe_expert_offsets")
-    return [int(v) for v in off]
+def moe_expert_layout(H: int, I: int, bits: int, group: int):
+    """[unit bytes U, down offset, down block bytes D, rows per block, gate/up code row bytes, down code row bytes]"""
+    lay = (ctypes.c_size_t * 6)()
+    _check(lib().moe_expert_layout(H, I, bits, group, lay), "moe_expert_layout")
+    return [int(v) for v in lay]
 
 
 def moe_workspace_bytes(B: int, K: int, H: int, I: int, E: int) -> int:
@@ -129,6 +131,13 @@ def moe_pack_q(codes, scale_bf16, bias_bf16, rows: int, cols: int, bits: int, gr
                ws=None, stream=None) -> None:
     _check(lib().moe_pack_q(_ptr(codes), _ptr(scale_bf16), _ptr(bias_bf16), rows, cols, bits, group,
                             _ptr(packed_out), _ptr(sb_out), _ptr(ws), _stream(stream)), "moe_pack_q")
+
+
+def moe_pack_expert(gate, up, down, H: int, I: int, bits: int, group: int, record_out, ws=None, stream=None) -> None:
+    """gate/up/down = (codes u8, scale bf16, bias bf16) device buffers."""
+    args = [_ptr(t) for m in (gate, up, down) for t in m]
+    _check(lib().moe_pack_expert(*args, H, I, bits, group, _ptr(record_out), _ptr(ws), _stream(stream)),
+           "moe_pack_expert")
 
 
 def moe_router_topk(x_bf16, router_w_bf16, B: int, H: int, E: int, K: int, renorm: bool, forced_idx, idx_out, w_out,

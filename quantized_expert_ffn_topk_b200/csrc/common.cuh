@@ -35,6 +35,27 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   return (uint16_t)(u >> 16);
 }
 
+// Geometry of one expert record (bytes). Gate/up unit i at i*U:
+// [gate code row][up code row][gate table row][up table row]; down block b at
+// down_off + b*D: [4 down code rows][their 4 table rows].
+constexpr int kRowsPerDownBlock = 4;
+struct RecGeom {
+  uint32_t U, rowb_h, sbb_h;  // gate/up unit, code row of H inputs, table row
+  uint32_t D, rowb_i, sbb_i;  // down block, code row of I inputs, table row
+  unsigned long long down_off;
+};
+__host__ __device__ inline RecGeom rec_geom(int H, int I, int bits, int group) {
+  RecGeom g;
+  g.rowb_h = (uint32_t)(H * bits / 8);
+  g.sbb_h = (uint32_t)(H / group * 4);
+  g.U = 2 * (g.rowb_h + g.sbb_h);
+  g.rowb_i = (uint32_t)(I * bits / 8);
+  g.sbb_i = (uint32_t)(I / group * 4);
+  g.D = kRowsPerDownBlock * (g.rowb_i + g.sbb_i);
+  g.down_off = (unsigned long long)I * g.U;
+  return g;
+}
+
 // Programmatic dependent launch (PTX griddepcontrol; no-ops when the launch
 // did not ask for it).
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
@@ -139,6 +160,9 @@ __device__ __forceinline__ void mbar_arrive_expect_tx(uint64_t* bar, uint32_t by
 __device__ __forceinline__ void mbar_arrive(uint64_t* bar) {
   asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0];" ::"r"(smem_u32(bar)) : "memory");
 }
+__device__ __forceinline__ void mbar_arrive_cnt(uint64_t* bar, uint32_t count) {
+  asm volatile("mbarrier.arrive.shared::cta.b64 _, [%0], %1;" ::"r"(smem_u32(bar)), "r"(count) : "memory");
+}
 __device__ __forceinline__ bool mbar_try_wait(uint64_t* bar, uint32_t parity) {
   uint32_t ok;
   asm volatile(
@@ -164,14 +188,24 @@ __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {
   return v;
 }
 
+// Grid-wide arrival: a release-ordered reduction (no returned value, so the
+// arriving thread does not wait for the round trip). Writes of the whole CTA
+// that were ordered before it by a CTA barrier become visible first.
+__device__ __forceinline__ void arrive_release_gpu(unsigned* counter) {
+  asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
+}
+
 // Wait budget for every spin in the library: ~1 s of SM clock cycles.
 constexpr long long kWaitBudgetCycles = 2000000000LL;
 
 // Bounded wait for an mbarrier phase; false on timeout or when `abort` is set.
+// Waiting warps back off with __nanosleep so that they leave the issue slots
+// to the warps that have work.
 __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
+    __nanosleep(64);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
     if (clock64() - t0 > kWaitBudgetCycles) return false;

@@ -94,25 +94,13 @@ inline WsLayout ws_layout(int B, int K, int H, int I, int E) {
   return l;
 }
 
-inline void expert_offsets(int H, int I, int bits, int group, size_t off[6]) {
-  const size_t hi = (size_t)H * I;
-  const size_t cb = hi * bits / 8;          // one matrix of codes
-  const size_t tb = hi / group * 4;         // one (scale, bias) table
-  off[0] = 0;
-  off[1] = cb;
-  off[2] = 2 * cb;
-  off[3] = 3 * cb;
-  off[4] = 3 * cb + tb;
-  off[5] = 3 * cb + 2 * tb;
-}
-
 moe_status check_layer(const moe_layer_q* L) {
   if (!L) return MOE_ERR_INVALID_ARG;
   if (L->H <= 0 || L->I <= 0 || L->E <= 0 || L->K <= 0) return MOE_ERR_INVALID_ARG;
   if (L->K > MOEQ_MAX_K || L->K > L->E) return MOE_ERR_INVALID_ARG;
   if (!bits_ok(L->bits_routed) || !bits_ok(L->bits_shared) || !group_ok(L->group)) return MOE_ERR_UNSUPPORTED;
   for (int bits : {L->bits_routed, L->bits_shared})
-    if (!cols_ok(L->H, bits, L->group) || !cols_ok(L->I, bits, L->group)) return MOE_ERR_UNSUPPORTED;
+    if (moe_expert_bytes(L->H, L->I, bits, L->group) == 0) return MOE_ERR_UNSUPPORTED;
   if (!L->experts || !L->shared || !L->router_w) return MOE_ERR_INVALID_ARG;
   if (!aligned16(L->experts) || !aligned16(L->shared) || !aligned16(L->router_w)) return MOE_ERR_ALIGN;
   if (L->shared_gate_w && !aligned16(L->shared_gate_w)) return MOE_ERR_ALIGN;
@@ -146,14 +134,21 @@ const char* moe_status_str(moe_status s) {
 size_t moe_expert_bytes(int H, int I, int bits, int group) {
   if (H <= 0 || I <= 0 || !bits_ok(bits) || !group_ok(group)) return 0;
   if (!cols_ok(H, bits, group) || !cols_ok(I, bits, group)) return 0;
+  if ((H / group) % 2 != 0) return 0;  // a gate/up unit must stay a multiple of 16 bytes
   const size_t hi = 3 * (size_t)H * I;
   return hi * bits / 8 + hi / group * 4;
 }
 
-moe_status moe_expert_offsets(int H, int I, int bits, int group, size_t off[6]) {
-  if (!off) return MOE_ERR_INVALID_ARG;
+moe_status moe_expert_layout(int H, int I, int bits, int group, size_t lay[6]) {
+  if (!lay) return MOE_ERR_INVALID_ARG;
   if (moe_expert_bytes(H, I, bits, group) == 0) return MOE_ERR_UNSUPPORTED;
-  expert_offsets(H, I, bits, group, off);
+  const RecGeom g = rec_geom(H, I, bits, group);
+  lay[0] = g.U;
+  lay[1] = (size_t)g.down_off;
+  lay[2] = g.D;
+  lay[3] = kRowsPerDownBlock;
+  lay[4] = g.rowb_h;
+  lay[5] = g.rowb_i;
   return MOE_OK;
 }
 
@@ -188,12 +183,58 @@ moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* 
   unsigned g1 = (unsigned)std::min<int64_t>((nchunks + 255) / 256, maxg);
   unsigned g2 = (unsigned)std::min<int64_t>((nsb + 255) / 256, maxg);
   WsCtrl* ctrl = reinterpret_cast<WsCtrl*>(ws);
+  const size_t rowb = (size_t)cols * bits / 8, sbb = (size_t)(cols / group) * 4;
+  const RowPlace pc{reinterpret_cast<unsigned char*>(packed_out), rows, rowb, rowb * rows};
+  const RowPlace ps{reinterpret_cast<unsigned char*>(sb_out), rows, sbb, sbb * rows};
+  const int cpr = (int)(rowb / 16);
   if (bits == 4)
-    k_pack_codes<4><<<g1, 256, 0, s>>>(codes, nchunks, reinterpret_cast<uint8_t*>(packed_out), ctrl);
+    k_pack_codes<4><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
   else
-    k_pack_codes<2><<<g1, 256, 0, s>>>(codes, nchunks, reinterpret_cast<uint8_t*>(packed_out), ctrl);
+    k_pack_codes<2><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
   k_pack_sb<<<g2, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(scale_bf16), reinterpret_cast<const uint16_t*>(bias_bf16),
-                               nsb, reinterpret_cast<uint32_t*>(sb_out));
+                               nsb, cols / group, ps);
+  return launch_status();
+}
+
+moe_status moe_pack_expert(const uint8_t* codes_gate, const void* scale_gate_bf16, const void* bias_gate_bf16,
+                           const uint8_t* codes_up, const void* scale_up_bf16, const void* bias_up_bf16,
+                           const uint8_t* codes_down, const void* scale_down_bf16, const void* bias_down_bf16,
+                           int H, int I, int bits, int group, void* record_out, void* ws, void* stream) {
+  const void* ptrs[10] = {codes_gate, scale_gate_bf16, bias_gate_bf16, codes_up, scale_up_bf16, bias_up_bf16,
+                          codes_down, scale_down_bf16, bias_down_bf16, record_out};
+  for (const void* q : ptrs) {
+    if (!q) return MOE_ERR_INVALID_ARG;
+    if (!aligned16(q)) return MOE_ERR_ALIGN;
+  }
+  if (ws && !aligned16(ws)) return MOE_ERR_ALIGN;
+  if (moe_expert_bytes(H, I, bits, group) == 0) return MOE_ERR_UNSUPPORTED;
+  cudaStream_t s = (cudaStream_t)stream;
+  WsCtrl* ctrl = reinterpret_cast<WsCtrl*>(ws);
+  const RecGeom g = rec_geom(H, I, bits, group);
+  unsigned char* rec = reinterpret_cast<unsigned char*>(record_out);
+  const unsigned maxg = (unsigned)num_sms() * 8;
+  auto launch = [&](const uint8_t* codes, const void* sc, const void* bi, int rows, int cols, RowPlace pc, RowPlace ps) {
+    const int64_t nchunks = (int64_t)rows * cols * bits / 128;
+    const int64_t nsb = (int64_t)rows * (cols / group);
+    const unsigned g1 = (unsigned)std::min<int64_t>((nchunks + 255) / 256, maxg);
+    const unsigned g2 = (unsigned)std::min<int64_t>((nsb + 255) / 256, maxg);
+    const int cpr = cols * bits / 128;
+    if (bits == 4)
+      k_pack_codes<4><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
+    else
+      k_pack_codes<2><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
+    k_pack_sb<<<g2, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(sc), reinterpret_cast<const uint16_t*>(bi), nsb,
+                                 cols / group, ps);
+  };
+  // gate and up: one row per unit
+  launch(codes_gate, scale_gate_bf16, bias_gate_bf16, I, H, RowPlace{rec, I, g.U, (size_t)g.U * I},
+         RowPlace{rec + 2 * g.rowb_h, I, g.U, (size_t)g.U * I});
+  launch(codes_up, scale_up_bf16, bias_up_bf16, I, H, RowPlace{rec + g.rowb_h, I, g.U, (size_t)g.U * I},
+         RowPlace{rec + 2 * g.rowb_h + g.sbb_h, I, g.U, (size_t)g.U * I});
+  // down: blocks of four rows
+  unsigned char* dn = rec + g.down_off;
+  launch(codes_down, scale_down_bf16, bias_down_bf16, H, I, RowPlace{dn, kRowsPerDownBlock, g.rowb_i, g.D},
+         RowPlace{dn + kRowsPerDownBlock * g.rowb_i, kRowsPerDownBlock, g.sbb_i, g.D});
   return launch_status();
 }
 
@@ -239,9 +280,8 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
   p.experts = reinterpret_cast<const uint8_t*>(L->experts);
   p.shared = reinterpret_cast<const uint8_t*>(L->shared);
   p.rec_r = moe_expert_bytes(L->H, L->I, L->bits_routed, L->group);
-  p.rec_s = moe_expert_bytes(L->H, L->I, L->bits_shared, L->group);
-  expert_offsets(L->H, L->I, L->bits_routed, L->group, p.off_r);
-  expert_offsets(L->H, L->I, L->bits_shared, L->group, p.off_s);
+  p.geo_r = rec_geom(L->H, L->I, L->bits_routed, L->group);
+  p.geo_s = rec_geom(L->H, L->I, L->bits_shared, L->group);
   p.x = reinterpret_cast<const uint16_t*>(x_bf16);
   p.idx = idx;
   WsLayout wl = ws_layout(B, L->K, L->H, L->I, L->E);
@@ -333,21 +373,24 @@ bool stack_plan(StackParams& p, int G) {
   p.need4 = (p.bits_r == 4 || p.bits_s == 4);
   p.need2 = (p.bits_r == 2 || p.bits_s == 2);
   p.sm_xs = take((size_t)H * 2);
-  p.sm_img4 = take(p.need4 ? (size_t)H * 2 : 0);
-  p.sm_tab4 = take(p.need4 ? (size_t)(H / Img<4>::HC) * 8 : 0);
-  p.sm_img2 = take(p.need2 ? (size_t)H * 2 : 0);
-  p.sm_tab2 = take(p.need2 ? (size_t)(H / Img<2>::HC) * 8 : 0);
-  p.himg_stride = (int)align_up((size_t)I * 2, 128);
-  p.htab_stride = (int)align_up((size_t)(I / Img<4>::HC) * 8, 128);
+  p.sm_img4 = take(p.need4 ? img_bytes(H) : 0);
+  p.sm_tab4 = take(p.need4 ? tab_bytes(H, 4) : 0);
+  p.sm_inv4 = take(p.need4 ? inv_bytes(H, 4) : 0);
+  p.sm_img2 = take(p.need2 ? img_bytes(H) : 0);
+  p.sm_tab2 = take(p.need2 ? tab_bytes(H, 2) : 0);
+  p.sm_inv2 = take(p.need2 ? inv_bytes(H, 2) : 0);
+  p.himg_stride = (int)align_up(img_bytes(I), 128);
+  p.htab_stride = (int)align_up(tab_bytes(I, 4), 128);  // 4-bit has the most chunks
+  p.hinv_stride = (int)align_up(inv_bytes(I, 4), 128);
   p.sm_himg = take((size_t)p.himg_stride * (K + 1));
   p.sm_htab = take((size_t)p.htab_stride * (K + 1));
-  p.nblk_max = strided_count(0, G, H / kDnBlk);
-  const int bmax = std::max(p.bits_r, p.bits_s);
-  p.dblk_bytes = (int)align_up((size_t)kDnBlk * ((size_t)I * bmax / 8 + (size_t)I / p.G * 4), 16);
-  p.sm_regc = take((size_t)p.dblk_bytes * p.nblk_max * (K + 1));
-  const size_t unit = std::max((size_t)H, 2 * ((size_t)H * bmax / 8) + 2 * ((size_t)H / p.G * 4));
+  p.sm_hinv = take((size_t)p.hinv_stride * (K + 1));
+  const int nblk_max = (H / kDnBlk + G - 1) / G;
+  p.regc_slot_bytes = (int)align_up((size_t)nblk_max * std::max(p.geo_r.D, p.geo_s.D), 128);
+  p.sm_regc = take((size_t)p.regc_slot_bytes * (K + 1));
+  const size_t unit = std::max((size_t)2 * H * 2, (size_t)kPiecesPerItem * std::max(p.geo_r.U, p.geo_s.U));
   p.slot_bytes = (int)align_up(unit, 128);
-  const size_t budget = 227 * 1024 - 2048;  // leave room for the static shared memory
+  const size_t budget = 227 * 1024 - 6 * 1024;  // leave room for the static shared memory
   if (o + (size_t)p.slot_bytes * 2 > budget) return false;
   p.nslot = (int)std::min<size_t>(kMaxSlots, (budget - o) / p.slot_bytes);
   p.sm_ring = take((size_t)p.slot_bytes * p.nslot);
@@ -381,8 +424,12 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   if (!ws) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_workspace_bytes(1, L0.K, L0.H, L0.I, L0.E)) return MOE_ERR_WORKSPACE;
   const int G = num_sms();
-  if (L0.E > 1024 || strided_count(0, G, L0.E) > kMaxRouterRowsPerCta) return MOE_ERR_UNSUPPORTED;
-  if ((L0.H / L0.group) % 4 != 0 || L0.H % (2 * 16) != 0) return MOE_ERR_UNSUPPORTED;
+  auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
+  if (L0.E > 1024 || cdiv(L0.E, G) > kMaxRouterRowsPerCta) return MOE_ERR_UNSUPPORTED;
+  if (cdiv(cdiv(L0.E, G), 2) + cdiv(cdiv(L0.I, G), kPiecesPerItem) + cdiv(cdiv(L0.K * L0.I, G), kPiecesPerItem) + L0.K >
+      kMaxItems)
+    return MOE_ERR_UNSUPPORTED;
+  if (L0.H % 32 != 0) return MOE_ERR_UNSUPPORTED;
 
   StackParams p{};
   for (int l = 0; l < n_layers; ++l) {
@@ -400,11 +447,8 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   p.bits_r = L0.bits_routed;
   p.bits_s = L0.bits_shared;
   p.rec_r = moe_expert_bytes(p.H, p.I, p.bits_r, p.G);
-  size_t off[6];
-  expert_offsets(p.H, p.I, p.bits_r, p.G, off);
-  for (int i = 0; i < 6; ++i) p.off_r[i] = (uint32_t)off[i];
-  expert_offsets(p.H, p.I, p.bits_s, p.G, off);
-  for (int i = 0; i < 6; ++i) p.off_s[i] = (uint32_t)off[i];
+  p.geo_r = rec_geom(p.H, p.I, p.bits_r, p.G);
+  p.geo_s = rec_geom(p.H, p.I, p.bits_s, p.G);
   p.x_in = reinterpret_cast<const uint16_t*>(x_bf16);
   p.resid_in = resid_in;
   p.forced = forced_idx;

@@ -9,31 +9,33 @@
 //
 //   stage x_l      every CTA: x_l = bf16(RMSNorm(r_l)) (l > 0) into shared
 //                  memory, plus the fp16 image the dequant dots read
-//   router         CTA c owns router rows c, c+G, ...; writes its logits
+//   router         CTA c owns a contiguous range of router rows
 //   sync 1         all logits written
 //   top-K          the producer warp of every CTA selects the K experts
-//   gate/up        shared-expert units (slot K, row i) and routed units
-//                  (slot k, row i), strided over the CTAs; h to global
+//   gate/up        CTA c owns a contiguous range of the shared expert's units
+//                  and of the routed units (slot-major); h to global memory
 //   sync 2         all of h written
-//   down+combine   CTA c owns output row blocks c, c+G, ... (4 rows): for
-//                  every slot the row dot with h_k, weighted by the routing
+//   down+combine   CTA c owns a contiguous range of 4-row output blocks: for
+//                  every slot the rows' dot with h_k, weighted by the routing
 //                  weight (shared: gamma), plus the residual
 //   sync 3         r_{l+1} and its sum of squares complete
 //
-// Warp roles: warps 0..7 compute, warp 8 moves data. The producer streams
-// every weight byte of the CTA's share into shared memory with bulk async
-// copies (cp.async.bulk, completion on mbarriers): router half-rows and
-// gate/up units through a ring of slots, down-projection row blocks into a
-// region that is filled as soon as the experts are known, so down weights
-// arrive while gate/up still computes. Router rows and shared-expert units of
-// layer l+1 enter the ring while layer l finishes. Grid-wide syncs are
-// monotonic arrival counters in the workspace; every wait (counter or
-// mbarrier) gives up after about a second, sets MOE_ERR_TIMEOUT and lets the
-// kernel run to its end without further work.
+// Warp roles: warps 0..7 compute, warp 8 moves data. Because the record keeps
+// a unit's gate/up rows and tables adjacent, and a CTA's ranges are
+// contiguous, every weight byte the CTA needs arrives in few large bulk
+// copies (cp.async.bulk, completion on mbarriers): ring items of up to four
+// units or two router rows (about 16-18 KB), and one copy per slot of the
+// CTA's down blocks into a region that fills as soon as the experts are
+// known. A bulk copy's cost on this part is nearly fixed per copy below
+// ~16 KB, so size, not count in flight, sets the rate. Router rows and
+// shared-expert units of layer l+1 enter the ring while layer l finishes.
+// Grid-wide syncs are monotonic arrival counters in the workspace (release
+// reductions, acquire polls); every wait gives up after about a second, sets
+// MOE_ERR_TIMEOUT and lets the kernel run to its end without further work.
 #pragma once
 
 #include "common.cuh"
-#include "ffn.cuh"
+#include "dqdot.cuh"
 #include "router.cuh"
 
 namespace moeq {
@@ -42,11 +44,14 @@ constexpr int kStackMaxLayers = 64;
 constexpr int kCWarps = 8;                          // compute warps
 constexpr int kCThreads = kCWarps * 32;
 constexpr int kStackThreads = kCThreads + 32;       // + producer warp
-constexpr int kDnBlk = 4;                           // rows per down block
-constexpr int kMaxSlots = 32;
+constexpr int kDnBlk = kRowsPerDownBlock;           // rows per down block
+constexpr int kMaxSlots = 16;
 constexpr int kMaxRouterRowsPerCta = 8;
+constexpr int kPiecesPerItem = 4;                   // units, or router half-rows, per ring item
+constexpr int kMaxItems = 32;                       // ring items per layer per CTA
+constexpr int kMaxPieces = kMaxItems * kPiecesPerItem;
 
-enum { kItemRouterHalf = 0, kItemGateUp = 1, kItemZero = 2 };
+enum { kItemRouter = 0, kItemGateUp = 1, kItemZero = 2 };
 
 struct StackLayerPtrs {
   const uint8_t* experts;
@@ -60,7 +65,7 @@ struct StackParams {
   int n_layers;
   int H, I, E, K, G, bits_r, bits_s;
   unsigned long long rec_r;
-  uint32_t off_r[6], off_s[6];
+  RecGeom geo_r, geo_s;
   const uint16_t* x_in;     // [H]
   const float* resid_in;    // [H] or null
   const int32_t* forced;    // [n_layers, K] or null
@@ -76,118 +81,140 @@ struct StackParams {
   float* r;                 // [H]
   float* ss;                // [kStackMaxLayers]
   // shared-memory plan (byte offsets into the dynamic buffer)
-  int sm_xs, sm_img4, sm_tab4, sm_img2, sm_tab2, sm_himg, sm_htab, himg_stride, htab_stride;
-  int sm_ring, slot_bytes, nslot, sm_regc, dblk_bytes, nblk_max;
+  int sm_xs, sm_img4, sm_tab4, sm_inv4, sm_img2, sm_tab2, sm_inv2;
+  int sm_himg, sm_htab, sm_hinv, himg_stride, htab_stride, hinv_stride;
+  int sm_ring, slot_bytes, nslot, sm_regc, regc_slot_bytes;
   int need4, need2;
 };
 
-__host__ __device__ inline int strided_count(int c, int G, int n) { return n > c ? (n - c - 1) / G + 1 : 0; }
+// CTA c's share [lo, hi) of n items split evenly over G CTAs.
+__host__ __device__ inline int share_lo(int c, int G, int n) { return (int)((long long)n * c / G); }
 
-// ---- producer pieces ---------------------------------------------------------
+// The static item plan of one CTA (identical for every layer): router items
+// of up to two rows, shared-expert items of up to four units, routed items of
+// up to four units that never straddle two slots.
+struct ItemPlan {
+  int n_items, n_router_items, n_pre;     // n_pre: router + shared items
+  int n_pieces, n_router_pieces;
+  int kind[kMaxItems];                    // kItemRouter or kItemGateUp
+  int k[kMaxItems];                       // slot (routed), K (shared)
+  int first[kMaxItems];                   // first router row / unit row of the item
+  int npieces[kMaxItems];
+  int piece0[kMaxItems];                  // index of the item's first piece
+  int r0, nr;                             // router rows [r0, r0+nr)
+  int b0, nblk;                           // down blocks [b0, b0+nblk)
+};
+
+__device__ void make_plan(const StackParams& p, ItemPlan& P) {
+  const int c = blockIdx.x, G = gridDim.x;
+  int n = 0, pc = 0;
+  P.r0 = share_lo(c, G, p.E);
+  P.nr = share_lo(c + 1, G, p.E) - P.r0;
+  for (int r = 0; r < P.nr; r += 2) {
+    P.kind[n] = kItemRouter;
+    P.k[n] = 0;
+    P.first[n] = r;
+    P.npieces[n] = 2 * min(2, P.nr - r);
+    P.piece0[n] = pc;
+    pc += P.npieces[n];
+    ++n;
+  }
+  P.n_router_items = n;
+  P.n_router_pieces = pc;
+  const int s0 = share_lo(c, G, p.I), s1 = share_lo(c + 1, G, p.I);
+  for (int i = s0; i < s1; i += kPiecesPerItem) {
+    P.kind[n] = kItemGateUp;
+    P.k[n] = p.K;
+    P.first[n] = i;
+    P.npieces[n] = min(kPiecesPerItem, s1 - i);
+    P.piece0[n] = pc;
+    pc += P.npieces[n];
+    ++n;
+  }
+  P.n_pre = n;
+  const int u0 = share_lo(c, G, p.K * p.I), u1 = share_lo(c + 1, G, p.K * p.I);
+  for (int u = u0; u < u1;) {
+    const int k = u / p.I, i = u % p.I;
+    const int cnt = min(kPiecesPerItem, min(u1 - u, p.I - i));
+    P.kind[n] = kItemGateUp;
+    P.k[n] = k;
+    P.first[n] = i;
+    P.npieces[n] = cnt;
+    P.piece0[n] = pc;
+    pc += cnt;
+    ++n;
+    u += cnt;
+  }
+  P.n_items = n;
+  P.n_pieces = pc;
+  P.b0 = share_lo(c, G, p.H / kDnBlk);
+  P.nblk = share_lo(c + 1, G, p.H / kDnBlk) - P.b0;
+}
+
+// ---- producer pieces (lane 0 issues; the warp waits together) -------------
 
 struct Ring {
   uint64_t* full;
   uint64_t* empty;
-  int* kind;
-  int* a;
-  int* b;
-  int* last;     // per slot: sequence number of the last fill actually issued (-1: none)
+  int* last;     // per slot: item sequence number of the last fill issued (-1: none)
   unsigned char* base;
   int slot_bytes, nslot;
-  uint32_t seq;  // items issued so far
 };
 
-// Issue one ring item (lane 0 copies, the whole warp waits for the slot).
-__device__ __forceinline__ void ring_issue(Ring& R, int kind, int a, int b, const void* const* src,
-                                           const uint32_t* bytes, int ncopy, const volatile int* abort) {
-  const uint32_t slot = R.seq % R.nslot, n = R.seq / R.nslot;
+// Issue ring item `it` of layer l as ring sequence number `seq`.
+__device__ void issue_item(const StackParams& p, const ItemPlan& P, Ring& R, int l, int it, uint32_t seq,
+                           const int* s_idx, const volatile int* abort) {
+  const int lane = threadIdx.x & 31;
+  const uint32_t slot = seq % R.nslot, fill = seq / R.nslot;
   bool ok = true;
-  if (n > 0) ok = mbar_wait(&R.empty[slot], (n - 1) & 1, abort);
-  if ((threadIdx.x & 31) == 0) {
-    if (ok) {
-      R.kind[slot] = kind;
-      R.a[slot] = a;
-      R.b[slot] = b;
-      R.last[slot] = (int)R.seq;
-      uint32_t tot = 0;
-      for (int i = 0; i < ncopy; ++i) tot += bytes[i];
-      mbar_arrive_expect_tx(&R.full[slot], tot);
-      unsigned char* dst = R.base + (size_t)slot * R.slot_bytes;
-      for (int i = 0; i < ncopy; ++i) {
-        bulk_g2s(dst, src[i], bytes[i], &R.full[slot]);
-        dst += bytes[i];
+  if (fill > 0) ok = mbar_wait(&R.empty[slot], (fill - 1) & 1, abort);
+  if (lane == 0 && ok) {
+    const void* src = nullptr;
+    uint32_t bytes = 0;
+    if (P.kind[it] == kItemRouter) {
+      src = p.L[l].router_w + (size_t)(P.r0 + P.first[it]) * p.H;
+      bytes = (uint32_t)(P.npieces[it] / 2) * (uint32_t)p.H * 2;
+    } else if (P.k[it] == p.K) {
+      src = p.L[l].shared + (size_t)P.first[it] * p.geo_s.U;
+      bytes = (uint32_t)P.npieces[it] * p.geo_s.U;
+    } else {
+      const int e = s_idx[P.k[it]];
+      if (e >= 0) {
+        src = p.L[l].experts + (size_t)e * p.rec_r + (size_t)P.first[it] * p.geo_r.U;
+        bytes = (uint32_t)P.npieces[it] * p.geo_r.U;
       }
+    }
+    R.last[slot] = (int)seq;
+    mbar_arrive_expect_tx(&R.full[slot], bytes);
+    if (bytes) bulk_g2s(R.base + (size_t)slot * R.slot_bytes, src, bytes, &R.full[slot]);
+  }
+  __syncwarp();
+}
+
+// The CTA's down blocks of slots [k0, k1): one copy per slot, arming `bar`.
+__device__ void issue_down(const StackParams& p, const ItemPlan& P, unsigned char* regc, int l, int k0, int k1,
+                           const int* s_idx, uint64_t* bar) {
+  if ((threadIdx.x & 31) == 0) {
+    uint32_t tot = 0;
+    for (int k = k0; k < k1; ++k)
+      if (k == p.K || s_idx[k] >= 0) tot += (uint32_t)P.nblk * (k == p.K ? p.geo_s.D : p.geo_r.D);
+    mbar_arrive_expect_tx(bar, tot);
+    for (int k = k0; k < k1; ++k) {
+      const bool shared = (k == p.K);
+      if (!shared && s_idx[k] < 0) continue;
+      const RecGeom& g = shared ? p.geo_s : p.geo_r;
+      const uint8_t* rec = shared ? p.L[l].shared : p.L[l].experts + (size_t)s_idx[k] * p.rec_r;
+      if (P.nblk > 0)
+        bulk_g2s(regc + (size_t)k * p.regc_slot_bytes, rec + g.down_off + (size_t)P.b0 * g.D, (uint32_t)P.nblk * g.D,
+                 bar);
     }
   }
   __syncwarp();
-  R.seq++;
-}
-
-// Router half-rows and shared-expert gate/up units of layer l (they do not
-// depend on the routing).
-__device__ void issue_pre(const StackParams& p, Ring& R, int l, int nr, int nsu, const volatile int* abort) {
-  const int c = blockIdx.x, G = gridDim.x;
-  const uint32_t half_bytes = (uint32_t)p.H;  // H/2 bf16
-  for (int m = 0; m < nr; ++m) {
-    const int e = c + G * m;
-    for (int hh = 0; hh < 2; ++hh) {
-      const void* src[1] = {p.L[l].router_w + (size_t)e * p.H + (size_t)hh * (p.H / 2)};
-      const uint32_t by[1] = {half_bytes};
-      ring_issue(R, kItemRouterHalf, m, hh, src, by, 1, abort);
-    }
-  }
-  const uint32_t rowb = (uint32_t)(p.H * p.bits_s / 8), sbb = (uint32_t)(p.H / p.G * 4);
-  for (int m = 0; m < nsu; ++m) {
-    const int i = c + G * m;
-    const uint8_t* rec = p.L[l].shared;
-    const void* src[4] = {rec + p.off_s[0] + (size_t)i * rowb, rec + p.off_s[1] + (size_t)i * rowb,
-                          rec + p.off_s[3] + (size_t)i * sbb, rec + p.off_s[4] + (size_t)i * sbb};
-    const uint32_t by[4] = {rowb, rowb, sbb, sbb};
-    ring_issue(R, kItemGateUp, p.K, i, src, by, 4, abort);
-  }
-}
-
-// Routed gate/up units of layer l (needs the experts in s_idx).
-__device__ void issue_routed(const StackParams& p, Ring& R, int l, int nru, const int* s_idx, const volatile int* abort) {
-  const int c = blockIdx.x, G = gridDim.x;
-  const uint32_t rowb = (uint32_t)(p.H * p.bits_r / 8), sbb = (uint32_t)(p.H / p.G * 4);
-  for (int m = 0; m < nru; ++m) {
-    const int u = c + G * m;
-    const int k = u / p.I, i = u % p.I;
-    const int e = s_idx[k];
-    if (e < 0) {
-      ring_issue(R, kItemZero, k, i, nullptr, nullptr, 0, abort);
-      continue;
-    }
-    const uint8_t* rec = p.L[l].experts + (size_t)e * p.rec_r;
-    const void* src[4] = {rec + p.off_r[0] + (size_t)i * rowb, rec + p.off_r[1] + (size_t)i * rowb,
-                          rec + p.off_r[3] + (size_t)i * sbb, rec + p.off_r[4] + (size_t)i * sbb};
-    const uint32_t by[4] = {rowb, rowb, sbb, sbb};
-    ring_issue(R, kItemGateUp, k, i, src, by, 4, abort);
-  }
-}
-
-// Down-projection row blocks of slot k (expert record `rec`, `bits`) into the
-// down region; lane 0 only. Returns the bytes issued.
-__device__ uint32_t issue_down_slot(const StackParams& p, unsigned char* regc, int k, const uint8_t* rec,
-                                    const uint32_t* off, int bits, int nblk, uint64_t* bar, bool issue) {
-  const int c = blockIdx.x, G = gridDim.x;
-  const uint32_t rowb = (uint32_t)(p.I * bits / 8), sbb = (uint32_t)(p.I / p.G * 4);
-  uint32_t tot = 0;
-  for (int m = 0; m < nblk; ++m) {
-    const int i0 = (c + G * m) * kDnBlk;
-    unsigned char* dst = regc + ((size_t)k * p.nblk_max + m) * p.dblk_bytes;
-    if (issue) {
-      bulk_g2s(dst, rec + off[2] + (size_t)i0 * rowb, kDnBlk * rowb, bar);
-      bulk_g2s(dst + kDnBlk * rowb, rec + off[5] + (size_t)i0 * sbb, kDnBlk * sbb, bar);
-    }
-    tot += kDnBlk * (rowb + sbb);
-  }
-  return tot;
 }
 
 // Top-K (or forced picks) of layer l by the producer warp, from the logits
-// every CTA published. Writes s_idx (-1 for an invalid forced index) and s_w.
+// every CTA published; registers only. Writes s_idx (-1 for an invalid pick)
+// and s_w.
 __device__ void producer_topk(const StackParams& p, int l, int* s_idx, float* s_w) {
   const int lane = threadIdx.x & 31;
   constexpr int MAXV = 32;  // E <= 1024
@@ -202,60 +229,64 @@ __device__ void producer_topk(const StackParams& p, int l, int* s_idx, float* s_
   mx = warp_max(mx);
   float z = 0.f;
 #pragma unroll
-  for (int j = 0; j < MAXV; ++j)
-    if (lane + 32 * j < p.E) z += expf(v[j] - mx);
+  for (int j = 0; j < MAXV; ++j) z += (lane + 32 * j < p.E) ? __expf(v[j] - mx) : 0.f;
   z = warp_sum(z);
-  int picked[MOEQ_MAX_K];
   const int32_t* forced = p.forced ? p.forced + (size_t)l * p.K : nullptr;
+  int pick_e = -1;     // lane k (< K) ends up holding pick k
+  float pick_l = 0.f;  // and its logit
   for (int k = 0; k < p.K; ++k) {
+    int bi;
+    float best;
     if (forced) {
-      const int e = forced[k];
-      picked[k] = (e >= 0 && e < p.E) ? e : -1;
-      if (picked[k] < 0 && lane == 0) set_error(p.ctrl, MOE_ERR_INDEX);
-      continue;
-    }
-    float best = -INFINITY;
-    int bi = 0x7FFFFFFF;
+      bi = forced[k];
+      const bool okf = bi >= 0 && bi < p.E;
+      best = okf ? __ldcg(p.logits + bi) : -INFINITY;
+      if (!okf) bi = -1;
+    } else {
+      best = -INFINITY;
+      bi = 0x7FFFFFFF;
 #pragma unroll
-    for (int j = 0; j < MAXV; ++j) {
-      const int e = lane + 32 * j;
-      bool taken = false;
-      for (int q = 0; q < k; ++q) taken |= (picked[q] == e);
-      if (e < p.E && !taken && (v[j] > best || (v[j] == best && e < bi))) {
-        best = v[j];
-        bi = e;
+      for (int j = 0; j < MAXV; ++j) {
+        const int e = lane + 32 * j;
+        if (v[j] > best || (v[j] == best && e < bi)) {
+          best = v[j];
+          bi = e;
+        }
       }
-    }
 #pragma unroll
-    for (int o = 16; o > 0; o >>= 1) {
-      const float ov = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-      const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-      if (ov > best || (ov == best && oi < bi)) {
-        best = ov;
-        bi = oi;
+      for (int o = 16; o > 0; o >>= 1) {
+        const float ov = __shfl_xor_sync(0xFFFFFFFFu, best, o);
+        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
+        if (ov > best || (ov == best && oi < bi)) {
+          best = ov;
+          bi = oi;
+        }
+      }
+      if (bi >= p.E || !(best > -INFINITY)) {
+        bi = -1;  // no finite logit left (NaN input): no expert
+      } else {
+#pragma unroll
+        for (int j = 0; j < MAXV; ++j)  // remove the pick from its owner lane
+          if (lane + 32 * j == bi) v[j] = -INFINITY;
       }
     }
-    if (bi < 0 || bi >= p.E) {  // no finite logit left (NaN input): no expert
-      if (lane == 0) set_error(p.ctrl, MOE_ERR_INDEX);
-      bi = -1;
+    if (lane == k) {
+      pick_e = bi;
+      pick_l = best;
     }
-    picked[k] = bi;
   }
-  float pw[MOEQ_MAX_K];
-  float tot = 0.f;
-  for (int k = 0; k < p.K; ++k) {
-    pw[k] = picked[k] >= 0 ? expf(__ldcg(p.logits + picked[k]) - mx) / z : 0.f;
-    tot += pw[k];
-  }
-  if (lane == 0) {
-    for (int k = 0; k < p.K; ++k) {
-      const float wk = (p.renorm && tot > 0.f) ? pw[k] / tot : pw[k];
-      s_idx[k] = picked[k];
-      s_w[k] = wk;
-      if (blockIdx.x == 0) {
-        if (p.idx_out) p.idx_out[(size_t)l * p.K + k] = forced ? forced[k] : picked[k];
-        if (p.w_out) p.w_out[(size_t)l * p.K + k] = wk;
-      }
+  if (lane < p.K && pick_e < 0) set_error(p.ctrl, MOE_ERR_INDEX);
+  float pw = (lane < p.K && pick_e >= 0) ? __expf(pick_l - mx) / z : 0.f;
+  float tot = pw;
+#pragma unroll
+  for (int o = 16; o > 0; o >>= 1) tot += __shfl_xor_sync(0xFFFFFFFFu, tot, o);
+  if (lane < p.K) {
+    const float wk = (p.renorm && tot > 0.f) ? pw / tot : pw;
+    s_idx[lane] = pick_e;
+    s_w[lane] = wk;
+    if (blockIdx.x == 0) {
+      if (p.idx_out) p.idx_out[(size_t)l * p.K + lane] = forced ? forced[lane] : pick_e;
+      if (p.w_out) p.w_out[(size_t)l * p.K + lane] = wk;
     }
   }
   __syncwarp();
@@ -265,8 +296,7 @@ __device__ void producer_topk(const StackParams& p, int l, int* s_idx, float* s_
 
 // Gate and up rows of one unit from a ring slot; returns h in lane 0.
 template <int BITS>
-__device__ __forceinline__ float gateup_from_slot(const unsigned char* slot, int H, int G, const uint4* img,
-                                                  const float2* tab, float inv_sc) {
+__device__ __forceinline__ float gateup_from_slot(const unsigned char* slot, int H, int G, const ImgRef& R) {
   const int lane = threadIdx.x & 31;
   const int rowb = H * BITS / 8, ng = H / G, nchunk = H * BITS / 128;
   const bool two = (BITS == 2) && (G == 32);
@@ -277,25 +307,25 @@ __device__ __forceinline__ float gateup_from_slot(const unsigned char* slot, int
     const uint4 qg = *reinterpret_cast<const uint4*>(slot + (size_t)c * 16);
     const uint4 qu = *reinterpret_cast<const uint4*>(slot + rowb + (size_t)c * 16);
     const int g = chunk_group<BITS>(c, G, two);
-    const ChunkX<BITS> X = load_chunk_x<BITS>(c, nchunk, img, tab);
+    const ChunkX<BITS> X = load_chunk_x<BITS>(c, nchunk, R);
     part[0] += chunk_dot_x<BITS>(qg, X, gsb[g], two ? gsb[g + 1] : 0u, two);
     part[1] += chunk_dot_x<BITS>(qu, X, usb[g], two ? usb[g + 1] : 0u, two);
   }
   const float v = transpose_reduce<2>(part);
   const float up = __shfl_sync(0xFFFFFFFFu, v, 16);
-  return silu_f(v * inv_sc) * (up * inv_sc);
+  return silu_f(v) * up;
 }
 
 // Adds coef * (4 rows of one down block) into acc (per-lane partials).
 template <int BITS>
-__device__ __forceinline__ void down_block_acc(const unsigned char* blk, int I, int G, const uint4* img,
-                                               const float2* tab, float coef, float (&acc)[kDnBlk]) {
+__device__ __forceinline__ void down_block_acc(const unsigned char* blk, int I, int G, const ImgRef& R, float coef,
+                                               float (&acc)[kDnBlk]) {
   const int lane = threadIdx.x & 31;
   const int rowb = I * BITS / 8, ng = I / G, nchunk = I * BITS / 128;
   const bool two = (BITS == 2) && (G == 32);
   const uint32_t* sb = reinterpret_cast<const uint32_t*>(blk + kDnBlk * rowb);
   for (int c = lane; c < nchunk; c += 32) {
-    const ChunkX<BITS> X = load_chunk_x<BITS>(c, nchunk, img, tab);
+    const ChunkX<BITS> X = load_chunk_x<BITS>(c, nchunk, R);
     const int g = chunk_group<BITS>(c, G, two);
 #pragma unroll
     for (int r = 0; r < kDnBlk; ++r) {
@@ -305,37 +335,118 @@ __device__ __forceinline__ void down_block_acc(const unsigned char* blk, int I, 
   }
 }
 
+__device__ __forceinline__ ImgRef stack_img(unsigned char* sm, int img, int tab, int inv) {
+  return ImgRef{reinterpret_cast<uint4*>(sm + img), reinterpret_cast<float4*>(sm + tab),
+                reinterpret_cast<float*>(sm + inv)};
+}
+
+__device__ __forceinline__ ImgRef stack_himg(unsigned char* sm, const StackParams& p, int k) {
+  return ImgRef{reinterpret_cast<uint4*>(sm + p.sm_himg + (size_t)k * p.himg_stride),
+                reinterpret_cast<float4*>(sm + p.sm_htab + (size_t)k * p.htab_stride),
+                reinterpret_cast<float*>(sm + p.sm_hinv + (size_t)k * p.hinv_stride)};
+}
+
+// Stage x_l: chunk tasks of the primary width read their inputs (x_in for
+// layer 0, else bf16(r * inv_norm)), write the bf16 copy the router reads and
+// the image; returns the thread's partial dot with the shared-gate vector.
+template <int BITS>
+__device__ __forceinline__ float stage_x_primary(const StackParams& p, int l, float inv_norm, uint16_t* xs, ImgRef R,
+                                                 const uint16_t* gw, int tid) {
+  constexpr int CIN = Img<BITS>::CIN;
+  const int nchunk = p.H / CIN;
+  float gdot = 0.f;
+  for (int c = tid; c < nchunk; c += kCThreads) {
+    float v[CIN];
+    if (l == 0) {
+      load_bf16_chunk<BITS>(p.x_in + (size_t)c * CIN, v);
+    } else {
+      load_f32_chunk_cg<BITS>(p.r + (size_t)c * CIN, v);
+#pragma unroll
+      for (int j = 0; j < CIN; ++j) v[j] = bf16_bits_to_f32(f32_to_bf16_bits(v[j] * inv_norm));
+    }
+#pragma unroll
+    for (int q = 0; q < CIN / 8; ++q) {
+      uint32_t w[4];
+#pragma unroll
+      for (int i = 0; i < 4; ++i)
+        w[i] = (__float_as_uint(v[8 * q + 2 * i]) >> 16) | (__float_as_uint(v[8 * q + 2 * i + 1]) & 0xFFFF0000u);
+      reinterpret_cast<uint4*>(xs + (size_t)c * CIN)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+    }
+    if (gw) {
+#pragma unroll
+      for (int j = 0; j < CIN; ++j) gdot += bf16_bits_to_f32(gw[(size_t)c * CIN + j]) * v[j];
+    }
+    stage_chunk<BITS>(v, c, nchunk, R);
+  }
+  return gdot;
+}
+
+// A second image width staged from the bf16 copy in shared memory.
+template <int BITS>
+__device__ __forceinline__ void stage_x_secondary(int H, const uint16_t* xs, ImgRef R, int tid) {
+  constexpr int CIN = Img<BITS>::CIN;
+  const int nchunk = H / CIN;
+  for (int c = tid; c < nchunk; c += kCThreads) {
+    float v[CIN];
+    load_bf16_chunk<BITS>(xs + (size_t)c * CIN, v);
+    stage_chunk<BITS>(v, c, nchunk, R);
+  }
+}
+
+// Stage h ([K+1, I] fp32 in the workspace): task = (slot, chunk).
+__device__ __forceinline__ void stage_h_stack(const StackParams& p, unsigned char* sm, int tid) {
+  const int I = p.I, K = p.K;
+  const int n4 = I / Img<4>::CIN, n2 = I / Img<2>::CIN;
+  const int nr = (p.bits_r == 4) ? n4 : n2, ns = (p.bits_s == 4) ? n4 : n2;
+  const int total = K * nr + ns;
+  for (int t = tid; t < total; t += kCThreads) {
+    const int k = t < K * nr ? t / nr : K;
+    const int c = t < K * nr ? t % nr : t - K * nr;
+    const float* hk = p.h + (size_t)k * I;
+    const ImgRef R = stack_himg(sm, p, k);
+    if ((k < K ? p.bits_r : p.bits_s) == 4) {
+      float v[Img<4>::CIN];
+      load_f32_chunk_cg<4>(hk + (size_t)c * Img<4>::CIN, v);
+      stage_chunk<4>(v, c, n4, R);
+    } else {
+      float v[Img<2>::CIN];
+      load_f32_chunk_cg<2>(hk + (size_t)c * Img<2>::CIN, v);
+      stage_chunk<2>(v, c, n2, R);
+    }
+  }
+}
+
+
 __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t full_bar[kMaxSlots], empty_bar[kMaxSlots], c_bar[2], cfree_bar;
-  __shared__ int s_kind[kMaxSlots], s_a[kMaxSlots], s_b[kMaxSlots], s_last[kMaxSlots];
+  __shared__ int s_last[kMaxSlots];
   __shared__ int s_idx[MOEQ_MAX_K];
   __shared__ float s_w[MOEQ_MAX_K];
   __shared__ float s_part[kMaxRouterRowsPerCta][2];
-  __shared__ float s_red[kCWarps][MOEQ_MAX_K + 1];
-  __shared__ float s_hsc[MOEQ_MAX_K + 1], s_hinv[MOEQ_MAX_K + 1];
-  __shared__ float s_misc[4];  // 0: 2^-e of the x image, 1: gamma, 2: CTA sum of squares
+  __shared__ float s_misc[4];  // 1: shared-gate dot; 2: CTA sum of squares
+  __shared__ unsigned char s_piece_item[kMaxPieces];
+  __shared__ ItemPlan P;
   __shared__ volatile int s_abort;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
-  const int G = gridDim.x, c = blockIdx.x;
-  const int nr = strided_count(c, G, p.E);
-  const int nsu = strided_count(c, G, p.I);
-  const int nru = strided_count(c, G, p.K * p.I);
-  const int nblk = strided_count(c, G, p.H / kDnBlk);
-  const int per_layer = 2 * nr + nsu + nru;
+  const int G = gridDim.x;
   unsigned* sync_count = &p.ctrl->sync_count;
 
   if (tid == 0) {
+    make_plan(p, P);
+    for (int it = 0; it < P.n_items; ++it)
+      for (int q = 0; q < P.npieces[it]; ++q) s_piece_item[P.piece0[it] + q] = (unsigned char)it;
     for (int i = 0; i < p.nslot; ++i) {
       mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], 1);
+      mbar_init(&empty_bar[i], kPiecesPerItem);
       s_last[i] = -1;
     }
     mbar_init(&c_bar[0], 1);
     mbar_init(&c_bar[1], 1);
     mbar_init(&cfree_bar, kCWarps);
     s_abort = 0;
+    s_misc[1] = 0.f;
     s_misc[2] = 0.f;
     fence_mbar_init();
   }
@@ -345,21 +456,20 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     set_error(p.ctrl, MOE_ERR_TIMEOUT);
     s_abort = 1;
   };
+  const int n_items = P.n_items;
 
   if (warp == kCWarps) {
     // ===================== producer warp =====================
-    Ring R{full_bar, empty_bar, s_kind, s_a, s_b, s_last, sm + p.sm_ring, p.slot_bytes, p.nslot, 0u};
-    int c_last[2] = {-1, -1};  // last layer whose down copies were issued, per down barrier
+    Ring R{full_bar, empty_bar, s_last, sm + p.sm_ring, p.slot_bytes, p.nslot};
     unsigned char* regc = sm + p.sm_regc;
-    issue_pre(p, R, 0, nr, nsu, &s_abort);
+    int c_last[2] = {-1, -1};  // last layer whose down copies were issued, per down barrier
+    for (int it = 0; it < P.n_pre; ++it) issue_item(p, P, R, 0, it, (uint32_t)it, s_idx, &s_abort);
     for (int l = 0; l < p.n_layers; ++l) {
       if (l > 0 && !mbar_wait(&cfree_bar, (l - 1) & 1, &s_abort) && lane == 0) fail();
       __syncwarp();
       // shared expert's down blocks (known before routing)
-      if (lane == 0 && !s_abort) {
-        const uint32_t tot = issue_down_slot(p, regc, p.K, p.L[l].shared, p.off_s, p.bits_s, nblk, &c_bar[0], false);
-        mbar_arrive_expect_tx(&c_bar[0], tot);
-        issue_down_slot(p, regc, p.K, p.L[l].shared, p.off_s, p.bits_s, nblk, &c_bar[0], true);
+      if (!s_abort) {
+        issue_down(p, P, regc, l, p.K, p.K + 1, s_idx, &c_bar[0]);
         c_last[0] = l;
       }
       // routing
@@ -367,22 +477,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       __syncwarp();
       producer_topk(p, l, s_idx, s_w);
       // routed experts' down blocks, then their gate/up units
-      if (lane == 0 && !s_abort) {
-        uint32_t tot = 0;
-        for (int k = 0; k < p.K; ++k)
-          if (s_idx[k] >= 0)
-            tot += issue_down_slot(p, regc, k, p.L[l].experts + (size_t)s_idx[k] * p.rec_r, p.off_r, p.bits_r, nblk,
-                                   &c_bar[1], false);
-        mbar_arrive_expect_tx(&c_bar[1], tot);
-        for (int k = 0; k < p.K; ++k)
-          if (s_idx[k] >= 0)
-            issue_down_slot(p, regc, k, p.L[l].experts + (size_t)s_idx[k] * p.rec_r, p.off_r, p.bits_r, nblk,
-                            &c_bar[1], true);
+      if (!s_abort) {
+        issue_down(p, P, regc, l, 0, p.K, s_idx, &c_bar[1]);
         c_last[1] = l;
       }
-      __syncwarp();
-      issue_routed(p, R, l, nru, s_idx, &s_abort);
-      if (l + 1 < p.n_layers) issue_pre(p, R, l + 1, nr, nsu, &s_abort);
+      for (int it = P.n_pre; it < n_items; ++it)
+        issue_item(p, P, R, l, it, (uint32_t)(l * n_items + it), s_idx, &s_abort);
+      if (l + 1 < p.n_layers)
+        for (int it = 0; it < P.n_pre; ++it)
+          issue_item(p, P, R, l + 1, it, (uint32_t)((l + 1) * n_items + it), s_idx, &s_abort);
     }
     // drain: every copy issued must have landed before the CTA exits
     if (lane == 0) {
@@ -405,12 +508,11 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     // ===================== compute warps =====================
     const int H = p.H, I = p.I, K = p.K;
     uint16_t* xs = reinterpret_cast<uint16_t*>(sm + p.sm_xs);
-    const uint4* img4 = reinterpret_cast<const uint4*>(sm + p.sm_img4);
-    const float2* tab4 = reinterpret_cast<const float2*>(sm + p.sm_tab4);
-    const uint4* img2 = reinterpret_cast<const uint4*>(sm + p.sm_img2);
-    const float2* tab2 = reinterpret_cast<const float2*>(sm + p.sm_tab2);
+    const ImgRef X4 = stack_img(sm, p.sm_img4, p.sm_tab4, p.sm_inv4);
+    const ImgRef X2 = stack_img(sm, p.sm_img2, p.sm_tab2, p.sm_inv2);
     const unsigned char* ring = sm + p.sm_ring;
     const unsigned char* regc = sm + p.sm_regc;
+    const int n_pieces = P.n_pieces, n_rp = P.n_router_pieces;
 
     for (int l = 0; l < p.n_layers; ++l) {
       // ---- stage x_l ----
@@ -420,168 +522,110 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         named_sync(1, kCThreads);
         inv_norm = rsqrtf(__ldcg(p.ss + (l - 1)) / (float)H + p.eps);
       }
-      float amax = 0.f, gdot = 0.f;
       const uint16_t* gw = p.L[l].gate_w;
-      for (int j = tid; j < H; j += kCThreads) {
-        uint16_t xb;
-        if (l == 0)
-          xb = p.x_in[j];
-        else
-          xb = f32_to_bf16_bits(__ldcg(p.r + j) * inv_norm);
-        xs[j] = xb;
-        const float xf = bf16_bits_to_f32(xb);
-        amax = fmaxf(amax, fabsf(xf));
-        if (gw) gdot += bf16_bits_to_f32(gw[j]) * xf;
-      }
-      amax = warp_max(amax);
-      gdot = warp_sum(gdot);
-      if (lane == 0) {
-        s_red[warp][0] = amax;
-        s_red[warp][1] = gdot;
+      const float gdot = p.need4 ? stage_x_primary<4>(p, l, inv_norm, xs, X4, gw, tid)
+                                 : stage_x_primary<2>(p, l, inv_norm, xs, X2, gw, tid);
+      if (gw) {
+        const float d = warp_sum(gdot);
+        if (lane == 0) atomicAdd(&s_misc[1], d);
       }
       named_sync(1, kCThreads);
-      if (tid == 0) {
-        float m = 0.f, d = 0.f;
-        for (int w = 0; w < kCWarps; ++w) {
-          m = fmaxf(m, s_red[w][0]);
-          d += s_red[w][1];
-        }
-        const int ex = fp16_scale_exp(m);
-        s_misc[0] = pow2f(ex);
-        s_misc[1] = gw ? 1.f / (1.f + expf(-d)) : 1.f;
-        s_misc[3] = pow2f(-ex);
+      if (p.need4 && p.need2) {
+        stage_x_secondary<2>(H, xs, X2, tid);
+        named_sync(1, kCThreads);
       }
-      named_sync(1, kCThreads);
-      {
-        const float sc = s_misc[0];
-        auto get = [&](int j) { return bf16_bits_to_f32(xs[j]); };
-        if (p.need4)
-          stage_image<4>(get, H, sc, reinterpret_cast<__half*>(sm + p.sm_img4), reinterpret_cast<float2*>(sm + p.sm_tab4),
-                         tid, kCThreads);
-        if (p.need2)
-          stage_image<2>(get, H, sc, reinterpret_cast<__half*>(sm + p.sm_img2), reinterpret_cast<float2*>(sm + p.sm_tab2),
-                         tid, kCThreads);
-      }
-      named_sync(1, kCThreads);
-      const float x_inv = s_misc[3];
+      const float gamma = gw ? 1.f / (1.f + expf(-s_misc[1])) : 1.f;
 
-      // ---- ring items: router half-rows, then gate/up units ----
-      const int base = l * per_layer;
+      // ---- ring pieces: router half-rows, then gate/up units ----
       bool router_synced = false;
       auto router_barrier = [&](void) {
         if (warp == 0) {
           named_sync(2, kCThreads);
           if (lane == 0) {
-            for (int m = 0; m < nr; ++m) __stcg(p.logits + c + G * m, s_part[m][0] + s_part[m][1]);
-            __threadfence();
-            atomicAdd(sync_count, 1u);
+            for (int m = 0; m < P.nr; ++m) __stcg(p.logits + P.r0 + m, s_part[m][0] + s_part[m][1]);
+            arrive_release_gpu(sync_count);
           }
           __syncwarp();
         } else {
           named_arrive(2, kCThreads);
         }
       };
-      for (int j = base + warp; j < base + per_layer; j += kCWarps) {
-        if (!router_synced && j >= base + 2 * nr) {
+      for (int pc = warp; pc < n_pieces; pc += kCWarps) {
+        if (!router_synced && pc >= n_rp) {
           router_barrier();
           router_synced = true;
         }
-        const int slot = j % p.nslot;
-        const bool ok = mbar_wait(&full_bar[slot], (j / p.nslot) & 1, &s_abort);
+        const int it = s_piece_item[pc];
+        const int pos = pc - P.piece0[it];
+        const uint32_t seq = (uint32_t)(l * n_items + it);
+        const int slot = seq % p.nslot;
+        const bool ok = mbar_wait(&full_bar[slot], (seq / p.nslot) & 1, &s_abort);
         if (!ok && lane == 0 && !s_abort) fail();
         if (ok) {
-          const int kind = s_kind[slot], a = s_a[slot], b = s_b[slot];
           const unsigned char* sl = ring + (size_t)slot * p.slot_bytes;
-          if (kind == kItemRouterHalf) {
+          if (P.kind[it] == kItemRouter) {
+            const int row = pos >> 1, half = pos & 1;
             const int nv = H / 16;  // 16-byte words in a half row
-            const uint4* wv = reinterpret_cast<const uint4*>(sl);
-            const uint4* xv = reinterpret_cast<const uint4*>(xs + b * (H / 2));
+            const uint4* wv = reinterpret_cast<const uint4*>(sl + (size_t)row * H * 2 + (size_t)half * H);
+            const uint4* xv = reinterpret_cast<const uint4*>(xs + half * (H / 2));
             float acc = 0.f;
             for (int v = lane; v < nv; v += 32) acc = dot8_bf16(wv[v], xv[v], acc);
             acc = warp_sum(acc);
-            if (lane == 0) s_part[a][b] = acc;
+            if (lane == 0) s_part[P.first[it] + row][half] = acc;
           } else {
+            const int k = P.k[it], i = P.first[it] + pos;
+            const bool routed = k < K;
             float hv = 0.f;
-            if (kind == kItemGateUp) {
-              const int bits = a < K ? p.bits_r : p.bits_s;
-              hv = bits == 4 ? gateup_from_slot<4>(sl, H, p.G, img4, tab4, x_inv)
-                             : gateup_from_slot<2>(sl, H, p.G, img2, tab2, x_inv);
+            if (!routed || s_idx[k] >= 0) {
+              const int bits = routed ? p.bits_r : p.bits_s;
+              const RecGeom& g = routed ? p.geo_r : p.geo_s;
+              const unsigned char* unit = sl + (size_t)pos * g.U;
+              hv = bits == 4 ? gateup_from_slot<4>(unit, H, p.G, X4) : gateup_from_slot<2>(unit, H, p.G, X2);
             }
-            if (lane == 0) __stcg(p.h + (size_t)a * I + b, hv);
+            if (lane == 0) __stcg(p.h + (size_t)k * I + i, hv);
           }
         }
         __syncwarp();
-        if (lane == 0) mbar_arrive(&empty_bar[slot]);
+        if (lane == 0) {
+          const uint32_t cnt = (pos == 0) ? (uint32_t)(kPiecesPerItem - P.npieces[it] + 1) : 1u;
+          mbar_arrive_cnt(&empty_bar[slot], cnt);
+        }
       }
       if (!router_synced) router_barrier();
 
       // ---- sync 2: h complete ----
       named_sync(1, kCThreads);
       if (tid == 0) {
-        __threadfence();
-        atomicAdd(sync_count, 1u);
+        arrive_release_gpu(sync_count);
         if (!counter_wait(sync_count, (unsigned)(3 * l + 2) * G, &s_abort)) fail();
       }
       named_sync(1, kCThreads);
 
       // ---- stage h images (one per slot) ----
-      {
-        float am[MOEQ_MAX_K + 1];
-#pragma unroll
-        for (int k = 0; k <= MOEQ_MAX_K; ++k) am[k] = 0.f;
-        for (int j = tid; j < I; j += kCThreads) {
-#pragma unroll
-          for (int k = 0; k <= MOEQ_MAX_K; ++k)
-            if (k <= K) am[k] = fmaxf(am[k], fabsf(__ldcg(p.h + (size_t)k * I + j)));
-        }
-#pragma unroll
-        for (int k = 0; k <= MOEQ_MAX_K; ++k) {
-          const float m = warp_max(am[k]);
-          if (lane == 0 && k <= K) s_red[warp][k] = m;
-        }
-        named_sync(1, kCThreads);
-        if (tid <= K) {
-          float m = 0.f;
-          for (int w = 0; w < kCWarps; ++w) m = fmaxf(m, s_red[w][tid]);
-          const int ex = fp16_scale_exp(m);
-          s_hsc[tid] = pow2f(ex);
-          s_hinv[tid] = pow2f(-ex);
-        }
-        named_sync(1, kCThreads);
-        for (int k = 0; k <= K; ++k) {
-          const float* hk = p.h + (size_t)k * I;
-          auto get = [&](int j) { return __ldcg(hk + j); };
-          __half* img = reinterpret_cast<__half*>(sm + p.sm_himg + (size_t)k * p.himg_stride);
-          float2* tab = reinterpret_cast<float2*>(sm + p.sm_htab + (size_t)k * p.htab_stride);
-          if ((k < K ? p.bits_r : p.bits_s) == 4)
-            stage_image<4>(get, I, s_hsc[k], img, tab, tid, kCThreads);
-          else
-            stage_image<2>(get, I, s_hsc[k], img, tab, tid, kCThreads);
-        }
-        named_sync(1, kCThreads);
-      }
+      if (tid == 0) s_misc[1] = 0.f;  // gate dot of the next layer starts from zero
+      stage_h_stack(p, sm, tid);
+      named_sync(1, kCThreads);
 
       // ---- down + combine for this CTA's row blocks ----
       const bool ok0 = mbar_wait(&c_bar[0], l & 1, &s_abort);
       const bool ok1 = mbar_wait(&c_bar[1], l & 1, &s_abort);
       if (!(ok0 && ok1) && tid == 0 && !s_abort) fail();
-      const float gamma = s_misc[1];
       float ssq = 0.f;
-      for (int m = warp; m < nblk; m += kCWarps) {
-        const int i0 = (c + G * m) * kDnBlk;
+      for (int m = warp; m < P.nblk; m += kCWarps) {
+        const int i0 = (P.b0 + m) * kDnBlk;
         float acc[kDnBlk] = {0.f, 0.f, 0.f, 0.f};
         if (!s_abort) {
           for (int k = 0; k <= K; ++k) {
+            // s_idx/s_w were written before the routed down copies were armed
             const float wk = k < K ? (s_idx[k] >= 0 ? s_w[k] : 0.f) : gamma;
             if (wk == 0.f) continue;
-            const float coef = wk * s_hinv[k];
-            const unsigned char* blk = regc + ((size_t)k * p.nblk_max + m) * p.dblk_bytes;
-            const uint4* img = reinterpret_cast<const uint4*>(sm + p.sm_himg + (size_t)k * p.himg_stride);
-            const float2* tab = reinterpret_cast<const float2*>(sm + p.sm_htab + (size_t)k * p.htab_stride);
+            const RecGeom& g = k < K ? p.geo_r : p.geo_s;
+            const unsigned char* blk = regc + (size_t)k * p.regc_slot_bytes + (size_t)m * g.D;
+            const ImgRef R = stack_himg(sm, p, k);
             if ((k < K ? p.bits_r : p.bits_s) == 4)
-              down_block_acc<4>(blk, I, p.G, img, tab, coef, acc);
+              down_block_acc<4>(blk, I, p.G, R, wk, acc);
             else
-              down_block_acc<2>(blk, I, p.G, img, tab, coef, acc);
+              down_block_acc<2>(blk, I, p.G, R, wk, acc);
           }
         }
         const float tot = transpose_reduce<kDnBlk>(acc);
@@ -610,8 +654,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       if (tid == 0) {
         atomicAdd(p.ss + l, s_misc[2]);
         s_misc[2] = 0.f;
-        __threadfence();
-        atomicAdd(sync_count, 1u);
+        arrive_release_gpu(sync_count);
       }
     }
 
@@ -620,9 +663,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       if (tid == 0 && !counter_wait(sync_count, (unsigned)(3 * p.n_layers) * G, &s_abort)) fail();
       named_sync(1, kCThreads);
       const float inv = rsqrtf(__ldcg(p.ss + (p.n_layers - 1)) / (float)H + p.eps);
-      for (int t = tid; t < nblk * kDnBlk; t += kCThreads) {
-        const int i = (c + G * (t / kDnBlk)) * kDnBlk + (t % kDnBlk);
-        p.xnorm_out[i] = f32_to_bf16_bits(p.resid_out[i] * inv);
+      for (int t = tid; t < P.nblk * kDnBlk; t += kCThreads) {
+        const int i = P.b0 * kDnBlk + t;
+        p.xnorm_out[i] = f32_to_bf16_bits(__ldcg(p.resid_out + i) * inv);
       }
     }
   }

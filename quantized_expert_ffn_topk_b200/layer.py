@@ -4,8 +4,8 @@ from __future__ import annotations
 
 import torch
 
-from . import (moe_combine_residual, moe_expert_bytes, moe_expert_offsets, moe_expert_ffn_q, moe_layer_q,
-               moe_pack_q, moe_router_topk, moe_workspace_bytes, moe_workspace_init)
+from . import (moe_combine_residual, moe_expert_bytes, moe_expert_ffn_q, moe_expert_layout, moe_layer_q,
+               moe_pack_expert, moe_router_topk, moe_workspace_bytes, moe_workspace_init)
 
 GATE, UP, DOWN = 0, 1, 2
 
@@ -36,8 +36,8 @@ class QuantLayer:
         self.rec_s = moe_expert_bytes(H, I, bits_shared, group)
         if self.rec_r == 0 or self.rec_s == 0:
             raise ValueError("unsupported layer shape")
-        self.off_r = moe_expert_offsets(H, I, bits_routed, group)
-        self.off_s = moe_expert_offsets(H, I, bits_shared, group)
+        self.lay_r = moe_expert_layout(H, I, bits_routed, group)
+        self.lay_s = moe_expert_layout(H, I, bits_shared, group)
         self.experts = torch.empty(E * self.rec_r, dtype=torch.uint8, device=device)
         self.shared = torch.empty(self.rec_s, dtype=torch.uint8, device=device)
         self.router_w = torch.empty((E, H), dtype=torch.bfloat16, device=device)
@@ -63,27 +63,24 @@ class QuantLayer:
             return self.shared.data_ptr()
         return self.experts.data_ptr() + expert * self.rec_r
 
-    def pack_matrix(self, expert: int, matrix: int, codes, scale, bias, ws=None, stream=None) -> None:
-        """Pack one code matrix (device u8 codes, bf16 scale/bias) into its place."""
-        rows, cols = self.matrix_shape(matrix)
+    def pack_expert(self, expert: int, gate, up, down, ws=None, stream=None) -> None:
+        """Pack one expert (each matrix: device u8 codes, bf16 scale/bias) into its record."""
         bits = self.bits_shared if expert == self.E else self.bits_routed
-        off = self.off_s if expert == self.E else self.off_r
-        base = self.record_ptr(expert)
-        moe_pack_q(codes, scale, bias, rows, cols, bits, self.group, base + off[matrix], base + off[3 + matrix],
-                   ws, stream)
+        moe_pack_expert(gate, up, down, self.H, self.I, bits, self.group, self.record_ptr(expert), ws, stream)
 
     def fill(self, fill_matrix, ws=None, stream=None) -> None:
         """Build every record: fill_matrix(expert, matrix, codes_ptr, scale_ptr, bias_ptr)
         writes one matrix's u8 codes and bf16 scale/bias into scratch device
         buffers, which are then packed into the arena."""
         n = self.I * self.H
-        codes = torch.empty(n, dtype=torch.uint8, device=self.experts.device)
-        scale = torch.empty(n // self.group, dtype=torch.bfloat16, device=self.experts.device)
-        bias = torch.empty(n // self.group, dtype=torch.bfloat16, device=self.experts.device)
+        dev = self.experts.device
+        bufs = [(torch.empty(n, dtype=torch.uint8, device=dev), torch.empty(n // self.group, dtype=torch.bfloat16, device=dev),
+                 torch.empty(n // self.group, dtype=torch.bfloat16, device=dev)) for _ in range(3)]
         for e in range(self.E + 1):
             for m in (GATE, UP, DOWN):
-                fill_matrix(e, m, codes.data_ptr(), scale.data_ptr(), bias.data_ptr())
-                self.pack_matrix(e, m, codes, scale, bias, ws, stream)
+                c, s, b = bufs[m]
+                fill_matrix(e, m, c.data_ptr(), s.data_ptr(), b.data_ptr())
+            self.pack_expert(e, bufs[GATE], bufs[UP], bufs[DOWN], ws, stream)
 
     def forward(self, x, ws: Workspace, out: dict, resid_in=None, renorm=False, forced_idx=None, eps=None,
                 stream=None) -> dict:

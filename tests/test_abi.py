@@ -46,13 +46,16 @@ def test_abi_version_and_status_strings(moeq):
 
 
 def test_record_sizes_agree_with_oracle(moeq, ref):
-    for (H, I, bits, group) in ((4096, 1024, 4, 64), (4096, 1024, 2, 64), (256, 128, 4, 32), (384, 128, 2, 128)):
+    for (H, I, bits, group) in ((4096, 1024, 4, 64), (4096, 1024, 2, 64), (256, 128, 4, 32), (512, 128, 2, 128)):
         assert moeq.moe_expert_bytes(H, I, bits, group) == ref.expert_bytes(H, I, bits, group)
     assert moeq.moe_expert_bytes(4096, 1024, 4, 64) == 7077888
-    off = moeq.moe_expert_offsets(4096, 1024, 4, 64)
-    assert off == [0, 2097152, 4194304, 6291456, 6553600, 6815744]
+    lay = moeq.moe_expert_layout(4096, 1024, 4, 64)
+    # unit = gate row 2048 + up row 2048 + two table rows of 64 pairs; block = 4 down rows of 512 + 4 tables of 16 pairs
+    assert lay == [4608, 1024 * 4608, 4 * (512 + 64), 4, 2048, 512]
+    assert lay[1] + (4096 // 4) * lay[2] == 7077888
     assert moeq.moe_expert_bytes(4096, 1024, 3, 64) == 0
     assert moeq.moe_expert_bytes(4096, 1000, 4, 64) == 0
+    assert moeq.moe_expert_bytes(384, 128, 2, 128) == 0  # H/group odd: units would not be 16-byte multiples
 
 
 def test_workspace_size(moeq):
@@ -64,6 +67,15 @@ def test_workspace_size(moeq):
 
 A = 0x10000  # aligned fake device address: never dereferenced, every call below fails validation first
 M = 0x10008  # misaligned
+
+
+def test_pack_expert_rejects_bad_arguments(moeq):
+    L = moeq.lib()
+    good = [A] * 9
+    assert L.moe_pack_expert(*([None] + good[1:]), 4096, 1024, 4, 64, A, None, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_expert(*good, 4096, 1024, 4, 64, None, None, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_pack_expert(*good, 4096, 1024, 3, 64, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_pack_expert(*(good[:4] + [M] + good[5:]), 4096, 1024, 4, 64, A, None, None) == moeq.MOE_ERR_ALIGN
 
 
 def test_pack_rejects_bad_arguments(moeq):

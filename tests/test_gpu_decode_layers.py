@@ -78,9 +78,10 @@ def test_one_layer_matches_oracle(name):
     assert list(idx[0]) == list(ro["idx"])
     assert np.abs(wt[0] - ro["w"]).max() <= W_TOL
     assert hz.max_rel_err(out, ro["out"]) <= FFN_TOL
+    # RMSNorm'd bf16 output: one bf16 rounding plus the propagated FFN error
     xg = hz.bf16_to_f64(xn)
     rn = ro["out"] / np.sqrt(np.mean(ro["out"] ** 2) + EPS)
-    assert (np.abs(xg - rn) <= np.abs(rn) * 2.0 ** -7 + 1e-6).all()
+    assert (np.abs(xg - rn) <= np.abs(rn) * 2.0 ** -8 + FFN_TOL * np.abs(rn).max()).all()
 
 
 def test_chain_of_layers_router_driven():
@@ -93,7 +94,7 @@ def test_chain_of_layers_router_driven():
     ties = sum("near_tie" in ro for ro in res)
     assert ties <= 1
     for l in range(n):
-        assert np.abs(wt[l] - res[l]["w"]).max() <= W_TOL
+        assert np.abs(wt[l] - res[l]["w"]).max() <= (W_TOL if l == 0 else FFN_TOL)
     assert hz.max_rel_err(out, res[-1]["out"]) <= FFN_TOL
 
 
@@ -108,7 +109,7 @@ def test_stack_with_forced_overlap_routing():
         assert (idx == routing[t]).all()
         res = oracle_chain(w, n, synth.x_host(w, 1000 + t)[0], forced=routing[t])
         for l in range(n):
-            assert np.abs(wt[l] - res[l]["w"]).max() <= W_TOL
+            assert np.abs(wt[l] - res[l]["w"]).max() <= (W_TOL if l == 0 else FFN_TOL)
         assert hz.max_rel_err(out, res[-1]["out"]) <= FFN_TOL
 
 
@@ -124,7 +125,9 @@ def test_residual_input_and_renorm():
         experts = hz.oracle_experts(w, l)
         ro = ref_layer.layer_token(w.H, w.I, w.E, w.K, w.group, xb, synth.router_host(w, l), experts, experts(w.E),
                                    renorm=True, forced=idx[l], resid=r, eps=EPS)
-        assert np.abs(wt[l] - ro["w"]).max() <= W_TOL
+        # layer 0 sees the oracle's own input; later layers see an input that
+        # carries the previous layers' rounding, so their weights may move more
+        assert np.abs(wt[l] - ro["w"]).max() <= (W_TOL if l == 0 else FFN_TOL)
         xb, r = ro["xn"], ro["out"]
     assert hz.max_rel_err(out, r) <= FFN_TOL
 

@@ -111,18 +111,37 @@ def test_pack_flags_out_of_range_code():
     assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK  # read clears it
 
 
-def test_packed_arena_matches_oracle_pack():
-    w, L = get_layer("tiny")
-    rec = L.experts.cpu().numpy()
-    for e in (0, 5):
-        base = e * L.rec_r
-        g, u, d = synth.expert_host(w, 0, e)
-        for m, (codes, scale, bias) in enumerate((g, u, d)):
-            rp, rsb = ref.pack(codes, scale, bias, w.bits_routed, w.group)
-            got = rec[base + L.off_r[m]: base + L.off_r[m] + rp.size]
-            assert (got == rp.ravel()).all()
-            gsb = rec[base + L.off_r[3 + m]: base + L.off_r[3 + m] + rsb.size * 2].view(np.uint16)
-            assert (gsb == rsb.ravel()).all()
+def record_rows(rec, lay, H, I, bits, group):
+    """Read the gate/up/down code rows and table rows back out of one record
+    (numpy u8), following the layout moe_expert_layout describes."""
+    U, down_off, D, rpb, rowb_h, rowb_i = lay
+    sbb_h, sbb_i = H // group * 4, I // group * 4
+    units = rec[:I * U].reshape(I, U)
+    gate = units[:, :rowb_h]
+    up = units[:, rowb_h:2 * rowb_h]
+    gate_sb = units[:, 2 * rowb_h:2 * rowb_h + sbb_h].copy().view(np.uint16).reshape(I, -1, 2)
+    up_sb = units[:, 2 * rowb_h + sbb_h:].copy().view(np.uint16).reshape(I, -1, 2)
+    blocks = rec[down_off:down_off + (H // rpb) * D].reshape(H // rpb, D)
+    down = blocks[:, :rpb * rowb_i].reshape(H, rowb_i)
+    down_sb = blocks[:, rpb * rowb_i:].copy().view(np.uint16).reshape(H, -1, 2)
+    return (gate, gate_sb), (up, up_sb), (down, down_sb)
+
+
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny", dict(bits_routed=2, bits_shared=2, group=64))])
+def test_packed_arena_matches_oracle_pack(name, over):
+    w = synth.WORKLOADS[name].with_(**over)
+    L = hz.build_layer(w, 0)
+    torch.cuda.synchronize()
+    arena = L.experts.cpu().numpy()
+    shared = L.shared.cpu().numpy()
+    for e in (0, w.E - 1, w.E):
+        rec = shared if e == w.E else arena[e * L.rec_r:(e + 1) * L.rec_r]
+        lay = L.lay_s if e == w.E else L.lay_r
+        got = record_rows(rec, lay, w.H, w.I, w.bits_of(e), w.group)
+        for m, (codes, scale, bias) in enumerate(synth.expert_host(w, 0, e)):
+            rp, rsb = ref.pack(codes, scale, bias, w.bits_of(e), w.group)
+            assert (got[m][0] == rp).all(), (e, m)
+            assert (got[m][1] == rsb).all(), (e, m)
 
 
 # ---- A1+A2 router ------------------------------------------------------------
@@ -272,7 +291,7 @@ def test_batched_zipf_routing_layer():
 
 
 @pytest.mark.parametrize("over", [dict(H=320, I=96, E=5, K=1, group=32), dict(H=512, I=192, E=9, K=8, group=64),
-                                  dict(H=384, I=128, E=6, K=3, group=128, bits_routed=2),
+                                  dict(H=512, I=128, E=6, K=3, group=128, bits_routed=2),
                                   dict(H=256, I=64, E=4, K=4, group=32, bits_routed=2, bits_shared=2)])
 def test_ragged_and_edge_shapes(over):
     w = synth.WORKLOADS["tiny"].with_(**over)
