@@ -57,6 +57,7 @@ extern "C" {
 #define MOEQ_ABI_VERSION 1
 #define MOEQ_MAX_K 8      /* largest routed top-K */
 #define MOEQ_MAX_B 64     /* largest token batch per call */
+#define MOEQ_STATIC_SCRATCH_BYTES (2u << 20) /* scratch of moe_expert_ffn_q_static, per GPU */
 
 typedef enum moe_status {
   MOE_OK = 0,
@@ -231,6 +232,31 @@ moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers, const void
  * Returns MOE_OK, MOE_ERR_INDEX, MOE_ERR_RANGE, MOE_ERR_TIMEOUT, or
  * MOE_ERR_CUDA if the copy itself failed. */
 moe_status moe_get_device_error(void* ws, void* stream);
+
+/*
+ * moe_expert_ffn_q_static -- moe_expert_ffn_q without a caller workspace,
+ * for callers that cannot allocate device memory: code handed only its
+ * input and output buffers by a runtime that owns all device allocation, or
+ * code running where cudaMalloc may not be called. (The pages describe no
+ * such call; it is a convenience of this library.)
+ *   L, x_bf16, B, idx, y_out, stream  as in moe_expert_ffn_q
+ *   error_out  int32 device word, or NULL: receives the call's device error
+ *              (0, or MOE_ERR_INDEX when an index was outside [0,E) and its
+ *              slot was zeroed) in stream order
+ * Scratch is a MOEQ_STATIC_SCRATCH_BYTES array inside the library, held by
+ * every GPU that loads it until the process exits. A shape whose
+ * moe_workspace_bytes(B, K, H, I, E) exceeds that size is rejected with
+ * MOE_ERR_WORKSPACE before anything is launched. The call allocates nothing:
+ * it clears the array's control block with cudaMemsetAsync and runs the
+ * kernels of moe_expert_ffn_q on the array. All calls on a device share the
+ * array and it keeps the last call's contents, so calls that overlap on the
+ * GPU (different streams or host threads) race and must be ordered by the
+ * caller. The first call on each device looks the array's device address up
+ * (cudaGetSymbolAddress, with that device current); make that first call
+ * before any stream capture.
+ */
+moe_status moe_expert_ffn_q_static(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx,
+                                   float* y_out, int32_t* error_out, void* stream);
 
 const char* moe_status_str(moe_status s);
 int moe_abi_version(void);

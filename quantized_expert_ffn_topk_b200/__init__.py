@@ -22,6 +22,7 @@ MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 
 MOE_ERR_INDEX, MOE_ERR_TIMEOUT, MOE_ERR_WORKSPACE, MOE_ERR_RANGE = 5, 6, 7, 8
 MOEQ_MAX_K = 8
 MOEQ_MAX_B = 64
+MOEQ_STATIC_SCRATCH_BYTES = 2 << 20
 
 
 class MoeError(RuntimeError):
@@ -55,6 +56,7 @@ _SIGS = {
     "moe_combine_residual": (_INT, [_LP, _VP, _VP, _VP, _VP, _INT, _VP, _VP, _FLT, _VP]),
     "moe_decode_layers": (_INT, [_LP, _INT, _VP, _VP, _INT, _VP, _VP, _VP, _VP, _VP, _FLT, _VP, _SZ, _VP]),
     "moe_get_device_error": (_INT, [_VP, _VP]),
+    "moe_expert_ffn_q_static": (_INT, [_LP, _VP, _INT, _VP, _VP, _VP, _VP]),
 }
 
 
@@ -167,6 +169,12 @@ def moe_decode_layers(layers, x_bf16, resid_in, renorm: bool, forced_idx, idx_ou
                                    _ptr(forced_idx), _ptr(idx_out), _ptr(w_out), _ptr(resid_out),
                                    _ptr(xnorm_bf16_out), float(eps), _ptr(ws), ws_bytes, _stream(stream)),
            "moe_decode_layers")
+
+
+def moe_expert_ffn_q_static(layer: moe_layer_q, x_bf16, B: int, idx, y_out, error_out=None, stream=None) -> None:
+    """moe_expert_ffn_q on the library's own static scratch (no workspace argument)."""
+    _check(lib().moe_expert_ffn_q_static(ctypes.byref(layer), _ptr(x_bf16), B, _ptr(idx), _ptr(y_out),
+                                         _ptr(error_out), _stream(stream)), "moe_expert_ffn_q_static")
 
 
 def moe_get_device_error(ws, stream=None) -> int:
