@@ -54,42 +54,67 @@ struct ImgRef {
   float* inv;
 };
 
-// Stage chunk c from its CIN input values v (fp32, final values).
+// Staging is done 16 inputs per thread: a chunk is split into TPC = CIN/16
+// segments held by TPC adjacent lanes (4-bit: 2 lanes of two words each;
+// 2-bit: 4 lanes of one word each). The lanes agree on the chunk's scale and
+// table entry through shuffles. Every lane of the warp must call the staging
+// functions together; lanes without a segment pass active = false.
 template <int BITS>
-__device__ __forceinline__ void stage_chunk(const float* v, int c, int nchunk, ImgRef R) {
+struct Seg {
+  static constexpr int TPC = Img<BITS>::CIN / 16;  // lanes per chunk
+  static constexpr int WORDS = 16 / Img<BITS>::EPW;  // words per segment (2 or 1)
+};
+
+// Stage segment s of chunk c from its 16 input values v (fp32, final values).
+template <int BITS>
+__device__ __forceinline__ void stage_seg(const float (&v)[16], int c, int s, int nchunk, ImgRef R, bool active) {
   using I = Img<BITS>;
+  using SG = Seg<BITS>;
   float amax = 0.f;
 #pragma unroll
-  for (int j = 0; j < I::CIN; ++j) amax = fmaxf(amax, fabsf(v[j]));
+  for (int j = 0; j < 16; ++j) amax = fmaxf(amax, fabsf(v[j]));
+#pragma unroll
+  for (int o = 1; o < SG::TPC; o <<= 1) amax = fmaxf(amax, __shfl_xor_sync(0xFFFFFFFFu, amax, o));
   const int e = fp16_scale_exp(amax);
   const float sc = pow2f(e);
-  float C[2] = {0.f, 0.f}, S[2] = {0.f, 0.f};
+  float C = 0.f, S = 0.f;
 #pragma unroll
-  for (int t = 0; t < 4; ++t) {
+  for (int tw = 0; tw < SG::WORDS; ++tw) {
+    const int t = s * SG::WORDS + tw;  // word within the chunk
     uint32_t packed[I::PAIRS];
 #pragma unroll
     for (int m = 0; m < I::PAIRS; ++m) {
-      const float lo = v[t * I::EPW + m], hi = v[t * I::EPW + m + I::PAIRS];
-      const float s = sc * (1.0f / (float)(1 << I::shift_of(m)));
-      const __half hl = __float2half_rn(lo * s), hh = __float2half_rn(hi * s);
+      const float lo = v[tw * I::EPW + m], hi = v[tw * I::EPW + m + I::PAIRS];
+      const float f = sc * (1.0f / (float)(1 << I::shift_of(m)));
+      const __half hl = __float2half_rn(lo * f), hh = __float2half_rn(hi * f);
       packed[m] = (uint32_t)__half_as_ushort(hl) | ((uint32_t)__half_as_ushort(hh) << 16);
-      C[t >> 1] += 1024.f * (__half2float(hl) + __half2float(hh));
-      S[t >> 1] += lo + hi;
+      C += 1024.f * (__half2float(hl) + __half2float(hh));
+      S += lo + hi;
     }
+    if (active) {
 #pragma unroll
-    for (int q = 0; q < I::PAIRS / 4; ++q)
-      R.img[(t * (I::PAIRS / 4) + q) * nchunk + c] =
-          make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+      for (int q = 0; q < I::PAIRS / 4; ++q)
+        R.img[(t * (I::PAIRS / 4) + q) * nchunk + c] =
+            make_uint4(packed[4 * q], packed[4 * q + 1], packed[4 * q + 2], packed[4 * q + 3]);
+    }
   }
-  R.tab[c] = make_float4(C[0], C[1], S[0], S[1]);
-  R.inv[c] = pow2f(-e);
+  // half-chunk sums: 4-bit segments are half chunks; 2-bit half chunks are two segments
+  if (BITS == 2) {
+    C += __shfl_xor_sync(0xFFFFFFFFu, C, 1);
+    S += __shfl_xor_sync(0xFFFFFFFFu, S, 1);
+  }
+  const int other = BITS == 4 ? 1 : 2;  // lane offset of the chunk's second half
+  const float C1 = __shfl_xor_sync(0xFFFFFFFFu, C, other), S1 = __shfl_xor_sync(0xFFFFFFFFu, S, other);
+  if (active && s == 0) {
+    R.tab[c] = make_float4(C, C1, S, S1);
+    R.inv[c] = pow2f(-e);
+  }
 }
 
-// CIN bf16 inputs (global or shared memory, 16-byte aligned) -> fp32 values.
-template <int BITS>
-__device__ __forceinline__ void load_bf16_chunk(const uint16_t* src, float* v) {
+// 16 bf16 inputs (global or shared memory, 16-byte aligned) -> fp32 values.
+__device__ __forceinline__ void load_bf16_16(const uint16_t* src, float (&v)[16]) {
 #pragma unroll
-  for (int q = 0; q < Img<BITS>::CIN / 8; ++q) {
+  for (int q = 0; q < 2; ++q) {
     const uint4 w = reinterpret_cast<const uint4*>(src)[q];
     const uint32_t ww[4] = {w.x, w.y, w.z, w.w};
 #pragma unroll
@@ -100,18 +125,39 @@ __device__ __forceinline__ void load_bf16_chunk(const uint16_t* src, float* v) {
   }
 }
 
-// CIN fp32 inputs written by other CTAs of this grid or an earlier kernel
-// (read at L2, 16-byte aligned).
-template <int BITS>
-__device__ __forceinline__ void load_f32_chunk_cg(const float* src, float* v) {
+// 16 fp32 inputs written by other CTAs or an earlier kernel (read at L2).
+__device__ __forceinline__ void load_f32_16_cg(const float* src, float (&v)[16]) {
 #pragma unroll
-  for (int q = 0; q < Img<BITS>::CIN / 4; ++q) {
+  for (int q = 0; q < 4; ++q) {
     const float4 f = __ldcg(reinterpret_cast<const float4*>(src) + q);
     v[4 * q] = f.x;
     v[4 * q + 1] = f.y;
     v[4 * q + 2] = f.z;
     v[4 * q + 3] = f.w;
   }
+}
+
+// One warp stages segments [32*gi, 32*gi + 32) of a vector of n inputs
+// (n a multiple of CIN); get(j0, v) fills the 16 values starting at input j0.
+template <int BITS, typename Get>
+__device__ __forceinline__ void stage_group(Get get, int n, ImgRef R, int gi, int lane) {
+  constexpr int TPC = Seg<BITS>::TPC;
+  const int t = gi * 32 + lane;
+  const bool active = t < n / 16;
+  float v[16];
+  if (active) {
+    get(t * 16, v);
+  } else {
+#pragma unroll
+    for (int j = 0; j < 16; ++j) v[j] = 0.f;
+  }
+  stage_seg<BITS>(v, t / TPC, t % TPC, n / Img<BITS>::CIN, R, active);
+}
+
+// Stage a whole vector with nthr threads (a multiple of 32).
+template <int BITS, typename Get>
+__device__ __forceinline__ void stage_vector(Get get, int n, ImgRef R, int tid, int nthr) {
+  for (int gi = tid >> 5; gi * 32 < n / 16; gi += nthr >> 5) stage_group<BITS>(get, n, R, gi, tid & 31);
 }
 
 // One 32-bit word of codes against its staged pairs (packed fp16 words).

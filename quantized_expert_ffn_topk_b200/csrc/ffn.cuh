@@ -90,15 +90,10 @@ __host__ __device__ inline GuSmem gu_smem_plan(int H, bool need4, bool need2) {
   return s;
 }
 
-// Every thread stages whole chunks of x straight from global memory.
+// The CTA stages x straight from global memory, 16 inputs per thread.
 template <int BITS>
 __device__ __forceinline__ void stage_x_chunks(const uint16_t* xb, int H, ImgRef R) {
-  const int nchunk = H / Img<BITS>::CIN;
-  for (int c = threadIdx.x; c < nchunk; c += blockDim.x) {
-    float v[Img<BITS>::CIN];
-    load_bf16_chunk<BITS>(xb + (size_t)c * Img<BITS>::CIN, v);
-    stage_chunk<BITS>(v, c, nchunk, R);
-  }
+  stage_vector<BITS>([&](int j0, float (&v)[16]) { load_bf16_16(xb + j0, v); }, H, R, threadIdx.x, blockDim.x);
 }
 
 // Persistent over units: grid (ctas, B), CTA c takes units
@@ -169,31 +164,21 @@ __device__ __forceinline__ ImgRef dn_img(unsigned char* smem, const DnSmem& sp, 
                 reinterpret_cast<float*>(smem + sp.inv + (size_t)k * sp.inv_stride)};
 }
 
-// Stage h (fp32, [K+1, I]) of one token: task t = (slot, chunk).
+// Stage h (fp32, [K+1, I]) of one token: warp job j = (slot, 32 segments of
+// 16 inputs), so that every warp stages one width at a time.
 __device__ __forceinline__ void stage_h(const float* hb, int I, int K, int bits_r, int bits_s, unsigned char* smem,
                                         const DnSmem& sp, int tid, int nthr) {
-  const int n4 = I / Img<4>::CIN, n2 = I / Img<2>::CIN;
-  int total = 0;
-  for (int k = 0; k <= K; ++k) total += ((k < K ? bits_r : bits_s) == 4) ? n4 : n2;
-  for (int t = tid; t < total; t += nthr) {
-    int k = 0, c = t;
-    while (true) {
-      const int nk = ((k < K ? bits_r : bits_s) == 4) ? n4 : n2;
-      if (c < nk) break;
-      c -= nk;
-      ++k;
-    }
+  const int jobs_per_slot = (I / 16 + 31) / 32;
+  const int lane = tid & 31;
+  for (int j = tid >> 5; j < (K + 1) * jobs_per_slot; j += nthr >> 5) {
+    const int k = j / jobs_per_slot, gi = j % jobs_per_slot;
     const float* hk = hb + (size_t)k * I;
     const ImgRef R = dn_img(smem, sp, k);
-    if ((k < K ? bits_r : bits_s) == 4) {
-      float v[Img<4>::CIN];
-      load_f32_chunk_cg<4>(hk + (size_t)c * Img<4>::CIN, v);
-      stage_chunk<4>(v, c, n4, R);
-    } else {
-      float v[Img<2>::CIN];
-      load_f32_chunk_cg<2>(hk + (size_t)c * Img<2>::CIN, v);
-      stage_chunk<2>(v, c, n2, R);
-    }
+    auto get = [&](int j0, float (&v)[16]) { load_f32_16_cg(hk + j0, v); };
+    if ((k < K ? bits_r : bits_s) == 4)
+      stage_group<4>(get, I, R, gi, lane);
+    else
+      stage_group<2>(get, I, R, gi, lane);
   }
 }
 

@@ -161,52 +161,79 @@ struct Ring {
   int slot_bytes, nslot;
 };
 
-// Issue ring item `it` of layer l as ring sequence number `seq`.
-__device__ void issue_item(const StackParams& p, const ItemPlan& P, Ring& R, int l, int it, uint32_t seq,
-                           const int* s_idx, const volatile int* abort) {
-  const int lane = threadIdx.x & 31;
-  const uint32_t slot = seq % R.nslot, fill = seq / R.nslot;
-  bool ok = true;
-  if (fill > 0) ok = mbar_wait(&R.empty[slot], (fill - 1) & 1, abort);
-  if (lane == 0 && ok) {
-    const void* src = nullptr;
-    uint32_t bytes = 0;
-    if (P.kind[it] == kItemRouter) {
-      src = p.L[l].router_w + (size_t)(P.r0 + P.first[it]) * p.H;
-      bytes = (uint32_t)(P.npieces[it] / 2) * (uint32_t)p.H * 2;
-    } else if (P.k[it] == p.K) {
-      src = p.L[l].shared + (size_t)P.first[it] * p.geo_s.U;
-      bytes = (uint32_t)P.npieces[it] * p.geo_s.U;
-    } else {
-      const int e = s_idx[P.k[it]];
-      if (e >= 0) {
-        src = p.L[l].experts + (size_t)e * p.rec_r + (size_t)P.first[it] * p.geo_r.U;
-        bytes = (uint32_t)P.npieces[it] * p.geo_r.U;
-      }
-    }
-    R.last[slot] = (int)seq;
-    mbar_arrive_expect_tx(&R.full[slot], bytes);
-    if (bytes) bulk_g2s(R.base + (size_t)slot * R.slot_bytes, src, bytes, &R.full[slot]);
+// Source and size of ring item `it` of layer l (0 bytes: an empty item,
+// for a slot whose expert index was invalid).
+__device__ __forceinline__ uint32_t item_source(const StackParams& p, const ItemPlan& P, int l, int it,
+                                                const int* s_idx, const void** src) {
+  if (P.kind[it] == kItemRouter) {
+    *src = p.L[l].router_w + (size_t)(P.r0 + P.first[it]) * p.H;
+    return (uint32_t)(P.npieces[it] / 2) * (uint32_t)p.H * 2;
   }
-  __syncwarp();
+  if (P.k[it] == p.K) {
+    *src = p.L[l].shared + (size_t)P.first[it] * p.geo_s.U;
+    return (uint32_t)P.npieces[it] * p.geo_s.U;
+  }
+  const int e = s_idx[P.k[it]];
+  if (e < 0) return 0u;
+  *src = p.L[l].experts + (size_t)e * p.rec_r + (size_t)P.first[it] * p.geo_r.U;
+  return (uint32_t)P.npieces[it] * p.geo_r.U;
 }
 
-// The CTA's down blocks of slots [k0, k1): one copy per slot, arming `bar`.
+// Issue ring items [it0, it1) of layer l, item it taking ring sequence number
+// seq0 + (it - it0). The lanes issue in parallel: each round takes the run
+// of next items whose slots are already free (lane j -> item next + j); if
+// none is, lane 0 waits for the first. Returns false if a wait gave up.
+__device__ bool issue_items(const StackParams& p, const ItemPlan& P, Ring& R, int l, int it0, int it1, uint32_t seq0,
+                            const int* s_idx, const volatile int* abort) {
+  const int lane = threadIdx.x & 31;
+  const int width = min(32, R.nslot);
+  for (int next = it0; next < it1;) {
+    const int n = min(width, it1 - next);
+    const uint32_t seq = seq0 + (uint32_t)(next - it0 + lane);
+    const uint32_t slot = seq % R.nslot, fill = seq / R.nslot;
+    const bool ready = lane < n && (fill == 0 || mbar_try_wait(&R.empty[slot], (fill - 1) & 1));
+    int nr = __ffs(~__ballot_sync(0xFFFFFFFFu, ready)) - 1;  // ready run starting at lane 0
+    if (nr < 0) nr = 32;
+    nr = min(nr, n);
+    if (nr == 0) {
+      bool ok = true;
+      if (lane == 0) ok = mbar_wait(&R.empty[slot], (fill - 1) & 1, abort);
+      if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) return false;
+      nr = 1;
+    }
+    if (lane < nr) {
+      const void* src = nullptr;
+      const uint32_t bytes = item_source(p, P, l, next + lane, s_idx, &src);
+      R.last[slot] = (int)seq;
+      mbar_arrive_expect_tx(&R.full[slot], bytes);
+      if (bytes) bulk_g2s(R.base + (size_t)slot * R.slot_bytes, src, bytes, &R.full[slot]);
+    }
+    __syncwarp();
+    next += nr;
+  }
+  return true;
+}
+
+// The CTA's down blocks of slots [k0, k1): one copy per slot (lane k - k0
+// issues slot k's), all arming `bar`.
 __device__ void issue_down(const StackParams& p, const ItemPlan& P, unsigned char* regc, int l, int k0, int k1,
                            const int* s_idx, uint64_t* bar) {
-  if ((threadIdx.x & 31) == 0) {
+  const int lane = threadIdx.x & 31;
+  if (lane == 0) {
     uint32_t tot = 0;
     for (int k = k0; k < k1; ++k)
       if (k == p.K || s_idx[k] >= 0) tot += (uint32_t)P.nblk * (k == p.K ? p.geo_s.D : p.geo_r.D);
     mbar_arrive_expect_tx(bar, tot);
-    for (int k = k0; k < k1; ++k) {
-      const bool shared = (k == p.K);
-      if (!shared && s_idx[k] < 0) continue;
+  }
+  __syncwarp();
+  const int k = k0 + lane;
+  if (k < k1 && P.nblk > 0) {
+    const bool shared = (k == p.K);
+    if (shared || s_idx[k] >= 0) {
       const RecGeom& g = shared ? p.geo_s : p.geo_r;
       const uint8_t* rec = shared ? p.L[l].shared : p.L[l].experts + (size_t)s_idx[k] * p.rec_r;
-      if (P.nblk > 0)
-        bulk_g2s(regc + (size_t)k * p.regc_slot_bytes, rec + g.down_off + (size_t)P.b0 * g.D, (uint32_t)P.nblk * g.D,
-                 bar);
+      bulk_g2s(regc + (size_t)k * p.regc_slot_bytes, rec + g.down_off + (size_t)P.b0 * g.D, (uint32_t)P.nblk * g.D,
+               bar);
     }
   }
   __syncwarp();
@@ -346,73 +373,60 @@ __device__ __forceinline__ ImgRef stack_himg(unsigned char* sm, const StackParam
                 reinterpret_cast<float*>(sm + p.sm_hinv + (size_t)k * p.hinv_stride)};
 }
 
-// Stage x_l: chunk tasks of the primary width read their inputs (x_in for
-// layer 0, else bf16(r * inv_norm)), write the bf16 copy the router reads and
-// the image; returns the thread's partial dot with the shared-gate vector.
+// Stage x_l, 16 inputs per thread: read the inputs (x_in for layer 0, else
+// bf16(r * inv_norm)), write the bf16 copy the router reads and the image of
+// the primary width; returns the thread's partial dot with the shared-gate
+// vector.
 template <int BITS>
 __device__ __forceinline__ float stage_x_primary(const StackParams& p, int l, float inv_norm, uint16_t* xs, ImgRef R,
                                                  const uint16_t* gw, int tid) {
-  constexpr int CIN = Img<BITS>::CIN;
-  const int nchunk = p.H / CIN;
   float gdot = 0.f;
-  for (int c = tid; c < nchunk; c += kCThreads) {
-    float v[CIN];
+  auto get = [&](int j0, float (&v)[16]) {
     if (l == 0) {
-      load_bf16_chunk<BITS>(p.x_in + (size_t)c * CIN, v);
+      load_bf16_16(p.x_in + j0, v);
     } else {
-      load_f32_chunk_cg<BITS>(p.r + (size_t)c * CIN, v);
+      load_f32_16_cg(p.r + j0, v);
 #pragma unroll
-      for (int j = 0; j < CIN; ++j) v[j] = bf16_bits_to_f32(f32_to_bf16_bits(v[j] * inv_norm));
+      for (int j = 0; j < 16; ++j) v[j] = bf16_bits_to_f32(f32_to_bf16_bits(v[j] * inv_norm));
     }
 #pragma unroll
-    for (int q = 0; q < CIN / 8; ++q) {
+    for (int q = 0; q < 2; ++q) {
       uint32_t w[4];
 #pragma unroll
       for (int i = 0; i < 4; ++i)
         w[i] = (__float_as_uint(v[8 * q + 2 * i]) >> 16) | (__float_as_uint(v[8 * q + 2 * i + 1]) & 0xFFFF0000u);
-      reinterpret_cast<uint4*>(xs + (size_t)c * CIN)[q] = make_uint4(w[0], w[1], w[2], w[3]);
+      reinterpret_cast<uint4*>(xs + j0)[q] = make_uint4(w[0], w[1], w[2], w[3]);
     }
     if (gw) {
+      float g[16];
+      load_bf16_16(gw + j0, g);
 #pragma unroll
-      for (int j = 0; j < CIN; ++j) gdot += bf16_bits_to_f32(gw[(size_t)c * CIN + j]) * v[j];
+      for (int j = 0; j < 16; ++j) gdot += g[j] * v[j];
     }
-    stage_chunk<BITS>(v, c, nchunk, R);
-  }
+  };
+  for (int gi = tid >> 5; gi * 32 < p.H / 16; gi += kCWarps) stage_group<BITS>(get, p.H, R, gi, tid & 31);
   return gdot;
 }
 
 // A second image width staged from the bf16 copy in shared memory.
 template <int BITS>
 __device__ __forceinline__ void stage_x_secondary(int H, const uint16_t* xs, ImgRef R, int tid) {
-  constexpr int CIN = Img<BITS>::CIN;
-  const int nchunk = H / CIN;
-  for (int c = tid; c < nchunk; c += kCThreads) {
-    float v[CIN];
-    load_bf16_chunk<BITS>(xs + (size_t)c * CIN, v);
-    stage_chunk<BITS>(v, c, nchunk, R);
-  }
+  stage_vector<BITS>([&](int j0, float (&v)[16]) { load_bf16_16(xs + j0, v); }, H, R, tid, kCThreads);
 }
 
-// Stage h ([K+1, I] fp32 in the workspace): task = (slot, chunk).
+// Stage h ([K+1, I] fp32 in the workspace): warp job = (slot, 32 segments).
 __device__ __forceinline__ void stage_h_stack(const StackParams& p, unsigned char* sm, int tid) {
   const int I = p.I, K = p.K;
-  const int n4 = I / Img<4>::CIN, n2 = I / Img<2>::CIN;
-  const int nr = (p.bits_r == 4) ? n4 : n2, ns = (p.bits_s == 4) ? n4 : n2;
-  const int total = K * nr + ns;
-  for (int t = tid; t < total; t += kCThreads) {
-    const int k = t < K * nr ? t / nr : K;
-    const int c = t < K * nr ? t % nr : t - K * nr;
+  const int jobs_per_slot = (I / 16 + 31) / 32;
+  for (int j = tid >> 5; j < (K + 1) * jobs_per_slot; j += kCWarps) {
+    const int k = j / jobs_per_slot, gi = j % jobs_per_slot;
     const float* hk = p.h + (size_t)k * I;
     const ImgRef R = stack_himg(sm, p, k);
-    if ((k < K ? p.bits_r : p.bits_s) == 4) {
-      float v[Img<4>::CIN];
-      load_f32_chunk_cg<4>(hk + (size_t)c * Img<4>::CIN, v);
-      stage_chunk<4>(v, c, n4, R);
-    } else {
-      float v[Img<2>::CIN];
-      load_f32_chunk_cg<2>(hk + (size_t)c * Img<2>::CIN, v);
-      stage_chunk<2>(v, c, n2, R);
-    }
+    auto get = [&](int j0, float (&v)[16]) { load_f32_16_cg(hk + j0, v); };
+    if ((k < K ? p.bits_r : p.bits_s) == 4)
+      stage_group<4>(get, I, R, gi, tid & 31);
+    else
+      stage_group<2>(get, I, R, gi, tid & 31);
   }
 }
 
@@ -463,7 +477,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     Ring R{full_bar, empty_bar, s_last, sm + p.sm_ring, p.slot_bytes, p.nslot};
     unsigned char* regc = sm + p.sm_regc;
     int c_last[2] = {-1, -1};  // last layer whose down copies were issued, per down barrier
-    for (int it = 0; it < P.n_pre; ++it) issue_item(p, P, R, 0, it, (uint32_t)it, s_idx, &s_abort);
+    if (!issue_items(p, P, R, 0, 0, P.n_pre, 0u, s_idx, &s_abort) && lane == 0) fail();
     for (int l = 0; l < p.n_layers; ++l) {
       if (l > 0 && !mbar_wait(&cfree_bar, (l - 1) & 1, &s_abort) && lane == 0) fail();
       __syncwarp();
@@ -476,16 +490,20 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       if (!counter_wait(sync_count, (unsigned)(3 * l + 1) * G, &s_abort) && lane == 0) fail();
       __syncwarp();
       producer_topk(p, l, s_idx, s_w);
-      // routed experts' down blocks, then their gate/up units
+      // routed gate/up units (first as many as the ring takes now), the
+      // routed down blocks, then the remaining units
+      const uint32_t seq_l = (uint32_t)(l * n_items);
+      const int first = min(n_items, P.n_pre + p.nslot);
+      bool ok = issue_items(p, P, R, l, P.n_pre, first, seq_l + P.n_pre, s_idx, &s_abort);
       if (!s_abort) {
         issue_down(p, P, regc, l, 0, p.K, s_idx, &c_bar[1]);
         c_last[1] = l;
       }
-      for (int it = P.n_pre; it < n_items; ++it)
-        issue_item(p, P, R, l, it, (uint32_t)(l * n_items + it), s_idx, &s_abort);
-      if (l + 1 < p.n_layers)
-        for (int it = 0; it < P.n_pre; ++it)
-          issue_item(p, P, R, l + 1, it, (uint32_t)((l + 1) * n_items + it), s_idx, &s_abort);
+      if (ok) ok = issue_items(p, P, R, l, first, n_items, seq_l + first, s_idx, &s_abort);
+      if (ok && l + 1 < p.n_layers)
+        ok = issue_items(p, P, R, l + 1, 0, P.n_pre, (uint32_t)((l + 1) * n_items), s_idx, &s_abort);
+      if (!ok && lane == 0 && !s_abort) fail();
+      __syncwarp();
     }
     // drain: every copy issued must have landed before the CTA exits
     if (lane == 0) {
