@@ -13,9 +13,9 @@ namespace moeq {
 struct WsCtrl {
   int error;                // first device-side moe_status (0 = none)
   unsigned router_ticket;   // last-CTA ticket of the router kernel (back to 0 after each call)
-  unsigned sync_count;      // grid-wide arrival counter of the fused decode kernel (0 between calls)
   unsigned exit_count;      // CTAs that left the fused decode kernel (0 between calls)
-  unsigned pad[60];
+  unsigned sync[4];         // arrival counters of the fused decode kernel (0 between calls)
+  unsigned pad[57];
 };
 static_assert(sizeof(WsCtrl) == 256, "control block is 256 bytes");
 
@@ -35,24 +35,32 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
   return (uint16_t)(u >> 16);
 }
 
-// Geometry of one expert record (bytes). Gate/up unit i at i*U:
-// [gate code row][up code row][gate table row][up table row]; down block b at
-// down_off + b*D: [4 down code rows][their 4 table rows].
-constexpr int kRowsPerDownBlock = 4;
+// Geometry of one expert record (bytes). Every matrix is stored as tiles of
+// 16 rows laid out for the int8 tensor-core dot (mma m16n8k32 fragments):
+// tile T holds, for each group of G inputs, one block of
+//   codes  32 lanes x (G/32 k-steps) x W bytes (W = 8 at 4 bits, 4 at 2 bits)
+//   table  8 x [(scale, bias) of local row g, (scale, bias) of local row g+8]
+// Gate/up tile T (at T*U, I/8 tiles of H inputs) holds gate rows 8T..8T+7 as
+// local rows 0..7 and up rows 8T..8T+7 as local rows 8..15; down tile T (at
+// down_off + T*D, H/16 tiles of I inputs) holds rows 16T..16T+15.
+constexpr int kTileRows = 16;
 struct RecGeom {
-  uint32_t U, rowb_h, sbb_h;  // gate/up unit, code row of H inputs, table row
-  uint32_t D, rowb_i, sbb_i;  // down block, code row of I inputs, table row
+  uint32_t blk;               // block bytes (one group of one tile)
+  uint32_t ng_h, U;           // gate/up: groups per tile, tile bytes
+  uint32_t ng_i, D;           // down: groups per tile, tile bytes
   unsigned long long down_off;
 };
+__host__ __device__ inline uint32_t tile_block_bytes(int bits, int group) {
+  return (uint32_t)(group * (bits == 4 ? 8 : 4) + 64);
+}
 __host__ __device__ inline RecGeom rec_geom(int H, int I, int bits, int group) {
   RecGeom g;
-  g.rowb_h = (uint32_t)(H * bits / 8);
-  g.sbb_h = (uint32_t)(H / group * 4);
-  g.U = 2 * (g.rowb_h + g.sbb_h);
-  g.rowb_i = (uint32_t)(I * bits / 8);
-  g.sbb_i = (uint32_t)(I / group * 4);
-  g.D = kRowsPerDownBlock * (g.rowb_i + g.sbb_i);
-  g.down_off = (unsigned long long)I * g.U;
+  g.blk = tile_block_bytes(bits, group);
+  g.ng_h = (uint32_t)(H / group);
+  g.U = g.ng_h * g.blk;
+  g.ng_i = (uint32_t)(I / group);
+  g.D = g.ng_i * g.blk;
+  g.down_off = (unsigned long long)(I / 8) * g.U;
   return g;
 }
 
@@ -80,19 +88,6 @@ __device__ __forceinline__ uint2 ld_stream8(const void* p) {
   uint2 v;
   asm("ld.global.nc.L1::no_allocate.v2.u32 {%0,%1}, [%2];" : "=r"(v.x), "=r"(v.y) : "l"(p));
   return v;
-}
-
-// c + a.lo*b.lo + a.hi*b.hi with a, b packed fp16 pairs and c fp32: the
-// products of two fp16 values are exact in fp32; accumulation is fp32.
-__device__ __forceinline__ float fma2_f16_f32(uint32_t a, uint32_t b, float c) {
-  float d;
-  asm("{ .reg .f16 al, ah, bl, bh;\n\t .reg .f32 t;\n\t"
-      "mov.b32 {al, ah}, %1;\n\t mov.b32 {bl, bh}, %2;\n\t"
-      "fma.rn.f32.f16 t, al, bl, %3;\n\t"
-      "fma.rn.f32.f16 %0, ah, bh, t; }"
-      : "=f"(d)
-      : "r"(a), "r"(b), "f"(c));
-  return d;
 }
 
 template <typename T>

@@ -134,7 +134,7 @@ const char* moe_status_str(moe_status s) {
 size_t moe_expert_bytes(int H, int I, int bits, int group) {
   if (H <= 0 || I <= 0 || !bits_ok(bits) || !group_ok(group)) return 0;
   if (!cols_ok(H, bits, group) || !cols_ok(I, bits, group)) return 0;
-  if ((H / group) % 2 != 0) return 0;  // a gate/up unit must stay a multiple of 16 bytes
+  if (H % kTileRows != 0 || I % 8 != 0) return 0;  // whole tiles of 16 rows
   const size_t hi = 3 * (size_t)H * I;
   return hi * bits / 8 + hi / group * 4;
 }
@@ -146,9 +146,9 @@ moe_status moe_expert_layout(int H, int I, int bits, int group, size_t lay[6]) {
   lay[0] = g.U;
   lay[1] = (size_t)g.down_off;
   lay[2] = g.D;
-  lay[3] = kRowsPerDownBlock;
-  lay[4] = g.rowb_h;
-  lay[5] = g.rowb_i;
+  lay[3] = kTileRows;
+  lay[4] = g.blk;
+  lay[5] = (size_t)(I / 8);
   return MOE_OK;
 }
 
@@ -213,28 +213,26 @@ moe_status moe_pack_expert(const uint8_t* codes_gate, const void* scale_gate_bf1
   const RecGeom g = rec_geom(H, I, bits, group);
   unsigned char* rec = reinterpret_cast<unsigned char*>(record_out);
   const unsigned maxg = (unsigned)num_sms() * 8;
-  auto launch = [&](const uint8_t* codes, const void* sc, const void* bi, int rows, int cols, RowPlace pc, RowPlace ps) {
-    const int64_t nchunks = (int64_t)rows * cols * bits / 128;
-    const int64_t nsb = (int64_t)rows * (cols / group);
-    const unsigned g1 = (unsigned)std::min<int64_t>((nchunks + 255) / 256, maxg);
+  auto u16 = [](const void* q) { return reinterpret_cast<const uint16_t*>(q); };
+  auto launch = [&](const TileSrc& src, int ntiles, int C, unsigned char* dst, uint32_t tile_bytes) {
+    const int64_t ncode = (int64_t)ntiles * C;  // threads: (tile, group, lane, k-step)
+    const int64_t nsb = (int64_t)ntiles * (C / group) * 8;
+    const unsigned g1 = (unsigned)std::min<int64_t>((ncode + 255) / 256, maxg);
     const unsigned g2 = (unsigned)std::min<int64_t>((nsb + 255) / 256, maxg);
-    const int cpr = cols * bits / 128;
     if (bits == 4)
-      k_pack_codes<4><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
+      k_pack_tile_codes<4><<<g1, 256, 0, s>>>(src, ntiles, C, group, dst, tile_bytes, g.blk, ctrl);
     else
-      k_pack_codes<2><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
-    k_pack_sb<<<g2, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(sc), reinterpret_cast<const uint16_t*>(bi), nsb,
-                                 cols / group, ps);
+      k_pack_tile_codes<2><<<g1, 256, 0, s>>>(src, ntiles, C, group, dst, tile_bytes, g.blk, ctrl);
+    k_pack_tile_sb<<<g2, 256, 0, s>>>(src, ntiles, C, group, dst, tile_bytes, g.blk, g.blk - 64);
   };
-  // gate and up: one row per unit
-  launch(codes_gate, scale_gate_bf16, bias_gate_bf16, I, H, RowPlace{rec, I, g.U, (size_t)g.U * I},
-         RowPlace{rec + 2 * g.rowb_h, I, g.U, (size_t)g.U * I});
-  launch(codes_up, scale_up_bf16, bias_up_bf16, I, H, RowPlace{rec + g.rowb_h, I, g.U, (size_t)g.U * I},
-         RowPlace{rec + 2 * g.rowb_h + g.sbb_h, I, g.U, (size_t)g.U * I});
-  // down: blocks of four rows
-  unsigned char* dn = rec + g.down_off;
-  launch(codes_down, scale_down_bf16, bias_down_bf16, H, I, RowPlace{dn, kRowsPerDownBlock, g.rowb_i, g.D},
-         RowPlace{dn + kRowsPerDownBlock * g.rowb_i, kRowsPerDownBlock, g.sbb_i, g.D});
+  // gate/up tiles: gate rows then up rows of 8 units each
+  launch(TileSrc{{codes_gate, codes_up}, {u16(scale_gate_bf16), u16(scale_up_bf16)},
+                 {u16(bias_gate_bf16), u16(bias_up_bf16)}, 8},
+         I / 8, H, rec, g.U);
+  // down tiles: 16 rows each
+  launch(TileSrc{{codes_down, codes_down}, {u16(scale_down_bf16), u16(scale_down_bf16)},
+                 {u16(bias_down_bf16), u16(bias_down_bf16)}, 16},
+         H / kTileRows, I, rec + g.down_off, g.D);
   return launch_status();
 }
 
@@ -296,22 +294,21 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
   p.bits_r = L->bits_routed;
   p.bits_s = L->bits_shared;
   p.B = B;
-  const bool need4 = p.bits_r == 4 || p.bits_s == 4, need2 = p.bits_r == 2 || p.bits_s == 2;
-  const GuSmem gs = gu_smem_plan(p.H, need4, need2);
-  const DnSmem ds = dn_smem_plan(p.I, p.K);
-  if (ensure_smem(k_gate_up, gs.bytes) != MOE_OK || ensure_smem(k_down, ds.bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
+  const int gs_bytes = gu_smem_bytes(p.H, p.G);
+  const DnSmem ds = dn_smem_plan(p.I, p.K, p.G);
+  if (ensure_smem(k_gate_up, gs_bytes) != MOE_OK || ensure_smem(k_down, ds.bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
 
   // persistent grids: about two CTAs per SM in total, spread over the tokens
-  const int gu_units = (p.K + 1) * p.I, dn_units = (p.K + 1) * (p.H / kDownRows);
+  const int gu_tiles = (p.K + 1) * (p.I / 8), dn_jobs = (p.K + 1) * (p.H / kTileRows);
   const int per_tok = std::max(1, 2 * num_sms() / B);
-  const int gu_ctas = std::min(per_tok, (gu_units + kFfnWarps - 1) / kFfnWarps);
-  const int dn_ctas = std::min(per_tok, (dn_units + kFfnWarps - 1) / kFfnWarps);
-  p.units_per_cta_gu = (gu_units + gu_ctas - 1) / gu_ctas;
-  p.units_per_cta_dn = (dn_units + dn_ctas - 1) / dn_ctas;
+  const int gu_ctas = std::min(per_tok, gu_tiles);
+  const int dn_ctas = std::min(per_tok, dn_jobs);
+  p.tiles_per_cta_gu = (gu_tiles + gu_ctas - 1) / gu_ctas;
+  p.jobs_per_cta_dn = (dn_jobs + dn_ctas - 1) / dn_ctas;
   cudaStream_t s = (cudaStream_t)stream;
-  st = launch_pdl(k_gate_up, dim3(gu_ctas, B), dim3(kFfnWarps * 32), gs.bytes, s, p);
+  st = launch_pdl(k_gate_up, dim3(gu_ctas, B), dim3(kFfnWarps * 32), (size_t)gs_bytes, s, p);
   if (st != MOE_OK) return st;
-  return launch_pdl(k_down, dim3(dn_ctas, B), dim3(kFfnWarps * 32), ds.bytes, s, p);
+  return launch_pdl(k_down, dim3(dn_ctas, B), dim3(kFfnWarps * 32), (size_t)ds.bytes, s, p);
 }
 
 moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const float* w, const void* x_bf16,
@@ -370,26 +367,26 @@ bool stack_plan(StackParams& p, int G) {
     o += align_up(bytes, 128);
     return (int)at;
   };
-  p.need4 = (p.bits_r == 4 || p.bits_s == 4);
-  p.need2 = (p.bits_r == 2 || p.bits_s == 2);
+  auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
   p.sm_xs = take((size_t)H * 2);
-  p.sm_img4 = take(p.need4 ? img_bytes(H) : 0);
-  p.sm_tab4 = take(p.need4 ? tab_bytes(H, 4) : 0);
-  p.sm_inv4 = take(p.need4 ? inv_bytes(H, 4) : 0);
-  p.sm_img2 = take(p.need2 ? img_bytes(H) : 0);
-  p.sm_tab2 = take(p.need2 ? tab_bytes(H, 2) : 0);
-  p.sm_inv2 = take(p.need2 ? inv_bytes(H, 2) : 0);
-  p.himg_stride = (int)align_up(img_bytes(I), 128);
-  p.htab_stride = (int)align_up(tab_bytes(I, 4), 128);  // 4-bit has the most chunks
-  p.hinv_stride = (int)align_up(inv_bytes(I, 4), 128);
-  p.sm_himg = take((size_t)p.himg_stride * (K + 1));
-  p.sm_htab = take((size_t)p.htab_stride * (K + 1));
-  p.sm_hinv = take((size_t)p.hinv_stride * (K + 1));
-  const int nblk_max = (H / kDnBlk + G - 1) / G;
-  p.regc_slot_bytes = (int)align_up((size_t)nblk_max * std::max(p.geo_r.D, p.geo_s.D), 128);
-  p.sm_regc = take((size_t)p.regc_slot_bytes * (K + 1));
-  const size_t unit = std::max((size_t)2 * H * 2, (size_t)kPiecesPerItem * std::max(p.geo_r.U, p.geo_s.U));
-  p.slot_bytes = (int)align_up(unit, 128);
+  p.sm_xplanes = take(qimg_plane_bytes(H));
+  p.sm_xgs = take(qimg_gs_bytes(H, p.G));
+  p.hplanes_stride = (int)align_up(qimg_plane_bytes(I), 128);
+  p.hgs_stride = (int)align_up(qimg_gs_bytes(I, p.G), 128);
+  p.sm_hplanes = take((size_t)p.hplanes_stride * (K + 1));
+  p.sm_hgs = take((size_t)p.hgs_stride * (K + 1));
+  const int ntiles_max = cdiv(I / 8, G) + cdiv(K * (I / 8), G) + 1;
+  const int nd_max = cdiv(H / kTileRows, G);
+  if (ntiles_max > kMaxTiles || nd_max > kMaxDnTiles) return false;
+  p.sm_gpart = take((size_t)ntiles_max * kGuPieces * kTileRows * 4);
+  p.sm_dpart = take((size_t)nd_max * (K + 1) * kDnPieces * kTileRows * 4);
+  // a ring slot holds two router rows, half of a gate/up tile or the CTA's
+  // down tiles of one slot
+  const int ng = H / p.G;
+  const size_t half_tile = (size_t)std::max(quarter_lo(2, ng), ng - quarter_lo(2, ng)) *
+                           std::max(p.geo_r.blk, p.geo_s.blk);
+  const size_t down_item = (size_t)nd_max * std::max(p.geo_r.D, p.geo_s.D);
+  p.slot_bytes = (int)align_up(std::max(std::max((size_t)2 * H * 2, half_tile), down_item), 128);
   const size_t budget = 227 * 1024 - 6 * 1024;  // leave room for the static shared memory
   if (o + (size_t)p.slot_bytes * 2 > budget) return false;
   p.nslot = (int)std::min<size_t>(kMaxSlots, (budget - o) / p.slot_bytes);
@@ -426,10 +423,10 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   const int G = num_sms();
   auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
   if (L0.E > 1024 || cdiv(L0.E, G) > kMaxRouterRowsPerCta) return MOE_ERR_UNSUPPORTED;
-  if (cdiv(cdiv(L0.E, G), 2) + cdiv(cdiv(L0.I, G), kPiecesPerItem) + cdiv(cdiv(L0.K * L0.I, G), kPiecesPerItem) + L0.K >
-      kMaxItems)
+  const int tps = L0.I / 8;
+  if (cdiv(cdiv(L0.E, G), 2) + 2 * (cdiv(tps, G) + cdiv(L0.K * tps, G) + 1) + L0.K + 1 > kMaxItems)
     return MOE_ERR_UNSUPPORTED;
-  if (L0.H % 32 != 0) return MOE_ERR_UNSUPPORTED;
+  if (L0.H % 32 != 0 || L0.H / 16 > kCThreads) return MOE_ERR_UNSUPPORTED;
 
   StackParams p{};
   for (int l = 0; l < n_layers; ++l) {
@@ -463,7 +460,7 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   p.logits = reinterpret_cast<float*>((char*)ws + wl.logits);
   p.h = reinterpret_cast<float*>((char*)ws + wl.h);
   p.r = reinterpret_cast<float*>((char*)ws + wl.r);
-  p.ss = reinterpret_cast<float*>((char*)ws + wl.ss);
+  p.sync = reinterpret_cast<WsCtrl*>(ws)->sync;
   if (!stack_plan(p, G)) return MOE_ERR_UNSUPPORTED;
   const size_t smem = stack_smem_bytes(p);
   if (ensure_smem(k_decode_layers, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;

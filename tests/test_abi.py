@@ -50,12 +50,12 @@ def test_record_sizes_agree_with_oracle(moeq, ref):
         assert moeq.moe_expert_bytes(H, I, bits, group) == ref.expert_bytes(H, I, bits, group)
     assert moeq.moe_expert_bytes(4096, 1024, 4, 64) == 7077888
     lay = moeq.moe_expert_layout(4096, 1024, 4, 64)
-    # unit = gate row 2048 + up row 2048 + two table rows of 64 pairs; block = 4 down rows of 512 + 4 tables of 16 pairs
-    assert lay == [4608, 1024 * 4608, 4 * (512 + 64), 4, 2048, 512]
-    assert lay[1] + (4096 // 4) * lay[2] == 7077888
+    # 16-row tiles; one block per group: 32 lanes x 2 k-steps x 8 bytes + 8 x 8 bytes of tables
+    assert lay == [64 * 576, 128 * 64 * 576, 16 * 576, 16, 576, 128]
+    assert lay[1] + (4096 // 16) * lay[2] == 7077888
     assert moeq.moe_expert_bytes(4096, 1024, 3, 64) == 0
     assert moeq.moe_expert_bytes(4096, 1000, 4, 64) == 0
-    assert moeq.moe_expert_bytes(384, 128, 2, 128) == 0  # H/group odd: units would not be 16-byte multiples
+    assert moeq.moe_expert_bytes(384, 128, 2, 128) == ref.expert_bytes(384, 128, 2, 128)  # odd H/group is fine
 
 
 def test_workspace_size(moeq):

@@ -111,24 +111,51 @@ def test_pack_flags_out_of_range_code():
     assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK  # read clears it
 
 
+def decode_tiles(region, ntiles, C, bits, group):
+    """Codes [ntiles, 16, C] and (scale, bias) [ntiles, 16, C/group, 2] of a
+    run of record tiles, read back as the header documents them: per tile and
+    group a block of 32 lanes x (group/32 k-steps) of lane bytes, then eight
+    (row g, row g+8) pairs of bf16 (scale, bias); lane 4*g + t of k-step j
+    holds inputs 32j + 8t .. 32j + 8t + 7 of the group for local rows g and
+    g + 8."""
+    ks, ng = group // 32, C // group
+    wb = 8 if bits == 4 else 4
+    cb = 32 * ks * wb
+    blk = region[:ntiles * ng * (cb + 64)].reshape(ntiles, ng, cb + 64)
+    words = np.ascontiguousarray(blk[:, :, :cb]).view("<u4")
+    if bits == 4:
+        # [T, g, gid, t, j, h] words; nibble i = input 8t + i of local row gid + 8h
+        w = words.reshape(ntiles, ng, 8, 4, ks, 2)
+        v = (w[..., None] >> (4 * np.arange(8, dtype=np.uint32))) & 0xF      # [T, g, gid, t, j, h, i]
+        v = v.transpose(0, 5, 2, 1, 4, 3, 6)                                   # [T, h, gid, g, j, t, i]
+    else:
+        # one word: bits 8i + 4*odd + 2h hold input 8t + 2i + odd of local row gid + 8h
+        w = words.reshape(ntiles, ng, 8, 4, ks)
+        v = (w[..., None] >> (2 * np.arange(16, dtype=np.uint32))) & 0x3     # position 4i + 2*odd + h
+        v = v.reshape(ntiles, ng, 8, 4, ks, 4, 2, 2)                          # [T, g, gid, t, j, i, odd, h]
+        v = v.transpose(0, 7, 2, 1, 4, 3, 5, 6)                                # [T, h, gid, g, j, t, i, odd]
+    codes = v.reshape(ntiles, 16, C).astype(np.uint8)
+    sb = np.ascontiguousarray(blk[:, :, cb:]).view(np.uint16).reshape(ntiles, ng, 8, 2, 2)  # [T, g, gid, h, 2]
+    sb = sb.transpose(0, 3, 2, 1, 4).reshape(ntiles, 16, ng, 2)
+    return codes, sb
+
+
 def record_rows(rec, lay, H, I, bits, group):
-    """Read the gate/up/down code rows and table rows back out of one record
-    (numpy u8), following the layout moe_expert_layout describes."""
-    U, down_off, D, rpb, rowb_h, rowb_i = lay
-    sbb_h, sbb_i = H // group * 4, I // group * 4
-    units = rec[:I * U].reshape(I, U)
-    gate = units[:, :rowb_h]
-    up = units[:, rowb_h:2 * rowb_h]
-    gate_sb = units[:, 2 * rowb_h:2 * rowb_h + sbb_h].copy().view(np.uint16).reshape(I, -1, 2)
-    up_sb = units[:, 2 * rowb_h + sbb_h:].copy().view(np.uint16).reshape(I, -1, 2)
-    blocks = rec[down_off:down_off + (H // rpb) * D].reshape(H // rpb, D)
-    down = blocks[:, :rpb * rowb_i].reshape(H, rowb_i)
-    down_sb = blocks[:, rpb * rowb_i:].copy().view(np.uint16).reshape(H, -1, 2)
-    return (gate, gate_sb), (up, up_sb), (down, down_sb)
+    """Gate, up and down as (codes [rows, cols], (scale, bias) [rows, cols/group, 2])
+    read back out of one record (numpy u8) with the layout moe_expert_layout gives."""
+    U, down_off, D, rows_per_tile, blk, gu_tiles = lay
+    assert rows_per_tile == 16 and gu_tiles == I // 8
+    gc, gsb = decode_tiles(rec[:gu_tiles * U], gu_tiles, H, bits, group)
+    dc, dsb = decode_tiles(rec[down_off:down_off + (H // 16) * D], H // 16, I, bits, group)
+    gate = (gc[:, :8].reshape(I, H), gsb[:, :8].reshape(I, H // group, 2))
+    up = (gc[:, 8:].reshape(I, H), gsb[:, 8:].reshape(I, H // group, 2))
+    down = (dc.reshape(H, I), dsb.reshape(H, I // group, 2))
+    return gate, up, down
 
 
-@pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny", dict(bits_routed=2, bits_shared=2, group=64))])
-def test_packed_arena_matches_oracle_pack(name, over):
+@pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny", dict(bits_routed=2, bits_shared=2, group=64)),
+                                       ("tiny", dict(bits_routed=2, bits_shared=4, group=128))])
+def test_packed_arena_matches_generator(name, over):
     w = synth.WORKLOADS[name].with_(**over)
     L = hz.build_layer(w, 0)
     torch.cuda.synchronize()
@@ -139,9 +166,9 @@ def test_packed_arena_matches_oracle_pack(name, over):
         lay = L.lay_s if e == w.E else L.lay_r
         got = record_rows(rec, lay, w.H, w.I, w.bits_of(e), w.group)
         for m, (codes, scale, bias) in enumerate(synth.expert_host(w, 0, e)):
-            rp, rsb = ref.pack(codes, scale, bias, w.bits_of(e), w.group)
-            assert (got[m][0] == rp).all(), (e, m)
-            assert (got[m][1] == rsb).all(), (e, m)
+            assert (got[m][0] == codes).all(), (e, m)
+            assert (got[m][1][..., 0] == scale).all(), (e, m)
+            assert (got[m][1][..., 1] == bias).all(), (e, m)
 
 
 # ---- A1+A2 router ------------------------------------------------------------
