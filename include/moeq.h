@@ -75,20 +75,24 @@ typedef enum moe_status {
  * One MoE layer's resident weights (all pointers are device memory).
  *
  * Expert record (expert-major: each expert is one contiguous block, as in
- * LOOM's layout), for `bits` in {2, 4} and group size `group`. A code row
- * stores element c in byte floor(c*bits/8) at bit offset (c*bits) mod 8,
- * lowest bits first; a table row stores one bf16 pair (scale, bias) per
- * group of `group` inputs, scale first; the dequantised weight is
- * w = q*scale + bias with q unsigned. The record is laid out so that the
- * rows a kernel needs together are adjacent in memory:
- *   I gate/up units, unit i (U bytes) =
- *       [gate code row i][up code row i][gate table row i][up table row i]
- *   then H/4 down blocks, block b (D bytes) =
- *       [down code rows 4b..4b+3][down table rows 4b..4b+3]
- * with gate/up rows of H inputs and down rows of I inputs. moe_expert_layout
- * gives U, D and the offsets; moe_pack_expert writes a record. At H=4096,
- * I=1024, 4-bit, group 64 a record is 7,077,888 bytes (6.75 MiB), the
- * per-expert size the Flash-MoE page gives ("SSD Expert Streaming").
+ * LOOM's layout), for `bits` in {2, 4} and group size `group`; the
+ * dequantised weight is w = q*scale + bias with q unsigned and one bf16
+ * (scale, bias) pair per row and group of `group` inputs. Every matrix is
+ * stored as tiles of 16 rows laid out for the int8 tensor-core dot: a tile
+ * holds, for each group g, one block of
+ *   codes: 32 lanes x (group/32 k-steps) x W bytes (W = 8 at 4 bits, 4 at
+ *          2 bits); lane 4*r + t of k-step j holds the codes of inputs
+ *          g*group + 32j + 8t .. +7 of local rows r and r+8: at 4 bits two
+ *          words, input 8t+i at nibble i; at 2 bits one word, input 8t+2i of
+ *          row r at bits 8i, of row r+8 at 8i+2, input 8t+2i+1 of row r at
+ *          8i+4, of row r+8 at 8i+6
+ *   tables: 8 x [(scale, bias) of local row r][(scale, bias) of row r+8]
+ * The record is I/8 gate/up tiles of H inputs (tile T: gate rows 8T..8T+7
+ * as local rows 0..7, up rows 8T..8T+7 as 8..15), then H/16 down tiles of I
+ * inputs (tile T: rows 16T..16T+15). moe_expert_layout gives the sizes;
+ * moe_pack_expert writes a record. At H=4096, I=1024, 4-bit, group 64 a
+ * record is 7,077,888 bytes (6.75 MiB), the per-expert size the Flash-MoE
+ * page gives ("SSD Expert Streaming").
  */
 typedef struct moe_layer_q {
   int H;           /* hidden size; H*bits/8 and I*bits/8 multiples of 16 */
@@ -108,12 +112,12 @@ typedef struct moe_layer_q {
 size_t moe_expert_bytes(int H, int I, int bits, int group);
 
 /* Layout of one expert record (see moe_layer_q):
- *   lay[0] U, bytes of one gate/up unit
- *   lay[1] byte offset of the first down block (= I * U)
- *   lay[2] D, bytes of one down block
- *   lay[3] rows per down block (4)
- *   lay[4] bytes of one gate/up code row (H*bits/8): the up row's offset in a unit
- *   lay[5] bytes of one down code row (I*bits/8) */
+ *   lay[0] bytes of one gate/up tile ((H/group) blocks)
+ *   lay[1] byte offset of the first down tile (= lay[5] * lay[0])
+ *   lay[2] bytes of one down tile ((I/group) blocks)
+ *   lay[3] rows per tile (16)
+ *   lay[4] bytes of one block (codes, then 64 bytes of tables)
+ *   lay[5] gate/up tiles (I/8) */
 moe_status moe_expert_layout(int H, int I, int bits, int group, size_t lay[6]);
 
 /* Workspace bytes for calls on up to B tokens of this layer shape. */
@@ -178,9 +182,10 @@ moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B,
  *          the shared expert's (unweighted)
  * Per group of G inputs a row contributes scale*sum(q*x) + bias*sum(x): the
  * group-summed form of fma(q, scale*x, bias*x) (Flash-MoE page, section
- * "Kernel dequant toi uu FMA"); products are exact and accumulate in fp32.
- * The down projection reads h rounded to fp16 under a per-expert power-of-
- * two scale. An index outside [0,E) sets MOE_ERR_INDEX and zeroes that slot.
+ * "Kernel dequant toi uu FMA"). The inputs (x, then h) are rounded once to
+ * 16-bit fixed point per group; code x input products and their group sums
+ * are exact integers (tensor cores); scale, bias and the sum over groups are
+ * fp32. An index outside [0,E) sets MOE_ERR_INDEX and zeroes that slot.
  */
 moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx,
                             float* y_out, void* ws, size_t ws_bytes, void* stream);
@@ -218,7 +223,7 @@ moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const floa
  *   resid_out   fp32 [H]: r_n
  *   xnorm_bf16_out  bf16 [H] or NULL: bf16(RMSNorm(r_n))
  * Needs one CTA per SM for the whole launch (co-resident; cooperative
- * launch), E <= 1024, (H/group) % 4 == 0, and a shared-memory plan that fits
+ * launch), E <= 1024, H/16 <= 512, and a shared-memory plan that fits
  * one SM (MOE_ERR_UNSUPPORTED otherwise; use the per-call path). A wait that
  * exceeds about one second ends the kernel with MOE_ERR_TIMEOUT in the
  * workspace, which must then be re-initialised with moe_workspace_init.
