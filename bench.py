@@ -231,6 +231,20 @@ def per_call_path(w, layers, ws, dev, stream, steps):
     return steps / (ms / 1e3), statistics.mean(ffn_ms)
 
 
+def replica_rate(ms: float, steps: int, world: int, device=None):
+    """Whole-job rate of `world` independent replicas, each having run `steps`
+    layer-token steps in `ms` milliseconds of its own device time: the job
+    takes the slowest replica's time (max over ranks), and processes
+    world * steps units in it. Returns (max ms, units per second)."""
+    if world > 1:
+        import torch
+        import torch.distributed as dist
+        t = torch.tensor([ms], dtype=torch.float64, device=device)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        ms = float(t.item())
+    return ms, world * steps / (ms / 1e3)
+
+
 def kernel_source_digest() -> str:
     """Digest of the sources the fused decode kernel is built from."""
     import hashlib
@@ -322,10 +336,7 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
         err = moeq.moe_get_device_error(ws.buf, s)
         if err != moeq.MOE_OK:
             raise RuntimeError("device error in timed region: %s" % moeq.status_str(err))
-        if world > 1:
-            tt = torch.tensor([ms], device=dev)
-            dist.all_reduce(tt, op=dist.ReduceOp.MAX)
-            ms = float(tt.item())
+        ms, tps = replica_rate(ms, args.steps, world, dev)
         launches = full + (1 if rem else 0)
         del g_full, g_rem
 
@@ -363,7 +374,6 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
 
     step_bytes, rec_r, rec_s = algorithmic_bytes(w)
     peak, peak_src = peaks()
-    tps = world * args.steps / (ms / 1e3)
     achieved = step_bytes * args.steps / (ms / 1e3) / 1e9
     ffn_bytes = w.K * rec_r + rec_s
     resident = sum(L.nbytes() for L in layers)
