@@ -1,0 +1,284 @@
+// grouped.cuh -- moe_expert_ffn_q for a batch of tokens, grouped by expert:
+// each active expert's weights are read once per step for all the tokens
+// routed to it (the batched-decode token grouping; the pages themselves run
+// one token at a time).
+//
+//   k_group           stable counting sort of the (token, slot) picks by
+//                     expert id: cnt, off, list, and the active experts
+//   k_stage_batch     the input image of every token (x, or h per slot) in
+//                     the workspace, so that a tile can be applied to
+//                     several tokens without restaging
+//   k_gate_up_grp     unit = (expert, gate/up tile): the tile is read once;
+//                     four tokens share each mma (columns 2t, 2t+1 carry
+//                     token t's hi and lo planes); h per (token, slot)
+//   k_down_grp        unit = (expert, down tile): y per (token, slot)
+//
+// The expert list of a step is [shared, active routed experts in increasing
+// id]; the shared expert serves every token (slot K).
+#pragma once
+
+#include "common.cuh"
+#include "ffn.cuh"
+#include "tiledot.cuh"
+
+namespace moeq {
+
+constexpr int kGrpWarps = 8;
+constexpr int kGrpUnits = kGrpWarps / kFfnPieces;  // units per round (four warps each)
+constexpr int kGrpMaxTok = MOEQ_MAX_B;              // tokens of one expert at most
+
+// A routed expert with more than kGrpMaxTok entries (forced picks may repeat
+// an expert within a token) is split into several chunks; a chunk is one
+// work item.
+constexpr int kGrpExtraChunks = (MOEQ_MAX_B * MOEQ_MAX_K) / kGrpMaxTok;
+struct GrpWs {
+  int* cnt;   // [E]
+  int* off;   // [E + 1]
+  int* list;  // [B*K]: entries b*K + k grouped by expert, in entry order
+  int* act;   // [E + kGrpExtraChunks][3]: (expert, first entry in its list, entries) per chunk, by expert id
+  int* nact;  // [1]: chunks
+};
+
+struct GrpParams {
+  FfnParams f;
+  GrpWs g;
+  unsigned char* img;   // per-source images: x [B] (gate/up) or h [B][K+1] (down)
+  int img_stride;       // bytes between consecutive images
+  int img_gs_off;       // byte offset of the gs array within an image
+  int tps;              // tiles per expert (I/8 gate/up, H/16 down)
+  int max_units;        // (1 + most work items) * tps
+};
+
+// ---- grouping -------------------------------------------------------------
+
+// One CTA. Picks outside [0, E) set MOE_ERR_INDEX, are left out of every
+// group, and get a zero output slot here.
+__global__ void __launch_bounds__(256) k_group(const int32_t* idx, int B, int K, int E, int H, GrpWs g, float* y,
+                                               WsCtrl* ctrl) {
+  extern __shared__ int s_cnt[];  // [E + 1]
+  pdl_wait();
+  const int n = B * K;
+  for (int e = threadIdx.x; e <= E; e += blockDim.x) s_cnt[e] = 0;
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = idx[i];
+    if (e >= 0 && e < E) {
+      atomicAdd(&s_cnt[e], 1);
+    } else {
+      set_error(ctrl, MOE_ERR_INDEX);
+      float* yk = y + ((size_t)(i / K) * (K + 1) + (i % K)) * H;
+      for (int h = 0; h < H; ++h) yk[h] = 0.f;
+    }
+  }
+  __syncthreads();
+  if (threadIdx.x == 0) {
+    int o = 0, na = 0;
+    for (int e = 0; e < E; ++e) {
+      const int c = s_cnt[e];
+      g.cnt[e] = c;
+      g.off[e] = o;
+      for (int c0 = 0; c0 < c; c0 += kGrpMaxTok, ++na) {
+        g.act[3 * na] = e;
+        g.act[3 * na + 1] = c0;
+        g.act[3 * na + 2] = min(kGrpMaxTok, c - c0);
+      }
+      o += c;
+    }
+    g.off[E] = o;
+    g.nact[0] = na;
+  }
+  __syncthreads();
+  for (int i = threadIdx.x; i < n; i += blockDim.x) {
+    const int e = idx[i];
+    if (e < 0 || e >= E) continue;
+    int r = 0;
+    for (int j = 0; j < i; ++j) r += idx[j] == e;
+    g.list[g.off[e] + r] = i;
+  }
+  pdl_trigger();
+}
+
+// Images of B tokens' x (grid B) or of every (token, slot)'s h (grid
+// (B, K+1)): image b (or b*(K+1)+k) at img + index * stride.
+__global__ void __launch_bounds__(256) k_stage_batch(const void* src, int is_h, int n, int G, unsigned char* img,
+                                                     int stride, int gs_off) {
+  pdl_wait();
+  const int j = blockIdx.x * gridDim.y + blockIdx.y;
+  QImg Q{reinterpret_cast<uint2*>(img + (size_t)j * stride), reinterpret_cast<float2*>(img + (size_t)j * stride + gs_off)};
+  if (is_h) {
+    const float* h = reinterpret_cast<const float*>(src) + (size_t)j * n;
+    qstage_vector([&](int j0, float (&v)[16]) { load_f32_16_cg(h + j0, v); }, n, G, Q, threadIdx.x, blockDim.x);
+  } else {
+    const uint16_t* x = reinterpret_cast<const uint16_t*>(src) + (size_t)j * n;
+    qstage_vector([&](int j0, float (&v)[16]) { load_bf16_16(x + j0, v); }, n, G, Q, threadIdx.x, blockDim.x);
+  }
+  pdl_trigger();
+}
+
+// ---- the multi-token tile dot ---------------------------------------------
+
+// Blocks [0, nblk) of one tile in global memory against groups [g0, g0+nblk)
+// of up to four tokens' images (imgs[c], c < nt; the lanes of column pair c
+// read image c). Lane (gid, t) accumulates token t: acc0 for local row gid,
+// acc1 for row gid+8.
+template <int BITS, int KS>
+__device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int nblk, int g0,
+                                                const unsigned char* const (&imgs)[4], int gs_off, float& acc0,
+                                                float& acc1) {
+  using F = TileFmt<BITS, KS>;
+  constexpr int P = 4;
+  const int lane = threadIdx.x & 31, gid = lane >> 2, t = lane & 3;
+  // B fragments of column gid: token gid/2, plane hi (gid even) or lo
+  const uint2* planes = reinterpret_cast<const uint2*>(imgs[gid >> 1]) + (gid & 1) * 4 + t;
+  const float2* gs = reinterpret_cast<const float2*>(imgs[t] + gs_off);  // this lane's token
+  for (int b0 = 0; b0 < nblk; b0 += P) {
+    uint32_t w[P][F::LB / 4];
+    uint2 sb[P], bf[P][KS];
+    float2 ms[P];
+#pragma unroll
+    for (int q = 0; q < P; ++q) {
+      const int b = min(b0 + q, nblk - 1);
+      const unsigned char* blk = blk0 + (size_t)b * F::BB;
+      const unsigned char* cp = blk + lane * F::LB;
+      if (F::LB >= 16) {
+#pragma unroll
+        for (int i = 0; i < F::LB / 16; ++i) {
+          const uint4 v = ld_stream16(cp + 16 * i);
+          w[q][4 * i] = v.x;
+          w[q][4 * i + 1] = v.y;
+          w[q][4 * i + 2] = v.z;
+          w[q][4 * i + 3] = v.w;
+        }
+      } else if (F::LB == 8) {
+        const uint2 v = ld_stream8(cp);
+        w[q][0] = v.x;
+        w[q][1] = v.y;
+      } else {
+        w[q][0] = ld_stream4(cp);
+      }
+      sb[q] = ld_stream8(blk + F::CB + gid * 8);
+      const int g = g0 + b;
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) bf[q][ks] = __ldcg(planes + (size_t)(g * KS + ks) * 8);
+      ms[q] = __ldcg(gs + g);
+    }
+#pragma unroll
+    for (int q = 0; q < P; ++q) {
+      if (b0 + q >= nblk) continue;
+      int d[4];
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a[4];
+        extract_a<BITS>(w[q], ks, a);
+        mma_u8s8(d, a, bf[q][ks], ks > 0);
+      }
+      const float p0 = (float)(d[0] * 256 + d[1]) * ms[q].x;
+      const float p1 = (float)(d[2] * 256 + d[3]) * ms[q].x;
+      acc0 = fmaf(__uint_as_float(sb[q].x << 16), p0, acc0);
+      acc0 = fmaf(__uint_as_float(sb[q].x & 0xFFFF0000u), ms[q].y, acc0);
+      acc1 = fmaf(__uint_as_float(sb[q].y << 16), p1, acc1);
+      acc1 = fmaf(__uint_as_float(sb[q].y & 0xFFFF0000u), ms[q].y, acc1);
+    }
+  }
+}
+
+// Token i of work item a: its (batch index, output slot). a == 0 is the
+// shared expert (every token, slot K); a >= 1 is chunk a-1 of a routed expert.
+__device__ __forceinline__ void unit_token(const GrpParams& p, int a, int i, int& b, int& k) {
+  if (a == 0) {
+    b = i;
+    k = p.f.K;
+  } else {
+    const int* c = p.g.act + 3 * (a - 1);
+    const int ent = p.g.list[p.g.off[c[0]] + c[1] + i];
+    b = ent / p.f.K;
+    k = ent % p.f.K;
+  }
+}
+
+// ---- grouped gate/up and down -----------------------------------------------
+
+// DOWN == false: gate/up tiles against x images, h per (token, slot).
+// DOWN == true: down tiles against h images, y per (token, slot).
+template <bool DOWN>
+__global__ void __launch_bounds__(kGrpWarps * 32, 2) k_ffn_grp(GrpParams p) {
+  __shared__ float part[kGrpUnits][kFfnPieces][kGrpMaxTok][kTileRows];
+  __shared__ int s_tok[kGrpUnits][kGrpMaxTok][2];
+  const FfnParams& f = p.f;
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_wait();
+  const int nunits = min(p.max_units, (1 + p.g.nact[0]) * p.tps);
+  const int u_end = nunits;
+  // rounds of kGrpUnits consecutive units, dealt to the CTAs in turn
+  for (int u0 = blockIdx.x * kGrpUnits; u0 < nunits; u0 += gridDim.x * kGrpUnits) {
+    // the units of this round and their token lists
+    int ntok[kGrpUnits];
+#pragma unroll
+    for (int r = 0; r < kGrpUnits; ++r) {
+      const int u = u0 + r;
+      ntok[r] = 0;
+      if (u < u_end) {
+        const int a = u / p.tps;
+        ntok[r] = a == 0 ? f.B : p.g.act[3 * (a - 1) + 2];
+        for (int i = threadIdx.x; i < ntok[r]; i += blockDim.x) unit_token(p, a, i, s_tok[r][i][0], s_tok[r][i][1]);
+      }
+    }
+    __syncthreads();
+    const int r = warp / kFfnPieces, q = warp % kFfnPieces, u = u0 + r;
+    if (u < u_end) {
+      const int a = u / p.tps, T = u % p.tps;
+      const bool routed = a != 0;
+      const RecGeom& g = routed ? f.geo_r : f.geo_s;
+      const uint8_t* rec = routed ? f.experts + (size_t)p.g.act[3 * (a - 1)] * f.rec_r : f.shared;
+      const int ng = DOWN ? (int)g.ng_i : (int)g.ng_h;
+      const int g0 = piece_lo(q, ng), g1 = piece_lo(q + 1, ng);
+      const unsigned char* blk =
+          rec + (DOWN ? g.down_off + (size_t)T * g.D : (size_t)T * g.U) + (size_t)g0 * g.blk;
+      for (int c0 = 0; c0 < ntok[r]; c0 += 4) {
+        const unsigned char* imgs[4];
+#pragma unroll
+        for (int c = 0; c < 4; ++c) {
+          const int i = min(c0 + c, ntok[r] - 1);
+          const int src = DOWN ? s_tok[r][i][0] * (f.K + 1) + s_tok[r][i][1] : s_tok[r][i][0];
+          imgs[c] = p.img + (size_t)src * p.img_stride;
+        }
+        float acc0 = 0.f, acc1 = 0.f;
+        with_fmt(routed ? f.bits_r : f.bits_s, f.G, [&]<int BITS, int KS>() {
+          tile_dot_tokens<BITS, KS>(blk, g1 - g0, g0, imgs, p.img_gs_off, acc0, acc1);
+        });
+        const int i = c0 + (lane & 3);
+        if (i < ntok[r]) {
+          part[r][q][i][lane >> 2] = acc0;
+          part[r][q][i][(lane >> 2) + 8] = acc1;
+        }
+      }
+    }
+    __syncthreads();
+    // finish: gate/up -> h = silu(gate) * up for 8 units; down -> y rows
+#pragma unroll
+    for (int rr = 0; rr < kGrpUnits; ++rr) {
+      const int uu = u0 + rr;
+      if (uu >= u_end) continue;
+      const int T = uu % p.tps;
+      const int per = DOWN ? kTileRows : 8;
+      for (int j = threadIdx.x; j < ntok[rr] * per; j += blockDim.x) {
+        const int i = j / per, row = j % per;
+        const int b = s_tok[rr][i][0], k = s_tok[rr][i][1];
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int qq = 0; qq < kFfnPieces; ++qq) {
+          s0 += part[rr][qq][i][row];
+          if (!DOWN) s1 += part[rr][qq][i][row + 8];
+        }
+        if (DOWN)
+          f.y[((size_t)b * (f.K + 1) + k) * f.H + (size_t)T * kTileRows + row] = s0;
+        else
+          f.h[((size_t)b * (f.K + 1) + k) * f.I + 8 * T + row] = silu_f(s0) * s1;
+      }
+    }
+    __syncthreads();
+  }
+  pdl_trigger();
+}
+
+}  // namespace moeq

@@ -8,6 +8,7 @@
 #include "combine.cuh"
 #include "common.cuh"
 #include "ffn.cuh"
+#include "grouped.cuh"
 #include "pack.cuh"
 #include "router.cuh"
 #include "stack.cuh"
@@ -77,7 +78,11 @@ moe_status ensure_smem(K kern, size_t bytes) {
 // Workspace layout: [control 256 B][logits B*E fp32][h B*(K+1)*I fp32]
 //                   [r B*H fp32][ss kStackMaxLayers fp32]
 struct WsLayout {
-  size_t logits, h, r, ss, total;
+  size_t logits, h, r, ss;
+  size_t cnt, off, list, act, nact;  // token grouping (batches)
+  size_t ximg, himg;                 // per-token input images (batches)
+  int ximg_stride, ximg_gs, himg_stride, himg_gs;
+  size_t total;
 };
 inline WsLayout ws_layout(int B, int K, int H, int I, int E) {
   WsLayout l{};
@@ -90,6 +95,25 @@ inline WsLayout ws_layout(int B, int K, int H, int I, int E) {
   o += align_up((size_t)B * H * sizeof(float));
   l.ss = o;
   o += align_up((size_t)kStackMaxLayers * sizeof(float));
+  l.cnt = o;
+  o += align_up((size_t)E * 4);
+  l.off = o;
+  o += align_up((size_t)(E + 1) * 4);
+  l.list = o;
+  o += align_up((size_t)B * K * 4);
+  l.act = o;
+  o += align_up((size_t)(E + kGrpExtraChunks) * 3 * 4);
+  l.nact = o;
+  o += align_up(4);
+  // images: planes then (scale, sum) per group; the smallest group (32) sizes them
+  l.ximg_gs = (int)align_up(qimg_plane_bytes(H), 16);
+  l.ximg_stride = (int)align_up(l.ximg_gs + qimg_gs_bytes(H, 32), 256);
+  l.himg_gs = (int)align_up(qimg_plane_bytes(I), 16);
+  l.himg_stride = (int)align_up(l.himg_gs + qimg_gs_bytes(I, 32), 256);
+  l.ximg = o;
+  o += (size_t)B * l.ximg_stride;
+  l.himg = o;
+  o += (size_t)B * (K + 1) * l.himg_stride;
   l.total = o;
   return l;
 }
@@ -294,18 +318,53 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
   p.bits_r = L->bits_routed;
   p.bits_s = L->bits_shared;
   p.B = B;
+  cudaStream_t s = (cudaStream_t)stream;
+  if (B > 1) {
+    // a batch: group the picks by expert so that each active expert's tiles
+    // are read once for all its tokens
+    GrpParams gp{};
+    gp.f = p;
+    gp.g = GrpWs{reinterpret_cast<int*>((char*)ws + wl.cnt), reinterpret_cast<int*>((char*)ws + wl.off),
+                 reinterpret_cast<int*>((char*)ws + wl.list), reinterpret_cast<int*>((char*)ws + wl.act),
+                 reinterpret_cast<int*>((char*)ws + wl.nact)};
+    const int max_act = std::min(p.E, B * p.K) + kGrpExtraChunks;  // work items at most
+    const int ctas = 2 * num_sms();
+    st = launch_pdl(k_group, dim3(1), dim3(256), (size_t)(p.E + 1) * 4, s, idx, B, p.K, p.E, p.H, gp.g, y_out,
+                    p.ctrl);
+    if (st != MOE_OK) return st;
+    unsigned char* ximg = reinterpret_cast<unsigned char*>(ws) + wl.ximg;
+    unsigned char* himg = reinterpret_cast<unsigned char*>(ws) + wl.himg;
+    st = launch_pdl(k_stage_batch, dim3(B, 1), dim3(256), 0, s, x_bf16, 0, p.H, p.G, ximg, wl.ximg_stride,
+                    wl.ximg_gs);
+    if (st != MOE_OK) return st;
+    gp.img = ximg;
+    gp.img_stride = wl.ximg_stride;
+    gp.img_gs_off = wl.ximg_gs;
+    gp.tps = p.I / 8;
+    gp.max_units = (1 + max_act) * gp.tps;
+    st = launch_pdl(k_ffn_grp<false>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
+    if (st != MOE_OK) return st;
+    st = launch_pdl(k_stage_batch, dim3(B, p.K + 1), dim3(256), 0, s, (const void*)p.h, 1, p.I, p.G, himg,
+                    wl.himg_stride, wl.himg_gs);
+    if (st != MOE_OK) return st;
+    gp.img = himg;
+    gp.img_stride = wl.himg_stride;
+    gp.img_gs_off = wl.himg_gs;
+    gp.tps = p.H / kTileRows;
+    gp.max_units = (1 + max_act) * gp.tps;
+    return launch_pdl(k_ffn_grp<true>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
+  }
+
   const int gs_bytes = gu_smem_bytes(p.H, p.G);
   const DnSmem ds = dn_smem_plan(p.I, p.K, p.G);
   if (ensure_smem(k_gate_up, gs_bytes) != MOE_OK || ensure_smem(k_down, ds.bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
 
-  // persistent grids: about two CTAs per SM in total, spread over the tokens
+  // persistent grids: about two CTAs per SM in total
   const int gu_tiles = (p.K + 1) * (p.I / 8), dn_jobs = (p.K + 1) * (p.H / kTileRows);
-  const int per_tok = std::max(1, 2 * num_sms() / B);
-  const int gu_ctas = std::min(per_tok, gu_tiles);
-  const int dn_ctas = std::min(per_tok, dn_jobs);
+  const int gu_ctas = std::min(2 * num_sms(), gu_tiles);
+  const int dn_ctas = std::min(2 * num_sms(), dn_jobs);
   p.tiles_per_cta_gu = (gu_tiles + gu_ctas - 1) / gu_ctas;
   p.jobs_per_cta_dn = (dn_jobs + dn_ctas - 1) / dn_ctas;
-  cudaStream_t s = (cudaStream_t)stream;
   st = launch_pdl(k_gate_up, dim3(gu_ctas, B), dim3(kFfnWarps * 32), (size_t)gs_bytes, s, p);
   if (st != MOE_OK) return st;
   return launch_pdl(k_down, dim3(dn_ctas, B), dim3(kFfnWarps * 32), (size_t)ds.bytes, s, p);

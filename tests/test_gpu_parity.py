@@ -255,6 +255,34 @@ def test_expert_ffn_bad_index_zeroes_slot():
     assert (y[0, 1] == 0).all() and (y[0, 0] != 0).any() and (y[0, 2] != 0).any()
 
 
+def test_grouped_batch_repeats_and_bad_index():
+    """A full batch whose picks repeat one expert (so that expert has more
+    entries than one work item holds) plus one index out of range."""
+    w, L = get_layer("tiny")
+    B = moeq.MOEQ_MAX_B
+    x = hz.x_device(w, 77, B)
+    idx_np = np.full((B, w.K), 3, dtype=np.int32)
+    idx_np[:, -1] = (np.arange(B) % w.E).astype(np.int32)
+    idx_np[5, 1] = 99
+    idx = torch.from_numpy(idx_np).cuda()
+    ws = moeq.Workspace(B, w.K, w.H, w.I, w.E)
+    y = torch.full((B, w.K + 1, w.H), 7.0, dtype=torch.float32, device="cuda")
+    moeq.moe_expert_ffn_q(L.struct, x, B, idx, y, ws.buf, ws.nbytes)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_ERR_INDEX
+    yg = y.cpu().numpy()
+    assert (yg[5, 1] == 0).all()
+    experts = hz.oracle_experts(w, 0)
+    xb = synth.x_host(w, 77, B)
+    for b in (0, 5, 31, B - 1):
+        xd = hz.bf16_to_f64(xb[b])
+        for k, e in enumerate(list(idx_np[b]) + [w.E]):
+            if e >= w.E and k < w.K:
+                continue
+            g, u, d = experts(int(e))
+            yr = ref.expert_ffn(w.H, w.I, w.group, g, u, d, xd)
+            assert hz.max_rel_err(yg[b, k], yr) <= FFN_TOL, (b, k, e)
+
+
 # ---- A6 combine ------------------------------------------------------------------
 
 @pytest.mark.parametrize("with_gate,with_resid", [(False, False), (True, True)])
