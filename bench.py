@@ -36,9 +36,10 @@ def parse():
     ap.add_argument("--warmup", type=int, default=200)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="layer4", choices=["layer4", "layer2"])
-    ap.add_argument("--layers", type=int, default=16, help="resident layers walked by the steps")
+    ap.add_argument("--layers", type=int, default=24, help="resident layers walked by the steps")
     ap.add_argument("--cpu-sample", type=int, default=12, help="tokens in the oracle CPU-baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-extra", action="store_true", help="skip the C0/C2/C3/C4 report lines")
     return ap.parse_args()
 
 
@@ -245,6 +246,123 @@ def replica_rate(ms: float, steps: int, world: int, device=None):
     return ms, world * steps / (ms / 1e3)
 
 
+def timed_graph(stream, fn, reps: int = 2):
+    """Capture fn() (a sequence of launches on `stream`) in a CUDA graph, replay
+    it once to warm up, then time `reps` replays with events. Returns ms per replay."""
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    g.replay()
+    torch.cuda.synchronize()
+    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    a.record(stream)
+    for _ in range(reps):
+        g.replay()
+    b.record(stream)
+    torch.cuda.synchronize()
+    ms = a.elapsed_time(b) / reps
+    del g
+    return ms
+
+
+def extra_configs(layers, ws, dev, stream, peak):
+    """The other workloads, each timed on the device with the data resident:
+    C0 (tiny, fused), C2 (2-bit routed experts, fused, own arena), C3 (256
+    tokens through all resident layer4 layers with forced 27 %-overlap
+    routing), C4 (32 tokens per step, forced Zipf routing, grouped per-call
+    path). Returns a dict of report lines."""
+    import numpy as np
+    import torch
+
+    import quantized_expert_ffn_topk_b200 as moeq
+    from synth import synth
+    s = stream.cuda_stream
+    out = {}
+    eps = 1e-6
+
+    def decode_rate(w, Ls, steps_layers):
+        x = torch.empty(w.H, dtype=torch.bfloat16, device=dev)
+        synth.x_dev(w, 7, 1, x.data_ptr(), s)
+        r = x.float().clone()
+        structs = [L.struct for L in Ls]
+        reps = max(1, steps_layers // len(Ls))
+        ms = timed_graph(stream, lambda: [moeq.moe_decode_layers(structs, x, r, False, None, None, None, r, x, eps,
+                                                                 ws_w.buf, ws_w.nbytes, s) for _ in range(reps)])
+        return reps * len(Ls) / (ms / 1e3)
+
+    # C0: tiny, one layer, fused (parity workload; a latency figure)
+    w0 = synth.WORKLOADS["tiny"]
+    L0 = build_layers(w0, 1, dev, s)
+    ws_w = moeq.Workspace(1, w0.K, w0.H, w0.I, w0.E, device=dev, stream=s)
+    tps0 = decode_rate(w0, L0, 256)
+    b0 = algorithmic_bytes(w0)[0]
+    out["C0"] = {"workload": "tiny H256 E8 I128 top-2 + shared, 4-bit, group 32", "tokens_per_s": tps0,
+                 "step_bytes": b0, "gbs": b0 * tps0 / 1e9}
+    del L0
+
+    # C2: 2-bit routed experts (4-bit shared), own 8-layer arena
+    w2 = synth.WORKLOADS["layer2"]
+    L2 = build_layers(w2, 8, dev, s)
+    ws_w = moeq.Workspace(1, w2.K, w2.H, w2.I, w2.E, device=dev, stream=s)
+    tps2 = decode_rate(w2, L2, 8 * 64)
+    b2 = algorithmic_bytes(w2)[0]
+    out["C2"] = {"workload": "layer2: as layer4 with 2-bit routed experts (shared 4-bit)", "tokens_per_s": tps2,
+                 "step_bytes": b2, "gbs": b2 * tps2 / 1e9, "frac_of_measured_hbm": b2 * tps2 / 1e9 / peak,
+                 "layers_resident": 8}
+    del L2
+    torch.cuda.empty_cache()
+
+    # C3: 256 tokens x all resident layer4 layers, forced routing with 27 % overlap
+    w = synth.WORKLOADS["layer4"]
+    nl = len(layers)
+    T = 256
+    routing = synth.overlap_routing(w.E, w.K, T, nl, 0.27, seed=3)
+    rd = torch.from_numpy(np.ascontiguousarray(routing)).to(dev)
+    xs = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
+    synth.x_dev(w, 9000, T, xs.data_ptr(), s)
+    r3 = torch.empty(w.H, dtype=torch.float32, device=dev)
+    structs = [L.struct for L in layers]
+    ws_w = ws
+    ms3 = timed_graph(stream, lambda: [moeq.moe_decode_layers(structs, xs[t], None, False, rd[t], None, None, r3, None,
+                                                              eps, ws.buf, ws.nbytes, s) for t in range(T)])
+    tps3 = T / (ms3 / 1e3)
+    b3 = algorithmic_bytes(w)[0] * nl
+    out["C3"] = {"workload": "%d layer4 layers resident, %d tokens, forced routing (overlap %.3f measured)" %
+                             (nl, T, synth.measured_overlap(routing)),
+                 "tokens_per_s": tps3, "token_bytes": b3, "gbs": b3 * tps3 / 1e9,
+                 "frac_of_measured_hbm": b3 * tps3 / 1e9 / peak}
+
+    # C4: 32 tokens per step, forced Zipf(1.1) routing, grouped per-call path
+    B, S = 32, 2 * nl
+    zr = synth.zipf_routing(w.E, w.K, B, S, 1.1, seed=5)
+    zd = torch.from_numpy(np.ascontiguousarray(zr)).to(dev)
+    wsb = moeq.Workspace(B, w.K, w.H, w.I, w.E, device=dev, stream=s)
+    xb = torch.empty((B, w.H), dtype=torch.bfloat16, device=dev)
+    synth.x_dev(w, 12000, B, xb.data_ptr(), s)
+    resid = xb.float().clone()
+    outs = [L.alloc_outputs(B, logits=False, xnorm=True) for L in layers]
+
+    def c4():
+        for st in range(S):
+            l = st % nl
+            L, o = layers[l], outs[l]
+            moeq.moe_router_topk(xb, L.router_w, B, w.H, w.E, w.K, False, zd[st], o["idx"], o["w"], None, wsb.buf,
+                                 wsb.nbytes, s)
+            moeq.moe_expert_ffn_q(L.struct, xb, B, o["idx"], o["y"], wsb.buf, wsb.nbytes, s)
+            moeq.moe_combine_residual(L.struct, o["y"], o["w"], xb, resid, B, resid, o["xnorm"], eps, s)
+
+    ms4 = timed_graph(stream, c4)
+    tps4 = B * S / (ms4 / 1e3)
+    rec = algorithmic_bytes(w)[1]
+    distinct = float(np.mean([len(np.unique(zr[st])) for st in range(S)]))
+    b4 = w.E * w.H * 2 + (1 + distinct) * rec
+    out["C4"] = {"workload": "layer4, 32 tokens per step, forced Zipf(1.1) routing, grouped per expert",
+                 "tokens_per_s": tps4, "distinct_experts_per_step": distinct, "step_bytes": b4,
+                 "gbs": b4 * (S / (ms4 / 1e3)) / 1e9, "frac_of_measured_hbm": b4 * (S / (ms4 / 1e3)) / 1e9 / peak}
+    return out
+
+
 def kernel_source_digest() -> str:
     """Digest of the sources the fused decode kernel is built from."""
     import hashlib
@@ -372,6 +490,11 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
                    "d2h_bytes_per_step": w.H * 4, "steps": n_e2e,
                    "path": "moe_decode_layers (1 layer per call) with pinned host input/output copies"}
 
+        # the other workloads (report lines), on one GPU only
+        extra = None
+        if not args.no_extra and world == 1 and w.name == "layer4":
+            extra = extra_configs(layers, ws, dev, stream, peaks()[0])
+
     step_bytes, rec_r, rec_s = algorithmic_bytes(w)
     peak, peak_src = peaks()
     achieved = step_bytes * args.steps / (ms / 1e3) / 1e9
@@ -403,6 +526,8 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
     }
     if e2e is not None:
         line["e2e"] = e2e
+    if extra is not None:
+        line["configs"] = extra
     return line
 
 
