@@ -12,7 +12,7 @@
 //                 input) as a bf16 copy for the router and an image for the
 //                 tensor-core dots
 //   router        CTA c owns a contiguous range of router rows
-//   top-K         the producer warp of every CTA selects from all logits
+//   top-K         the compute warps of every CTA select from all logits
 //   shared expert gate/up tiles before the routing is known, then its down
 //                 tiles as soon as every CTA's shared h is out
 //   routed        gate/up tiles (slot-major ranges), then down tiles
@@ -246,114 +246,154 @@ __device__ bool issue_items(const StackParams& p, const ItemPlan& P, Ring& R, in
   return true;
 }
 
-// (a, ia) ranks before (b, ib): larger value, then lower index.
-__device__ __forceinline__ bool topk_before(float a, int ia, float b, int ib) { return a > b || (a == b && ia < ib); }
+// ---- softmax and top-K -------------------------------------------------------
 
-// Top-K (or forced picks) of layer l by the producer warp, once every CTA's
-// logits are out; registers only. Lane j holds experts j, j+32, ... (NaN and
-// padding as -inf, never picked). Writes s_idx (-1 for an invalid pick) and s_w.
-template <int NV>
-__device__ bool producer_topk_nv(const StackParams& p, int l, int* s_idx, float* s_w, const volatile int* abort) {
-  const int lane = threadIdx.x & 31;
-  bool ok = true;
-  if (lane == 0) ok = counter_wait(p.sync + kSyncLogits, (unsigned)(l + 1) * gridDim.x, abort);
-  if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) return false;
-  float v[NV];
-#pragma unroll
-  for (int j = 0; j < NV; ++j) {
-    const float x = lane + 32 * j < p.E ? __ldcg(p.logits + lane + 32 * j) : -INFINITY;
-    v[j] = x == x ? x : -INFINITY;
+// Order-preserving key of a logit (NaN already mapped to -inf): a larger value
+// has a larger key, -0 ranks as +0, and key 0 lies below every value ("taken").
+constexpr uint32_t kKeyNegInf = 0x007FFFFFu;  // the key of -inf
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  uint32_t u = __float_as_uint(v);
+  u = u == 0x80000000u ? 0u : u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+struct TopkScratch {
+  uint32_t key[kCWarps][MOEQ_MAX_K];  // each warp's K best, in rank order
+  int idx[kCWarps][MOEQ_MAX_K];
+  float m[kCWarps], z[kCWarps];       // each warp's max logit and sum of exp(v - max)
+};
+
+// Softmax and top-K of layer l's logits (router gating as the Flash-MoE page
+// gives it in "Metal Compute Shaders": softmax over all experts, the K
+// largest, weights renormalised on request), run by all compute warps of the
+// CTA. Thread t holds logits t and t + kCThreads; a warp takes its K best by
+// K rounds of a warp-wide max over the keys and a warp-wide min over the
+// indices holding it (ties go to the lower expert index), and warp 0 takes
+// the K best of the warps' candidates the same way. The top K of all logits
+// are among the warps' top K, so the picks are those of one global ranking.
+// The normaliser is summed per warp around the warp's own maximum and
+// rescaled to the global one. Warp 0 writes the picks and weights to
+// s_idx/s_w and then raises *ready to l + 1 for the producer warp.
+__device__ void block_topk(const StackParams& p, int l, TopkScratch& S, int* s_idx, float* s_w, volatile int* ready) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  const int E = p.E, K = p.K;
+  const int t1 = tid + kCThreads;
+  float v0 = -INFINITY, v1 = -INFINITY;
+  if (tid < E) {
+    const float x = __ldcg(p.logits + tid);
+    v0 = x == x ? x : -INFINITY;
   }
+  if (t1 < E) {
+    const float x = __ldcg(p.logits + t1);
+    v1 = x == x ? x : -INFINITY;
+  }
+  uint32_t k0 = tid < E ? logit_key(v0) : 0u, k1 = t1 < E ? logit_key(v1) : 0u;
+  const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, max(k0, k1));
+  const float mw = wm > kKeyNegInf ? key_logit(wm) : -INFINITY;
+  float zw = 0.f;
+  if (mw > -INFINITY) {  // warp-uniform
+    zw = (tid < E ? __expf(v0 - mw) : 0.f) + (t1 < E ? __expf(v1 - mw) : 0.f);
+    zw = warp_sum(zw);
+  }
+  if (!p.forced) {
+    uint32_t ck = 0u;
+    int ci = -1;
+    for (int kk = 0; kk < K; ++kk) {
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(k0, k1));
+      const uint32_t cand = k0 == m ? (uint32_t)tid : (k1 == m ? (uint32_t)t1 : 0xFFFFFFFFu);
+      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, cand);
+      if (bi == (uint32_t)tid) {
+        k0 = 0u;
+      } else if (bi == (uint32_t)t1) {
+        k1 = 0u;
+      }
+      if (lane == kk) {
+        ck = m;
+        ci = (int)bi;
+      }
+    }
+    if (lane < K) {
+      S.key[warp][lane] = ck;
+      S.idx[warp][lane] = ci;
+    }
+  }
+  if (lane == 0) {
+    S.m[warp] = mw;
+    S.z[warp] = zw;
+  }
+  named_sync(1, kCThreads);
+  if (warp != 0) return;
+
   float mx = -INFINITY;
 #pragma unroll
-  for (int j = 0; j < NV; ++j) mx = fmaxf(mx, v[j]);
-  mx = warp_max(mx);
-  float z = 0.f;
-#pragma unroll
-  for (int j = 0; j < NV; ++j) z += (lane + 32 * j < p.E) ? __expf(v[j] - mx) : 0.f;
+  for (int w = 0; w < kCWarps; ++w) mx = fmaxf(mx, S.m[w]);
+  float z = (lane < kCWarps && S.m[lane] > -INFINITY) ? S.z[lane] * __expf(S.m[lane] - mx) : 0.f;
   z = warp_sum(z);
-  const int32_t* forced = p.forced ? p.forced + (size_t)l * p.K : nullptr;
-  // the lane's best (value, slot j) by a tree over its NV values
-  auto lane_best = [&](float& bv, int& bj) {
-    float tv[NV];
-    int tj[NV];
-#pragma unroll
-    for (int j = 0; j < NV; ++j) {
-      tv[j] = v[j];
-      tj[j] = j;
-    }
-#pragma unroll
-    for (int w = NV / 2; w > 0; w >>= 1)
-#pragma unroll
-      for (int j = 0; j < w; ++j) {
-        const bool take = topk_before(tv[j + w], tj[j + w], tv[j], tj[j]);
-        tv[j] = take ? tv[j + w] : tv[j];
-        tj[j] = take ? tj[j + w] : tj[j];
-      }
-    bv = tv[0];
-    bj = tj[0];
-  };
-  float lv;
-  int lj;
-  lane_best(lv, lj);
   int pick_e = -1;     // lane k (< K) ends up holding pick k
   float pick_l = 0.f;  // and its logit
-  for (int k = 0; k < p.K; ++k) {
-    int bi;
-    float best;
-    if (forced) {
-      bi = forced[k];
-      const bool okf = bi >= 0 && bi < p.E;
-      best = okf ? __ldcg(p.logits + bi) : -INFINITY;
-      if (!okf) bi = -1;
-    } else {
-      best = lv;
-      bi = lane + 32 * lj;
-#pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        const float ov = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-        const int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-        if (topk_before(ov, oi, best, bi)) {
-          best = ov;
-          bi = oi;
-        }
-      }
-      if (!(best > -INFINITY)) {
-        bi = -1;  // no finite logit left: no expert
-      } else if ((bi & 31) == lane) {
-        const int jj = bi >> 5;  // remove the pick from its owner lane
-#pragma unroll
-        for (int j = 0; j < NV; ++j) v[j] = j == jj ? -INFINITY : v[j];
-        lane_best(lv, lj);
-      }
+  const int32_t* forced = p.forced ? p.forced + (size_t)l * K : nullptr;
+  if (forced) {
+    if (lane < K) {
+      const int bi = forced[lane];
+      const bool okf = bi >= 0 && bi < E;
+      pick_e = okf ? bi : -1;
+      pick_l = okf ? __ldcg(p.logits + bi) : -INFINITY;
     }
-    if (lane == k) {
-      pick_e = bi;
-      pick_l = best;
+  } else {
+    // candidate c = lane + 32 j: rank c % K of warp c / K
+    const int nc = kCWarps * K;
+    uint32_t ck[4];
+    uint32_t ci[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int c = lane + 32 * j;
+      ck[j] = c < nc ? S.key[c / K][c % K] : 0u;
+      ci[j] = c < nc ? (uint32_t)S.idx[c / K][c % K] : 0xFFFFFFFFu;
+    }
+    for (int kk = 0; kk < K; ++kk) {
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(max(ck[0], ck[1]), max(ck[2], ck[3])));
+      uint32_t cand = 0xFFFFFFFFu;
+#pragma unroll
+      for (int j = 0; j < 4; ++j) cand = ck[j] == m ? min(cand, ci[j]) : cand;
+      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, cand);
+#pragma unroll
+      for (int j = 0; j < 4; ++j) ck[j] = (ck[j] == m && ci[j] == bi) ? 0u : ck[j];
+      if (lane == kk) {
+        const bool fin = m > kKeyNegInf;  // no finite logit left: no expert
+        pick_e = fin ? (int)bi : -1;
+        pick_l = fin ? key_logit(m) : -INFINITY;
+      }
     }
   }
-  if (lane < p.K && pick_e < 0) set_error(p.ctrl, MOE_ERR_INDEX);
-  const float pw = (lane < p.K && pick_e >= 0) ? __expf(pick_l - mx) / z : 0.f;
+  if (lane < K && pick_e < 0) set_error(p.ctrl, MOE_ERR_INDEX);
+  const float pw = (lane < K && pick_e >= 0) ? __expf(pick_l - mx) / z : 0.f;
   const float tot = warp_sum(pw);
-  if (lane < p.K) {
+  if (lane < K) {
     const float wk = (p.renorm && tot > 0.f) ? pw / tot : pw;
     s_idx[lane] = pick_e;
     s_w[lane] = wk;
     if (blockIdx.x == 0) {
-      if (p.idx_out) p.idx_out[(size_t)l * p.K + lane] = forced ? forced[lane] : pick_e;
-      if (p.w_out) p.w_out[(size_t)l * p.K + lane] = wk;
+      if (p.idx_out) p.idx_out[(size_t)l * K + lane] = forced ? forced[lane] : pick_e;
+      if (p.w_out) p.w_out[(size_t)l * K + lane] = wk;
     }
   }
   __syncwarp();
-  return true;
+  __threadfence_block();
+  if (lane == 0) *ready = l + 1;
 }
 
-__device__ bool producer_topk(const StackParams& p, int l, int* s_idx, float* s_w, const volatile int* abort) {
-  const int nv = (p.E + 31) / 32;
-  if (nv <= 4) return producer_topk_nv<4>(p, l, s_idx, s_w, abort);
-  if (nv <= 8) return producer_topk_nv<8>(p, l, s_idx, s_w, abort);
-  if (nv <= 16) return producer_topk_nv<16>(p, l, s_idx, s_w, abort);
-  return producer_topk_nv<32>(p, l, s_idx, s_w, abort);
+// Bounded wait until the shared-memory flag reaches target.
+__device__ __forceinline__ bool flag_wait(const volatile int* f, int target, const volatile int* abort) {
+  if (*f >= target) return true;
+  const long long t0 = clock64();
+  while (*f < target) {
+    if (*abort || clock64() - t0 > kWaitBudgetCycles) return false;
+    __nanosleep(32);
+  }
+  return true;
 }
 
 // ---- compute pieces ------------------------------------------------------------
@@ -388,7 +428,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
   __shared__ float s_red[2][kCWarps];
   __shared__ unsigned char s_piece_item[kMaxPieces];
   __shared__ ItemPlan P;
+  __shared__ TopkScratch s_topk;
   __shared__ volatile int s_abort;
+  __shared__ volatile int s_topk_ready;
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;
@@ -404,6 +446,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     }
     for (int t = 0; t < kMaxTiles; ++t) s_gcnt[t] = 0;
     s_abort = 0;
+    s_topk_ready = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -419,9 +462,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     Ring R{full_bar, empty_bar, s_last, sm + p.sm_ring, p.slot_bytes, p.nslot};
     if (!issue_items(p, P, R, 0, 0, P.n_pre_items, 0u, s_idx, &s_abort) && lane == 0) fail();
     for (int l = 0; l < p.n_layers; ++l) {
-      // routing
-      if (!s_abort && !producer_topk(p, l, s_idx, s_w, &s_abort) && lane == 0) fail();
+      // routing: the compute warps publish layer l's picks in s_idx/s_w
+      if (lane == 0 && !s_abort && !flag_wait(&s_topk_ready, l + 1, &s_abort) && !s_abort) fail();
       __syncwarp();
+      __threadfence_block();
       // routed gate/up items (they gate the h exchange), the routed down
       // items (needed only after it), then the next layer's router, shared
       // gate/up and shared down items
@@ -649,6 +693,11 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       run_items(l, P.n_router_items, P.n_sgu_items);
       named_sync(1, kCThreads);
       if (tid == 0) arrive_release_gpu(p.sync + kSyncSharedH);
+
+      // ---- softmax / top-K over every CTA's logits (the producer waits for it) ----
+      if (tid == 0 && !counter_wait(p.sync + kSyncLogits, (unsigned)(l + 1) * G1, &s_abort) && !s_abort) fail();
+      named_sync(1, kCThreads);
+      block_topk(p, l, s_topk, s_idx, s_w, &s_topk_ready);
 
       // ---- the shared expert's down tiles, once every CTA's shared h is out ----
       stage_h(K, K + 1, kSyncSharedH, (unsigned)(l + 1) * G1);
