@@ -261,8 +261,8 @@ __device__ __forceinline__ float key_logit(uint32_t k) {
 }
 
 struct TopkScratch {
-  uint32_t key[kCWarps][MOEQ_MAX_K];  // each warp's K best, in rank order
-  int idx[kCWarps][MOEQ_MAX_K];
+  uint32_t key[kCWarps * MOEQ_MAX_K];  // warp w's K best at w*K .. w*K+K-1, in rank order
+  uint32_t idx[kCWarps * MOEQ_MAX_K];
   float m[kCWarps], z[kCWarps];       // each warp's max logit and sum of exp(v - max)
 };
 
@@ -316,8 +316,8 @@ __device__ void block_topk(const StackParams& p, int l, TopkScratch& S, int* s_i
       }
     }
     if (lane < K) {
-      S.key[warp][lane] = ck;
-      S.idx[warp][lane] = ci;
+      S.key[warp * K + lane] = ck;
+      S.idx[warp * K + lane] = (uint32_t)ci;
     }
   }
   if (lane == 0) {
@@ -343,15 +343,15 @@ __device__ void block_topk(const StackParams& p, int l, TopkScratch& S, int* s_i
       pick_l = okf ? __ldcg(p.logits + bi) : -INFINITY;
     }
   } else {
-    // candidate c = lane + 32 j: rank c % K of warp c / K
+    // candidate c = lane + 32 j of the warps' kCWarps * K
     const int nc = kCWarps * K;
     uint32_t ck[4];
     uint32_t ci[4];
 #pragma unroll
     for (int j = 0; j < 4; ++j) {
       const int c = lane + 32 * j;
-      ck[j] = c < nc ? S.key[c / K][c % K] : 0u;
-      ci[j] = c < nc ? (uint32_t)S.idx[c / K][c % K] : 0xFFFFFFFFu;
+      ck[j] = c < nc ? S.key[c] : 0u;
+      ci[j] = c < nc ? S.idx[c] : 0xFFFFFFFFu;
     }
     for (int kk = 0; kk < K; ++kk) {
       const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(max(ck[0], ck[1]), max(ck[2], ck[3])));
