@@ -166,7 +166,9 @@ moe_status moe_pack_expert(const uint8_t* codes_gate, const void* scale_gate_bf1
  *   w_out         fp32 [B, K]: softmax probability over all E of each pick;
  *                 divided by their sum when renorm != 0
  *   logits_out    fp32 [B, E] or NULL
- * Logits accumulate in fp32 (bf16 products are exact in fp32).
+ * Logits accumulate in fp32 (bf16 products are exact in fp32). NaN logits
+ * rank as -inf; a pick left with no finite logit is -1 and sets
+ * MOE_ERR_INDEX (its weight is 0).
  * Source: "Kien truc mo hinh" (512 experts, K active per token).
  */
 moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B, int H, int E, int K,

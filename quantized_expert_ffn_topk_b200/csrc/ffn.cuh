@@ -1,7 +1,15 @@
-// ffn.cuh -- moe_expert_ffn_q: gate/up dequant mat-vecs with fused SwiGLU,
-// then the down dequant mat-vec, for the K routed experts and the shared
-// expert of each token (the per-call path; the arithmetic of a tile is in
-// tiledot.cuh). Weights stream from global memory straight into registers.
+// ffn.cuh -- moe_expert_ffn_q for one token: gate/up dequant mat-vecs with
+// fused SwiGLU, then the down dequant mat-vec, for the K routed experts and
+// the shared expert (the per-call path; the arithmetic of a tile is in
+// tiledot.cuh; the steps are the Flash-MoE page's expert FFN, "Metal Compute
+// Shaders").
+//
+// One CTA per SM. A CTA takes a contiguous share of the layer's tiles (split
+// over all selected experts at once) and bulk-copies all of them into shared
+// memory up front, each tile completing on its own mbarrier; while the copies
+// are in flight it stages the input image, and its warps then take
+// quarter-tile pieces as the tiles land. A share that does not fit shared
+// memory is worked in rounds of as many tiles as fit.
 #pragma once
 
 #include "common.cuh"
@@ -9,9 +17,9 @@
 
 namespace moeq {
 
-constexpr int kFfnWarps = 8;
-constexpr int kFfnPieces = 4;   // warps per tile: each takes a quarter of the tile's groups
-constexpr int kFfnPrefetch = 4; // blocks in flight per warp
+constexpr int kFfnWarps = 16;
+constexpr int kFfnPieces = 4;     // pieces of a tile: each takes a quarter of its groups
+constexpr int kFfnMaxBuf = 32;    // tile buffers (mbarriers) per CTA
 
 struct FfnParams {
   const uint8_t* experts;    // E routed records
@@ -24,164 +32,203 @@ struct FfnParams {
   float* y;                  // [B, K+1, H]
   WsCtrl* ctrl;
   int H, I, E, K, G, bits_r, bits_s, B;
-  int tiles_per_cta_gu;      // gate/up tiles (slot-major, (K+1)*I/8 per token) per CTA
-  int jobs_per_cta_dn;       // down jobs (slot, tile), (K+1)*H/16 per token, per CTA
+  // shared-memory plans of the one-token kernels (byte offsets)
+  int gu_nbuf, gu_gs, gu_part, gu_tiles, gu_stride;
+  int dn_nbuf, dn_img_stride, dn_img_gs, dn_part, dn_tiles, dn_stride;
 };
 
 // Groups [lo, hi) of piece q of a tile with ng groups.
 __host__ __device__ inline int piece_lo(int q, int ng) { return q * ng / kFfnPieces; }
 
-// Shared memory of the gate/up kernel: x's image and the per-round partials.
-__host__ __device__ inline int gu_smem_bytes(int H, int G) {
-  return (int)(align_up(qimg_plane_bytes(H), 16) + align_up(qimg_gs_bytes(H, G), 16)) +
-         (kFfnWarps / kFfnPieces) * kFfnPieces * kTileRows * 4;
+// Record of slot k of the token (routed expert idx[k], or the shared expert
+// for k == K); null for an invalid expert index.
+__device__ __forceinline__ const uint8_t* ffn_slot_rec(const FfnParams& p, int k) {
+  if (k == p.K) return p.shared;
+  const int e = p.idx[k];
+  return (e >= 0 && e < p.E) ? p.experts + (size_t)e * p.rec_r : nullptr;
 }
 
-// Persistent over tiles: grid (ctas, B); CTA c takes tiles [c*tpc, (c+1)*tpc)
-// of token blockIdx.y, tile u = (slot u / (I/8), tile u % (I/8)). Each round
-// two tiles are split into four pieces, one per warp; the partial sums meet
-// in shared memory and 16 threads finish h for the two tiles' 16 units.
-__global__ void __launch_bounds__(kFfnWarps * 32, 2) k_gate_up(FfnParams p) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  QImg X{reinterpret_cast<uint2*>(smem),
-         reinterpret_cast<float2*>(smem + align_up(qimg_plane_bytes(p.H), 16))};
-  float* part = reinterpret_cast<float*>(smem + align_up(qimg_plane_bytes(p.H), 16) +
-                                         align_up(qimg_gs_bytes(p.H, p.G), 16));  // [2][4][16]
-  pdl_wait();
-  const uint16_t* xb = p.x + (size_t)b * p.H;
-  qstage_vector([&](int j0, float (&v)[16]) { load_bf16_16(xb + j0, v); }, p.H, p.G, X, threadIdx.x, blockDim.x);
-  __syncthreads();
-
-  const int tiles_per_slot = p.I / 8;
-  const int total = (p.K + 1) * tiles_per_slot;
-  const int t_begin = blockIdx.x * p.tiles_per_cta_gu;
-  const int t_end = min(total, t_begin + p.tiles_per_cta_gu);
-  constexpr int kPerRound = kFfnWarps / kFfnPieces;
-  for (int t0 = t_begin; t0 < t_end; t0 += kPerRound) {
-    const int u = t0 + warp / kFfnPieces, q = warp % kFfnPieces;
-    float acc0 = 0.f, acc1 = 0.f;
-    bool bad = false;
-    if (u < t_end) {
-      const int k = u / tiles_per_slot, T = u % tiles_per_slot;
-      const bool routed = k < p.K;
-      const int e = routed ? p.idx[(size_t)b * p.K + k] : 0;
-      bad = routed && (e < 0 || e >= p.E);
-      if (!bad) {
-        const uint8_t* rec = routed ? p.experts + (size_t)e * p.rec_r : p.shared;
-        const RecGeom& g = routed ? p.geo_r : p.geo_s;
-        const int g0 = piece_lo(q, g.ng_h), g1 = piece_lo(q + 1, g.ng_h);
-        const unsigned char* blk = rec + (size_t)T * g.U + (size_t)g0 * g.blk;
-        with_fmt(routed ? p.bits_r : p.bits_s, p.G, [&]<int BITS, int KS>() {
-          tile_dot_global<BITS, KS, kFfnPrefetch>(blk, g1 - g0, g0, X, acc0, acc1);
-        });
-      } else if (lane == 0 && q == 0) {
-        set_error(p.ctrl, MOE_ERR_INDEX);
-      }
-    }
-    if ((lane & 3) == 0) {
-      float* pp = part + ((warp / kFfnPieces) * kFfnPieces + q) * kTileRows;
-      pp[lane >> 2] = bad ? 0.f : acc0;
-      pp[(lane >> 2) + 8] = bad ? 0.f : acc1;
-    }
-    __syncthreads();
-    if (threadIdx.x < kPerRound * 8) {
-      const int r = threadIdx.x / 8, unit = threadIdx.x % 8, tu = t0 + r;
-      if (tu < t_end) {
-        float gate = 0.f, up = 0.f;
-#pragma unroll
-        for (int qq = 0; qq < kFfnPieces; ++qq) {
-          gate += part[(r * kFfnPieces + qq) * kTileRows + unit];
-          up += part[(r * kFfnPieces + qq) * kTileRows + 8 + unit];
-        }
-        const int k = tu / tiles_per_slot, T = tu % tiles_per_slot;
-        p.h[((size_t)b * (p.K + 1) + k) * p.I + 8 * T + unit] = silu_f(gate) * up;
-      }
-    }
-    __syncthreads();
+// Issue the bulk copies of tiles [u0, u0 + nt) of the CTA's share (lane j
+// copies tile u0 + j into buffer j; 0 bytes for an invalid expert). `src`
+// gives a tile's record, offset and size.
+template <typename Src>
+__device__ __forceinline__ void ffn_issue(unsigned char* tiles, int stride, uint64_t* bar, int u0, int nt, Src src) {
+  const int lane = threadIdx.x & 31;
+  for (int j = lane; j < nt; j += 32) {
+    const unsigned char* from = nullptr;
+    const uint32_t bytes = src(u0 + j, &from);
+    mbar_arrive_expect_tx(&bar[j], bytes);
+    if (bytes) bulk_g2s(tiles + (size_t)j * stride, from, bytes, &bar[j]);
   }
+}
+
+// Bounded wait for buffer j of the current round; on a timeout the CTA
+// records MOE_ERR_TIMEOUT and stops.
+__device__ __forceinline__ bool ffn_wait(uint64_t* bar, int j, int round, WsCtrl* ctrl, volatile int* abort) {
+  const bool ok = mbar_wait(&bar[j], (uint32_t)(round & 1), abort);
+  if (!ok && (threadIdx.x & 31) == 0) {
+    if (!*abort) set_error(ctrl, MOE_ERR_TIMEOUT);
+    *abort = 1;
+  }
+  return ok;
+}
+
+// Before the CTA leaves after a timeout: every copy it issued must have
+// landed (bounded).
+__device__ __forceinline__ void ffn_drain(uint64_t* bar, int nt, int round) {
+  if (threadIdx.x < nt) {
+    const long long t0 = clock64();
+    while (!mbar_try_wait(&bar[threadIdx.x], (uint32_t)(round & 1)) && clock64() - t0 < kWaitBudgetCycles) {
+    }
+  }
+}
+
+// Gate/up: tile u = (slot u / (I/8), tile u % (I/8)) holds gate rows 8T..8T+7
+// and up rows 8T..8T+7; 8 threads per tile finish h = SiLU(gate) * up.
+__global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_constant__ FfnParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bar[kFfnMaxBuf];
+  __shared__ volatile int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  const QImg X{reinterpret_cast<uint2*>(smem), reinterpret_cast<float2*>(smem + p.gu_gs)};
+  float* part = reinterpret_cast<float*>(smem + p.gu_part);  // [buffer][piece][16]
+  unsigned char* tiles = smem + p.gu_tiles;
+  const int tps = p.I / 8, total = (p.K + 1) * tps;
+  const int t_lo = (int)((long long)total * blockIdx.x / gridDim.x);
+  const int t_hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
+  if (tid == 0) {
+    for (int j = 0; j < p.gu_nbuf; ++j) mbar_init(&bar[j], 1);
+    s_abort = 0;
+    fence_mbar_init();
+  }
+  __syncthreads();
+  pdl_wait();
+  auto src = [&](int u, const unsigned char** from) -> uint32_t {
+    const int k = u / tps, T = u % tps;
+    const uint8_t* rec = ffn_slot_rec(p, k);
+    if (!rec) return 0u;
+    const RecGeom& g = k < p.K ? p.geo_r : p.geo_s;
+    *from = rec + (size_t)T * g.U;
+    return g.U;
+  };
+  int round = 0, nt = 0;
+  for (int r0 = t_lo; r0 < t_hi; r0 += p.gu_nbuf, ++round) {
+    nt = min(p.gu_nbuf, t_hi - r0);
+    if (warp == 0) ffn_issue(tiles, p.gu_stride, bar, r0, nt, src);
+    if (r0 == t_lo) {  // the input image, while the first round's tiles are in flight
+      qstage_vector([&](int j0, float (&v)[16]) { load_bf16_16(p.x + j0, v); }, p.H, p.G, X, tid, blockDim.x);
+      __syncthreads();
+    }
+    for (int pc = warp; pc < nt * kFfnPieces; pc += kFfnWarps) {
+      const int j = pc / kFfnPieces, q = pc % kFfnPieces, k = (r0 + j) / tps;
+      const bool routed = k < p.K;
+      float acc0 = 0.f, acc1 = 0.f;
+      if (ffn_wait(bar, j, round, p.ctrl, &s_abort) && ffn_slot_rec(p, k)) {
+        const RecGeom& g = routed ? p.geo_r : p.geo_s;
+        const int g0 = piece_lo(q, (int)g.ng_h), g1 = piece_lo(q + 1, (int)g.ng_h);
+        const unsigned char* blk = tiles + (size_t)j * p.gu_stride + (size_t)g0 * g.blk;
+        with_fmt(routed ? p.bits_r : p.bits_s, p.G,
+                 [&]<int BITS, int KS>() { tile_dot<BITS, KS>(blk, g1 - g0, g0, X, acc0, acc1); });
+      }
+      if ((lane & 3) == 0) {
+        float* pp = part + ((size_t)j * kFfnPieces + q) * kTileRows;
+        pp[lane >> 2] = acc0;
+        pp[(lane >> 2) + 8] = acc1;
+      }
+    }
+    __syncthreads();
+    for (int i = tid; i < nt * 8; i += blockDim.x) {
+      const int j = i / 8, unit = i % 8, u = r0 + j, k = u / tps, T = u % tps;
+      float gate = 0.f, up = 0.f;
+#pragma unroll
+      for (int q = 0; q < kFfnPieces; ++q) {
+        gate += part[((size_t)j * kFfnPieces + q) * kTileRows + unit];
+        up += part[((size_t)j * kFfnPieces + q) * kTileRows + 8 + unit];
+      }
+      const bool ok = ffn_slot_rec(p, k) != nullptr;
+      if (!ok && unit == 0) set_error(p.ctrl, MOE_ERR_INDEX);
+      p.h[(size_t)k * p.I + 8 * T + unit] = ok ? silu_f(gate) * up : 0.f;
+    }
+    __syncthreads();  // buffers and partials free for the next round
+    if (s_abort) break;
+  }
+  if (s_abort) ffn_drain(bar, nt, round);
   pdl_trigger();
 }
 
-// Shared memory of the down kernel: one image of h per slot, then partials.
-struct DnSmem {
-  int planes_stride, gs_off, gs_stride, part, bytes;
-};
-__host__ __device__ inline DnSmem dn_smem_plan(int I, int K, int G) {
-  DnSmem s{};
-  s.planes_stride = (int)align_up(qimg_plane_bytes(I), 16);
-  s.gs_off = s.planes_stride * (K + 1);
-  s.gs_stride = (int)align_up(qimg_gs_bytes(I, G), 16);
-  s.part = s.gs_off + s.gs_stride * (K + 1);
-  s.bytes = s.part + (kFfnWarps / kFfnPieces) * kFfnPieces * kTileRows * 4;
-  return s;
-}
-
-__device__ __forceinline__ QImg dn_img(unsigned char* smem, const DnSmem& sp, int k) {
-  return QImg{reinterpret_cast<uint2*>(smem + (size_t)k * sp.planes_stride),
-              reinterpret_cast<float2*>(smem + sp.gs_off + (size_t)k * sp.gs_stride)};
-}
-
-// Persistent over jobs: grid (ctas, B); job u = (slot u / (H/16), down tile
-// u % (H/16)). Two jobs per round, four pieces each; 32 threads sum the
-// pieces into y.
-__global__ void __launch_bounds__(kFfnWarps * 32, 2) k_down(FfnParams p) {
-  extern __shared__ __align__(16) unsigned char smem[];
-  const int b = blockIdx.y;
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const DnSmem sp = dn_smem_plan(p.I, p.K, p.G);
-  float* part = reinterpret_cast<float*>(smem + sp.part);
-  pdl_wait();
-  const float* hb = p.h + (size_t)b * (p.K + 1) * p.I;
-  for (int k = 0; k <= p.K; ++k) {
-    const float* hk = hb + (size_t)k * p.I;
-    qstage_vector([&](int j0, float (&v)[16]) { load_f32_16_cg(hk + j0, v); }, p.I, p.G, dn_img(smem, sp, k),
-                  threadIdx.x, blockDim.x);
+// Down: job u = (slot u / (H/16), down tile u % (H/16)); 16 threads per job
+// sum its pieces into y.
+__global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constant__ FfnParams p) {
+  extern __shared__ __align__(128) unsigned char smem[];
+  __shared__ __align__(8) uint64_t bar[kFfnMaxBuf];
+  __shared__ volatile int s_abort;
+  const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
+  float* part = reinterpret_cast<float*>(smem + p.dn_part);  // [buffer][piece][16]
+  unsigned char* tiles = smem + p.dn_tiles;
+  const int tpd = p.H / kTileRows, total = (p.K + 1) * tpd;
+  const int t_lo = (int)((long long)total * blockIdx.x / gridDim.x);
+  const int t_hi = (int)((long long)total * (blockIdx.x + 1) / gridDim.x);
+  auto img = [&](int k) {
+    return QImg{reinterpret_cast<uint2*>(smem + (size_t)k * p.dn_img_stride),
+                reinterpret_cast<float2*>(smem + (size_t)k * p.dn_img_stride + p.dn_img_gs)};
+  };
+  if (tid == 0) {
+    for (int j = 0; j < p.dn_nbuf; ++j) mbar_init(&bar[j], 1);
+    s_abort = 0;
+    fence_mbar_init();
   }
   __syncthreads();
-
-  const int tiles_per_slot = p.H / kTileRows;
-  const int total = (p.K + 1) * tiles_per_slot;
-  const int j_begin = blockIdx.x * p.jobs_per_cta_dn;
-  const int j_end = min(total, j_begin + p.jobs_per_cta_dn);
-  constexpr int kPerRound = kFfnWarps / kFfnPieces;
-  for (int j0 = j_begin; j0 < j_end; j0 += kPerRound) {
-    const int u = j0 + warp / kFfnPieces, q = warp % kFfnPieces;
-    float acc0 = 0.f, acc1 = 0.f;
-    if (u < j_end) {
-      const int k = u / tiles_per_slot, T = u % tiles_per_slot;
+  pdl_wait();
+  auto src = [&](int u, const unsigned char** from) -> uint32_t {
+    const int k = u / tpd, T = u % tpd;
+    const uint8_t* rec = ffn_slot_rec(p, k);
+    if (!rec) return 0u;
+    const RecGeom& g = k < p.K ? p.geo_r : p.geo_s;
+    *from = rec + g.down_off + (size_t)T * g.D;
+    return g.D;
+  };
+  int round = 0, nt = 0;
+  for (int r0 = t_lo; r0 < t_hi; r0 += p.dn_nbuf, ++round) {
+    nt = min(p.dn_nbuf, t_hi - r0);
+    if (warp == 0) ffn_issue(tiles, p.dn_stride, bar, r0, nt, src);
+    if (r0 == t_lo) {  // images of the slots this CTA's jobs touch
+      for (int k = t_lo / tpd; k <= (t_hi - 1) / tpd; ++k) {
+        const float* hk = p.h + (size_t)k * p.I;
+        qstage_vector([&](int j0, float (&v)[16]) { load_f32_16_cg(hk + j0, v); }, p.I, p.G, img(k), tid,
+                      blockDim.x);
+      }
+      __syncthreads();
+    }
+    for (int pc = warp; pc < nt * kFfnPieces; pc += kFfnWarps) {
+      const int j = pc / kFfnPieces, q = pc % kFfnPieces, k = (r0 + j) / tpd;
       const bool routed = k < p.K;
-      const int e = routed ? p.idx[(size_t)b * p.K + k] : 0;
-      if (!routed || (e >= 0 && e < p.E)) {
-        const uint8_t* rec = routed ? p.experts + (size_t)e * p.rec_r : p.shared;
+      float acc0 = 0.f, acc1 = 0.f;
+      if (ffn_wait(bar, j, round, p.ctrl, &s_abort) && ffn_slot_rec(p, k)) {
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
-        const int g0 = piece_lo(q, g.ng_i), g1 = piece_lo(q + 1, g.ng_i);
-        const unsigned char* blk = rec + g.down_off + (size_t)T * g.D + (size_t)g0 * g.blk;
-        const QImg Xk = dn_img(smem, sp, k);
-        with_fmt(routed ? p.bits_r : p.bits_s, p.G, [&]<int BITS, int KS>() {
-          tile_dot_global<BITS, KS, kFfnPrefetch>(blk, g1 - g0, g0, Xk, acc0, acc1);
-        });
+        const int g0 = piece_lo(q, (int)g.ng_i), g1 = piece_lo(q + 1, (int)g.ng_i);
+        const unsigned char* blk = tiles + (size_t)j * p.dn_stride + (size_t)g0 * g.blk;
+        const QImg Hk = img(k);
+        with_fmt(routed ? p.bits_r : p.bits_s, p.G,
+                 [&]<int BITS, int KS>() { tile_dot<BITS, KS>(blk, g1 - g0, g0, Hk, acc0, acc1); });
+      }
+      if ((lane & 3) == 0) {
+        float* pp = part + ((size_t)j * kFfnPieces + q) * kTileRows;
+        pp[lane >> 2] = acc0;
+        pp[(lane >> 2) + 8] = acc1;
       }
     }
-    if ((lane & 3) == 0) {
-      float* pp = part + ((warp / kFfnPieces) * kFfnPieces + q) * kTileRows;
-      pp[lane >> 2] = acc0;
-      pp[(lane >> 2) + 8] = acc1;
-    }
     __syncthreads();
-    if (threadIdx.x < kPerRound * kTileRows) {
-      const int r = threadIdx.x / kTileRows, rho = threadIdx.x % kTileRows, ju = j0 + r;
-      if (ju < j_end) {
-        float y = 0.f;
+    for (int i = tid; i < nt * kTileRows; i += blockDim.x) {
+      const int j = i / kTileRows, rho = i % kTileRows, u = r0 + j, k = u / tpd, T = u % tpd;
+      float y = 0.f;
 #pragma unroll
-        for (int qq = 0; qq < kFfnPieces; ++qq) y += part[(r * kFfnPieces + qq) * kTileRows + rho];
-        const int k = ju / tiles_per_slot, T = ju % tiles_per_slot;
-        p.y[((size_t)b * (p.K + 1) + k) * p.H + (size_t)T * kTileRows + rho] = y;
-      }
+      for (int q = 0; q < kFfnPieces; ++q) y += part[((size_t)j * kFfnPieces + q) * kTileRows + rho];
+      p.y[(size_t)k * p.H + (size_t)T * kTileRows + rho] = y;
     }
     __syncthreads();
+    if (s_abort) break;
   }
+  if (s_abort) ffn_drain(bar, nt, round);
   pdl_trigger();
 }
 

@@ -131,6 +131,8 @@ moe_status check_layer(const moe_layer_q* L) {
   return MOE_OK;
 }
 
+bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes);  // below
+
 }  // namespace
 }  // namespace moeq
 
@@ -355,19 +357,14 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     return launch_pdl(k_ffn_grp<true>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
   }
 
-  const int gs_bytes = gu_smem_bytes(p.H, p.G);
-  const DnSmem ds = dn_smem_plan(p.I, p.K, p.G);
-  if (ensure_smem(k_gate_up, gs_bytes) != MOE_OK || ensure_smem(k_down, ds.bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
-
-  // persistent grids: about two CTAs per SM in total
+  // one token: every CTA bulk-copies its share of whole tiles into shared memory
+  size_t gu_bytes = 0, dn_bytes = 0;
+  if (!ffn_plan(p, num_sms(), gu_bytes, dn_bytes)) return MOE_ERR_UNSUPPORTED;
+  if (ensure_smem(k_gate_up, gu_bytes) != MOE_OK || ensure_smem(k_down, dn_bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
   const int gu_tiles = (p.K + 1) * (p.I / 8), dn_jobs = (p.K + 1) * (p.H / kTileRows);
-  const int gu_ctas = std::min(2 * num_sms(), gu_tiles);
-  const int dn_ctas = std::min(2 * num_sms(), dn_jobs);
-  p.tiles_per_cta_gu = (gu_tiles + gu_ctas - 1) / gu_ctas;
-  p.jobs_per_cta_dn = (dn_jobs + dn_ctas - 1) / dn_ctas;
-  st = launch_pdl(k_gate_up, dim3(gu_ctas, B), dim3(kFfnWarps * 32), (size_t)gs_bytes, s, p);
+  st = launch_pdl(k_gate_up, dim3(std::min(num_sms(), gu_tiles)), dim3(kFfnWarps * 32), gu_bytes, s, p);
   if (st != MOE_OK) return st;
-  return launch_pdl(k_down, dim3(dn_ctas, B), dim3(kFfnWarps * 32), (size_t)ds.bytes, s, p);
+  return launch_pdl(k_down, dim3(std::min(num_sms(), dn_jobs)), dim3(kFfnWarps * 32), dn_bytes, s, p);
 }
 
 moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const float* w, const void* x_bf16,
@@ -416,6 +413,40 @@ moe_status moe_get_device_error(void* ws, void* stream) {
 
 namespace moeq {
 namespace {
+
+// Shared-memory plans of the one-token gate/up and down kernels: the input
+// image(s), the pieces' partial sums and as many tile buffers as the CTA's
+// share needs (at most kFfnMaxBuf, and what fits). False when not one fits.
+bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes) {
+  const size_t budget = 227 * 1024 - 2 * 1024;  // leave room for the static shared memory
+  auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
+  const int gu_total = (p.K + 1) * (p.I / 8), dn_total = (p.K + 1) * (p.H / kTileRows);
+  // gate/up
+  size_t o = align_up(qimg_plane_bytes(p.H), 128);
+  p.gu_gs = (int)o;
+  o += align_up(qimg_gs_bytes(p.H, p.G), 128);
+  const int gu_want = std::min(kFfnMaxBuf, cdiv(gu_total, std::min(G, gu_total)));
+  p.gu_part = (int)o;
+  o += align_up((size_t)gu_want * kFfnPieces * kTileRows * 4, 128);
+  p.gu_tiles = (int)o;
+  p.gu_stride = (int)align_up(std::max(p.geo_r.U, p.geo_s.U), 128);
+  if (o + (size_t)p.gu_stride > budget) return false;
+  p.gu_nbuf = (int)std::min<size_t>(gu_want, (budget - o) / p.gu_stride);
+  gu_bytes = o + (size_t)p.gu_nbuf * p.gu_stride;
+  // down
+  p.dn_img_gs = (int)align_up(qimg_plane_bytes(p.I), 128);
+  p.dn_img_stride = p.dn_img_gs + (int)align_up(qimg_gs_bytes(p.I, p.G), 128);
+  o = (size_t)p.dn_img_stride * (p.K + 1);
+  const int dn_want = std::min(kFfnMaxBuf, cdiv(dn_total, std::min(G, dn_total)));
+  p.dn_part = (int)o;
+  o += align_up((size_t)dn_want * kFfnPieces * kTileRows * 4, 128);
+  p.dn_tiles = (int)o;
+  p.dn_stride = (int)align_up(std::max(p.geo_r.D, p.geo_s.D), 128);
+  if (o + (size_t)p.dn_stride > budget) return false;
+  p.dn_nbuf = (int)std::min<size_t>(dn_want, (budget - o) / p.dn_stride);
+  dn_bytes = o + (size_t)p.dn_nbuf * p.dn_stride;
+  return true;
+}
 
 // Shared-memory plan of the fused decode kernel; false when it does not fit.
 bool stack_plan(StackParams& p, int G) {

@@ -33,18 +33,41 @@ __device__ __forceinline__ float dot8_bf16(uint4 wv, const uint4 xv, float acc) 
   return acc;
 }
 
-// Top-K of one token's logits by one warp: K rounds of a warp arg-max with
-// ties to the lower index, then softmax weights at the picks.
+// Order-preserving key of a logit (NaN read as -inf): a larger value has a
+// larger key, -0 ranks as +0, and key 0 lies below every value ("taken").
+constexpr uint32_t kKeyNegInf = 0x007FFFFFu;  // the key of -inf
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  uint32_t u = __float_as_uint(v == v ? v : -INFINITY);
+  u = u == 0x80000000u ? 0u : u;
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
+// Top-K of one token's logits (E <= 1024) by one warp, softmax weights at
+// the picks (router gating of the Flash-MoE page, "Metal Compute Shaders").
+// Lane l keeps the keys of logits l + 32 j in registers; each of the K rounds
+// takes a warp-wide max over the keys and a warp-wide min over the indices
+// holding it (ties go to the lower index), and the owner lane clears its key.
 __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const int32_t* forced, int32_t* idx_out,
                                float* w_out, WsCtrl* ctrl) {
   const int lane = threadIdx.x & 31;
-  int picked[MOEQ_MAX_K];
-  float mx = -INFINITY;
-  for (int e = lane; e < E; e += 32) mx = fmaxf(mx, lg[e]);
-  mx = warp_max(mx);
+  constexpr int NV = 32;
+  uint32_t key[NV];
+  uint32_t lk = 0u;
+#pragma unroll
+  for (int j = 0; j < NV; ++j) {
+    const int e = lane + 32 * j;
+    key[j] = e < E ? logit_key(lg[e]) : 0u;
+    lk = max(lk, key[j]);
+  }
+  const uint32_t m0 = __reduce_max_sync(0xFFFFFFFFu, lk);
+  const float mx = m0 > kKeyNegInf ? key_logit(m0) : -INFINITY;
   float z = 0.f;
   for (int e = lane; e < E; e += 32) z += expf(lg[e] - mx);
   z = warp_sum(z);
+  int picked[MOEQ_MAX_K];
   if (forced) {
     for (int k = 0; k < K; ++k) {
       int e = forced[k];
@@ -56,31 +79,25 @@ __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const 
     }
   } else {
     for (int k = 0; k < K; ++k) {
-      float best = -INFINITY;
-      int bi = 0x7FFFFFFF;
-      for (int e = lane; e < E; e += 32) {
-        bool taken = false;
-        for (int j = 0; j < k; ++j) taken |= (picked[j] == e);
-        float v = lg[e];
-        if (!taken && (v > best || (v == best && e < bi))) {
-          best = v;
-          bi = e;
-        }
-      }
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, lk);
+      uint32_t cand = 0xFFFFFFFFu;
 #pragma unroll
-      for (int o = 16; o > 0; o >>= 1) {
-        float ov = __shfl_xor_sync(0xFFFFFFFFu, best, o);
-        int oi = __shfl_xor_sync(0xFFFFFFFFu, bi, o);
-        if (ov > best || (ov == best && oi < bi)) {
-          best = ov;
-          bi = oi;
+      for (int j = NV - 1; j >= 0; --j) cand = key[j] == m ? (uint32_t)(lane + 32 * j) : cand;
+      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, cand);
+      if ((bi & 31u) == (uint32_t)lane) {
+        lk = 0u;
+#pragma unroll
+        for (int j = 0; j < NV; ++j) {
+          key[j] = j == (int)(bi >> 5) ? 0u : key[j];
+          lk = max(lk, key[j]);
         }
       }
-      if (bi < 0 || bi >= E) {  // no finite logit left (NaN input): no expert
+      if (m > kKeyNegInf) {
+        picked[k] = (int)bi;
+      } else {  // no finite logit left (NaN input): no expert
         if (lane == 0) set_error(ctrl, MOE_ERR_INDEX);
-        bi = -1;
+        picked[k] = -1;
       }
-      picked[k] = bi;
     }
   }
   float p[MOEQ_MAX_K];

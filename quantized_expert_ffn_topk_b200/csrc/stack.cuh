@@ -248,18 +248,6 @@ __device__ bool issue_items(const StackParams& p, const ItemPlan& P, Ring& R, in
 
 // ---- softmax and top-K -------------------------------------------------------
 
-// Order-preserving key of a logit (NaN already mapped to -inf): a larger value
-// has a larger key, -0 ranks as +0, and key 0 lies below every value ("taken").
-constexpr uint32_t kKeyNegInf = 0x007FFFFFu;  // the key of -inf
-__device__ __forceinline__ uint32_t logit_key(float v) {
-  uint32_t u = __float_as_uint(v);
-  u = u == 0x80000000u ? 0u : u;
-  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
-}
-__device__ __forceinline__ float key_logit(uint32_t k) {
-  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
-}
-
 struct TopkScratch {
   uint32_t key[kCWarps * MOEQ_MAX_K];  // warp w's K best at w*K .. w*K+K-1, in rank order
   uint32_t idx[kCWarps * MOEQ_MAX_K];

@@ -244,46 +244,6 @@ __device__ __forceinline__ void tile_dot(const unsigned char* blk0, int nblk, in
   }
 }
 
-// The same over blocks in global memory, streamed: the codes and tables of P
-// blocks are loaded before any of them is used.
-template <int BITS, int KS, int P>
-__device__ __forceinline__ void tile_dot_global(const unsigned char* blk0, int nblk, int g0, const QImg& X,
-                                                float& acc0, float& acc1) {
-  using F = TileFmt<BITS, KS>;
-  const int lane = threadIdx.x & 31;
-  for (int b0 = 0; b0 < nblk; b0 += P) {
-    uint32_t w[P][F::LB / 4];
-    uint2 sb[P];
-#pragma unroll
-    for (int q = 0; q < P; ++q) {
-      if (b0 + q < nblk) {
-        const unsigned char* blk = blk0 + (size_t)(b0 + q) * F::BB;
-        const unsigned char* cp = blk + lane * F::LB;
-        if (F::LB >= 16) {
-#pragma unroll
-          for (int i = 0; i < F::LB / 16; ++i) {
-            const uint4 v = ld_stream16(cp + 16 * i);
-            w[q][4 * i] = v.x;
-            w[q][4 * i + 1] = v.y;
-            w[q][4 * i + 2] = v.z;
-            w[q][4 * i + 3] = v.w;
-          }
-        } else if (F::LB == 8) {
-          const uint2 v = ld_stream8(cp);
-          w[q][0] = v.x;
-          w[q][1] = v.y;
-        } else {
-          w[q][0] = ld_stream4(cp);
-        }
-        sb[q] = ld_stream8(blk + F::CB + (lane >> 2) * 8);
-      }
-    }
-#pragma unroll
-    for (int q = 0; q < P; ++q)
-      if (b0 + q < nblk) block_acc<BITS, KS>(w[q], sb[q], g0 + b0 + q, X, acc0, acc1);
-  }
-}
-
 // Dispatch on (bits, group) for callers with runtime values.
 template <typename Fn>
 __device__ __forceinline__ void with_fmt(int bits, int G, Fn fn) {
