@@ -9,6 +9,7 @@
 namespace moeq {
 
 constexpr int kCombineThreads = 512;
+constexpr int kCombineU = 8;  // elements per thread per pass (one pass covers H <= 4096)
 
 struct CombineParams {
   const float* y;          // [B, K+1, H]
@@ -22,10 +23,13 @@ struct CombineParams {
   float eps;
 };
 
-// grid: B CTAs, one token each.
+// grid: B CTAs, one token each. A thread keeps the outputs of its first pass
+// in registers for the RMSNorm'd copy; only when H > kCombineThreads *
+// kCombineU does it read later ones back (each thread only what it wrote).
 __global__ void __launch_bounds__(kCombineThreads) k_combine(CombineParams p) {
   __shared__ float red[32];
   const int b = blockIdx.x;
+  pdl_trigger();
   pdl_wait();
   const uint16_t* xb = p.x + (size_t)b * p.H;
   float gamma = 1.f;
@@ -36,46 +40,52 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(CombineParams p) {
     a = block_sum(a, red);
     gamma = 1.f / (1.f + expf(-a));
   }
-  float wk[MOEQ_MAX_K];
+  // weight of slot k: w_k for the routed slots, gamma for the shared one (k == K)
+  float wk[MOEQ_MAX_K + 1];
 #pragma unroll
-  for (int k = 0; k < MOEQ_MAX_K; ++k) wk[k] = k < p.K ? p.w[(size_t)b * p.K + k] : 0.f;
+  for (int k = 0; k <= MOEQ_MAX_K; ++k) wk[k] = k < p.K ? p.w[(size_t)b * p.K + k] : (k == p.K ? gamma : 0.f);
   const float* yb = p.y + (size_t)b * (p.K + 1) * p.H;
-  float ss = 0.f;
-  constexpr int U = 4;  // elements per thread in flight
-  for (int j0 = threadIdx.x; j0 < p.H; j0 += blockDim.x * U) {
-    float acc[U], ys[U][MOEQ_MAX_K + 1];
+  float* rb = p.resid_out + (size_t)b * p.H;
+  float ss = 0.f, keep[kCombineU];
+  const int stride = blockDim.x * kCombineU;
+  for (int j0 = threadIdx.x; j0 < p.H; j0 += stride) {
+    float acc[kCombineU];
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < kCombineU; ++u) {
       const int j = j0 + u * blockDim.x;
-      if (j < p.H) {
-        acc[u] = p.resid_in ? p.resid_in[(size_t)b * p.H + j] : bf16_bits_to_f32(xb[j]);
+      acc[u] = j < p.H ? (p.resid_in ? p.resid_in[(size_t)b * p.H + j] : bf16_bits_to_f32(xb[j])) : 0.f;
+    }
 #pragma unroll
-        for (int k = 0; k <= MOEQ_MAX_K; ++k)
-          if (k <= p.K) ys[u][k] = yb[(size_t)k * p.H + j];
+    for (int k = 0; k <= MOEQ_MAX_K; ++k) {
+      if (k <= p.K) {
+#pragma unroll
+        for (int u = 0; u < kCombineU; ++u) {
+          const int j = j0 + u * blockDim.x;
+          if (j < p.H) acc[u] += wk[k] * yb[(size_t)k * p.H + j];
+        }
       }
     }
 #pragma unroll
-    for (int u = 0; u < U; ++u) {
+    for (int u = 0; u < kCombineU; ++u) {
       const int j = j0 + u * blockDim.x;
+      if (j0 == (int)threadIdx.x) keep[u] = acc[u];
       if (j < p.H) {
-        float a = acc[u];
-#pragma unroll
-        for (int k = 0; k < MOEQ_MAX_K; ++k)
-          if (k < p.K) a += wk[k] * ys[u][k];
-        a += gamma * ys[u][p.K];
-        p.resid_out[(size_t)b * p.H + j] = a;
-        ss += a * a;
+        rb[j] = acc[u];
+        ss += acc[u] * acc[u];
       }
     }
   }
   if (p.xnorm) {
     ss = block_sum(ss, red);
     const float inv = rsqrtf(ss / (float)p.H + p.eps);
-    // each thread re-reads only the elements it wrote itself
-    for (int j = threadIdx.x; j < p.H; j += blockDim.x)
-      p.xnorm[(size_t)b * p.H + j] = f32_to_bf16_bits(p.resid_out[(size_t)b * p.H + j] * inv);
+    uint16_t* xn = p.xnorm + (size_t)b * p.H;
+#pragma unroll
+    for (int u = 0; u < kCombineU; ++u) {
+      const int j = threadIdx.x + u * blockDim.x;
+      if (j < p.H) xn[j] = f32_to_bf16_bits(keep[u] * inv);
+    }
+    for (int j = threadIdx.x + stride; j < p.H; j += blockDim.x) xn[j] = f32_to_bf16_bits(rb[j] * inv);
   }
-  pdl_trigger();
 }
 
 }  // namespace moeq

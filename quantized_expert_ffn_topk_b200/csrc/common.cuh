@@ -65,7 +65,10 @@ __host__ __device__ inline RecGeom rec_geom(int H, int I, int bits, int group) {
 }
 
 // Programmatic dependent launch (PTX griddepcontrol; no-ops when the launch
-// did not ask for it).
+// did not ask for it). A kernel of the per-call chain lets the next one launch
+// as soon as it starts (pdl_trigger first); the next one does only work that
+// reads constant weights before pdl_wait, which returns once this grid has
+// completed and its writes are visible.
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 __device__ __forceinline__ void pdl_trigger() { asm volatile("griddepcontrol.launch_dependents;" ::: "memory"); }
 
@@ -175,6 +178,12 @@ __device__ __forceinline__ void bulk_g2s(void* dst, const void* src, uint32_t by
                    smem_u32(dst)),
                "l"(src), "r"(bytes), "r"(smem_u32(bar))
                : "memory");
+}
+
+// Bulk prefetch of global memory into L2 (no shared memory, no completion).
+// Address 16-byte aligned, size a multiple of 16.
+__device__ __forceinline__ void prefetch_l2(const void* src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.prefetch.L2.global [%0], %1;" ::"l"(src), "r"(bytes) : "memory");
 }
 
 __device__ __forceinline__ unsigned ld_acquire_gpu(const unsigned* p) {

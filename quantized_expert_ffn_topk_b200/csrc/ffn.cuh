@@ -50,11 +50,14 @@ __device__ __forceinline__ const uint8_t* ffn_slot_rec(const FfnParams& p, int k
 
 // Issue the bulk copies of tiles [u0, u0 + nt) of the CTA's share (lane j
 // copies tile u0 + j into buffer j; 0 bytes for an invalid expert). `src`
-// gives a tile's record, offset and size.
-template <typename Src>
-__device__ __forceinline__ void ffn_issue(unsigned char* tiles, int stride, uint64_t* bar, int u0, int nt, Src src) {
+// gives a tile's record, offset and size; `take(u)` selects which tiles this
+// call issues (the shared expert's before pdl_wait, the routed ones after).
+template <typename Src, typename Take>
+__device__ __forceinline__ void ffn_issue(unsigned char* tiles, int stride, uint64_t* bar, int u0, int nt, Src src,
+                                          Take take) {
   const int lane = threadIdx.x & 31;
   for (int j = lane; j < nt; j += 32) {
+    if (!take(u0 + j)) continue;
     const unsigned char* from = nullptr;
     const uint32_t bytes = src(u0 + j, &from);
     mbar_arrive_expect_tx(&bar[j], bytes);
@@ -102,7 +105,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_wait();
+  pdl_trigger();
   auto src = [&](int u, const unsigned char** from) -> uint32_t {
     const int k = u / tps, T = u % tps;
     const uint8_t* rec = ffn_slot_rec(p, k);
@@ -111,10 +114,19 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
     *from = rec + (size_t)T * g.U;
     return g.U;
   };
+  auto is_shared = [&](int u) { return u / tps == p.K; };
+  auto is_routed = [&](int u) { return u / tps != p.K; };
+  auto any = [&](int) { return true; };
+  // the shared expert's tiles do not depend on the previous kernel
+  if (warp == 0 && t_lo < t_hi) ffn_issue(tiles, p.gu_stride, bar, t_lo, min(p.gu_nbuf, t_hi - t_lo), src, is_shared);
+  pdl_wait();
   int round = 0, nt = 0;
   for (int r0 = t_lo; r0 < t_hi; r0 += p.gu_nbuf, ++round) {
     nt = min(p.gu_nbuf, t_hi - r0);
-    if (warp == 0) ffn_issue(tiles, p.gu_stride, bar, r0, nt, src);
+    if (warp == 0) {
+      if (r0 == t_lo) ffn_issue(tiles, p.gu_stride, bar, r0, nt, src, is_routed);
+      else ffn_issue(tiles, p.gu_stride, bar, r0, nt, src, any);
+    }
     if (r0 == t_lo) {  // the input image, while the first round's tiles are in flight
       qstage_vector([&](int j0, float (&v)[16]) { load_bf16_16(p.x + j0, v); }, p.H, p.G, X, tid, blockDim.x);
       __syncthreads();
@@ -153,7 +165,6 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
     if (s_abort) break;
   }
   if (s_abort) ffn_drain(bar, nt, round);
-  pdl_trigger();
 }
 
 // Down: job u = (slot u / (H/16), down tile u % (H/16)); 16 threads per job
@@ -178,7 +189,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_wait();
+  pdl_trigger();
   auto src = [&](int u, const unsigned char** from) -> uint32_t {
     const int k = u / tpd, T = u % tpd;
     const uint8_t* rec = ffn_slot_rec(p, k);
@@ -187,10 +198,19 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
     *from = rec + g.down_off + (size_t)T * g.D;
     return g.D;
   };
+  auto is_shared = [&](int u) { return u / tpd == p.K; };
+  auto is_routed = [&](int u) { return u / tpd != p.K; };
+  auto any = [&](int) { return true; };
+  // the shared expert's tiles do not depend on the previous kernels
+  if (warp == 0 && t_lo < t_hi) ffn_issue(tiles, p.dn_stride, bar, t_lo, min(p.dn_nbuf, t_hi - t_lo), src, is_shared);
+  pdl_wait();
   int round = 0, nt = 0;
   for (int r0 = t_lo; r0 < t_hi; r0 += p.dn_nbuf, ++round) {
     nt = min(p.dn_nbuf, t_hi - r0);
-    if (warp == 0) ffn_issue(tiles, p.dn_stride, bar, r0, nt, src);
+    if (warp == 0) {
+      if (r0 == t_lo) ffn_issue(tiles, p.dn_stride, bar, r0, nt, src, is_routed);
+      else ffn_issue(tiles, p.dn_stride, bar, r0, nt, src, any);
+    }
     if (r0 == t_lo) {  // images of the slots this CTA's jobs touch
       for (int k = t_lo / tpd; k <= (t_hi - 1) / tpd; ++k) {
         const float* hk = p.h + (size_t)k * p.I;
@@ -229,7 +249,6 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
     if (s_abort) break;
   }
   if (s_abort) ffn_drain(bar, nt, round);
-  pdl_trigger();
 }
 
 }  // namespace moeq

@@ -8,7 +8,7 @@ namespace moeq {
 
 constexpr int kRouterWarps = 4;     // warps per CTA, one expert row per warp at a time
 constexpr int kRouterTokTile = 8;   // tokens whose x is staged in shared memory at once
-constexpr int kRouterUnroll = 16;   // 16-byte loads of one row in flight per lane
+constexpr int kRouterUnroll = 8;    // 16-byte loads of one row in flight per lane (the rows were prefetched to L2)
 
 struct RouterParams {
   const uint16_t* x;       // [B, H] bf16
@@ -122,6 +122,10 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(RouterParams 
   const int gwarp = blockIdx.x * kRouterWarps + warp, nwarps = gridDim.x * kRouterWarps;
   const int nvec = p.H / 8;  // 16-byte words per row
 
+  pdl_trigger();
+  // the weight rows do not depend on the previous kernel: pull them into L2
+  if (lane == 0)
+    for (int e = gwarp; e < p.E; e += nwarps) prefetch_l2(p.wr + (size_t)e * p.H, (uint32_t)p.H * 2);
   pdl_wait();
   for (int b0 = 0; b0 < p.B; b0 += kRouterTokTile) {
     const int tb = min(kRouterTokTile, p.B - b0);
@@ -158,8 +162,6 @@ __global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(RouterParams 
       }
     }
   }
-  pdl_trigger();
-
   // The last CTA to arrive selects for every token.
   __syncthreads();
   if (threadIdx.x == 0) {
