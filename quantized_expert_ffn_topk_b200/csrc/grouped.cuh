@@ -71,21 +71,55 @@ __global__ void __launch_bounds__(256) k_group(const int32_t* idx, int B, int K,
     }
   }
   __syncthreads();
-  if (threadIdx.x == 0) {
-    int o = 0, na = 0;
-    for (int e = 0; e < E; ++e) {
-      const int c = s_cnt[e];
-      g.cnt[e] = c;
-      g.off[e] = o;
-      for (int c0 = 0; c0 < c; c0 += kGrpMaxTok, ++na) {
-        g.act[3 * na] = e;
-        g.act[3 * na + 1] = c0;
-        g.act[3 * na + 2] = min(kGrpMaxTok, c - c0);
-      }
-      o += c;
+  // offsets of each expert's entries and of its chunks: exclusive scans over
+  // the experts, each thread taking a contiguous range of them
+  const int per = (E + blockDim.x - 1) / blockDim.x;
+  const int e0 = min(E, (int)threadIdx.x * per), e1 = min(E, e0 + per);
+  int sc = 0, sk = 0;
+  for (int e = e0; e < e1; ++e) {
+    sc += s_cnt[e];
+    sk += (s_cnt[e] + kGrpMaxTok - 1) / kGrpMaxTok;
+  }
+  __shared__ int s_wc[32], s_wk[32];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5, nw = blockDim.x >> 5;
+  int ic = sc, ik = sk;  // inclusive scans within the warp
+#pragma unroll
+  for (int o = 1; o < 32; o <<= 1) {
+    const int tc = __shfl_up_sync(0xFFFFFFFFu, ic, o), tk = __shfl_up_sync(0xFFFFFFFFu, ik, o);
+    if (lane >= o) {
+      ic += tc;
+      ik += tk;
     }
-    g.off[E] = o;
-    g.nact[0] = na;
+  }
+  if (lane == 31) {
+    s_wc[warp] = ic;
+    s_wk[warp] = ik;
+  }
+  __syncthreads();
+  int oc = ic - sc, ok = ik - sk;
+  for (int w = 0; w < warp; ++w) {
+    oc += s_wc[w];
+    ok += s_wk[w];
+  }
+  for (int e = e0; e < e1; ++e) {
+    const int c = s_cnt[e];
+    g.cnt[e] = c;
+    g.off[e] = oc;
+    for (int c0 = 0; c0 < c; c0 += kGrpMaxTok, ++ok) {
+      g.act[3 * ok] = e;
+      g.act[3 * ok + 1] = c0;
+      g.act[3 * ok + 2] = min(kGrpMaxTok, c - c0);
+    }
+    oc += c;
+  }
+  if (threadIdx.x == 0) {
+    int tc = 0, tk = 0;
+    for (int w = 0; w < nw; ++w) {
+      tc += s_wc[w];
+      tk += s_wk[w];
+    }
+    g.off[E] = tc;
+    g.nact[0] = tk;
   }
   __syncthreads();
   for (int i = threadIdx.x; i < n; i += blockDim.x) {

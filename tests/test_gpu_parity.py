@@ -244,6 +244,32 @@ def test_expert_ffn(name):
             assert hz.max_rel_err(yg[b, k], yr) <= FFN_TOL, (b, k, e, hz.max_rel_err(yg[b, k], yr))
 
 
+@pytest.mark.parametrize("bits_routed", [4, 2])
+def test_expert_ffn_one_token_in_rounds(bits_routed):
+    """One token through moe_expert_ffn_q at H=4096, I=8192, K=2: a CTA's share
+    is about 21 gate/up tiles (36,864 B each, five fit shared memory) and 6
+    down tiles (73,728 B each, two fit), so both kernels work in rounds."""
+    w = synth.WORKLOADS["layer4"].with_(name="rounds", I=8192, E=8, K=2, bits_routed=bits_routed)
+    L = hz.build_layer(w, 0)
+    x = hz.x_device(w, 21, 1)
+    idx_np = np.array([[5, 2]], dtype=np.int32)
+    idx = torch.from_numpy(idx_np).cuda()
+    ws = moeq.Workspace(1, w.K, w.H, w.I, w.E)
+    y = torch.empty((1, w.K + 1, w.H), dtype=torch.float32, device="cuda")
+    moeq.moe_expert_ffn_q(L.struct, x, 1, idx, y, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    experts = hz.oracle_experts(w, 0)
+    xd = hz.bf16_to_f64(synth.x_host(w, 21, 1)[0])
+    yg = y.cpu().numpy()
+    for k, e in enumerate(list(idx_np[0]) + [w.E]):
+        g, u, d = experts(int(e))
+        yr = ref.expert_ffn(w.H, w.I, w.group, g, u, d, xd)
+        assert hz.max_rel_err(yg[0, k], yr) <= FFN_TOL, (k, e, hz.max_rel_err(yg[0, k], yr))
+    del L
+    torch.cuda.empty_cache()
+
+
 def test_expert_ffn_bad_index_zeroes_slot():
     w, L = get_layer("tiny")
     x = hz.x_device(w, 1, 1)
@@ -348,10 +374,10 @@ def test_batched_zipf_routing_layer():
 @pytest.mark.parametrize("over", [dict(H=320, I=96, E=5, K=1, group=32), dict(H=512, I=192, E=9, K=8, group=64),
                                   dict(H=512, I=128, E=6, K=3, group=128, bits_routed=2),
                                   dict(H=256, I=64, E=4, K=4, group=32, bits_routed=2, bits_shared=2)])
-def test_ragged_and_edge_shapes(over):
+@pytest.mark.parametrize("B", [1, 3])
+def test_ragged_and_edge_shapes(over, B):
     w = synth.WORKLOADS["tiny"].with_(**over)
     L = hz.build_layer(w, 2)
-    B = 3
     x = hz.x_device(w, 77, B)
     out = run_layer(w, L, x, eps=1e-6)
     xb = synth.x_host(w, 77, B)
