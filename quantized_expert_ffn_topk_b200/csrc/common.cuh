@@ -12,10 +12,10 @@ namespace moeq {
 // Workspace control block: the first 256 bytes of every workspace.
 struct WsCtrl {
   int error;                // first device-side moe_status (0 = none)
-  unsigned router_ticket;   // last-CTA ticket of the router kernel (back to 0 after each call)
+  unsigned router_ticket[8];  // last-CTA tickets of the router kernel, one per 8-token tile (0 between calls)
   unsigned exit_count;      // CTAs that left the fused decode kernel (0 between calls)
   unsigned sync[4];         // arrival counters of the fused decode kernel (0 between calls)
-  unsigned pad[57];
+  unsigned pad[50];
 };
 static_assert(sizeof(WsCtrl) == 256, "control block is 256 bytes");
 

@@ -287,8 +287,11 @@ moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B,
   p.E = E;
   p.K = K;
   p.renorm = renorm;
+  static_assert(MOEQ_MAX_B / kRouterTokTile <= (int)(sizeof(WsCtrl::router_ticket) / sizeof(unsigned)),
+                "one router ticket per token tile");
   const int ctas = (E + kRouterWarps - 1) / kRouterWarps;
-  return launch_pdl(k_router_topk, dim3(ctas), dim3(kRouterWarps * 32), smem, (cudaStream_t)stream, p);
+  const dim3 grid(ctas, (B + kRouterTokTile - 1) / kRouterTokTile);
+  return launch_pdl(k_router_topk, grid, dim3(kRouterWarps * 32), smem, (cudaStream_t)stream, p);
 }
 
 moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx, float* y_out,

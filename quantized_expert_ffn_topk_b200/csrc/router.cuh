@@ -7,7 +7,7 @@
 namespace moeq {
 
 constexpr int kRouterWarps = 4;     // warps per CTA, one expert row per warp at a time
-constexpr int kRouterTokTile = 8;   // tokens whose x is staged in shared memory at once
+constexpr int kRouterTokTile = 8;   // tokens of one CTA (its x staged in shared memory)
 constexpr int kRouterUnroll = 8;    // 16-byte loads of one row in flight per lane (the rows were prefetched to L2)
 
 struct RouterParams {
@@ -114,78 +114,74 @@ __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const 
   }
 }
 
-__global__ void __launch_bounds__(kRouterWarps * 32) k_router_topk(RouterParams p) {
+// grid (E/kRouterWarps, ceil(B/kRouterTokTile)): CTA (c, j) dots rows of
+// warps c*kRouterWarps.. with tokens 8j..8j+7; the last CTA of column j to
+// finish selects for those tokens.
+__global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [tok_tile, H]
   __shared__ int s_last;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gwarp = blockIdx.x * kRouterWarps + warp, nwarps = gridDim.x * kRouterWarps;
   const int nvec = p.H / 8;  // 16-byte words per row
+  const int b0 = blockIdx.y * kRouterTokTile, tb = min(kRouterTokTile, p.B - b0);
 
   pdl_trigger();
   // the weight rows do not depend on the previous kernel: pull them into L2
-  if (lane == 0)
+  if (lane == 0 && blockIdx.y == 0)
     for (int e = gwarp; e < p.E; e += nwarps) prefetch_l2(p.wr + (size_t)e * p.H, (uint32_t)p.H * 2);
   pdl_wait();
-  for (int b0 = 0; b0 < p.B; b0 += kRouterTokTile) {
-    const int tb = min(kRouterTokTile, p.B - b0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < tb * nvec; i += blockDim.x)
-      reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x + (size_t)b0 * p.H)[i];
-    __syncthreads();
-    for (int e = gwarp; e < p.E; e += nwarps) {
-      const uint16_t* row = p.wr + (size_t)e * p.H;
-      float acc[kRouterTokTile];
+  for (int i = threadIdx.x; i < tb * nvec; i += blockDim.x)
+    reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x + (size_t)b0 * p.H)[i];
+  __syncthreads();
+  for (int e = gwarp; e < p.E; e += nwarps) {
+    const uint16_t* row = p.wr + (size_t)e * p.H;
+    float acc[kRouterTokTile];
 #pragma unroll
-      for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
-      for (int v0 = lane; v0 < nvec; v0 += 32 * kRouterUnroll) {
-        uint4 wv[kRouterUnroll];
+    for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
+    for (int v0 = lane; v0 < nvec; v0 += 32 * kRouterUnroll) {
+      uint4 wv[kRouterUnroll];
 #pragma unroll
-        for (int u = 0; u < kRouterUnroll; ++u)
-          if (v0 + 32 * u < nvec) wv[u] = ld_stream16(row + (size_t)(v0 + 32 * u) * 8);
+      for (int u = 0; u < kRouterUnroll; ++u)
+        if (v0 + 32 * u < nvec) wv[u] = ld_stream16(row + (size_t)(v0 + 32 * u) * 8);
 #pragma unroll
-        for (int u = 0; u < kRouterUnroll; ++u) {
-          const int v = v0 + 32 * u;
-          if (v < nvec) {
+      for (int u = 0; u < kRouterUnroll; ++u) {
+        const int v = v0 + 32 * u;
+        if (v < nvec) {
 #pragma unroll
-            for (int t = 0; t < kRouterTokTile; ++t)
-              if (t < tb) acc[t] = dot8_bf16(wv[u], reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
-          }
-        }
-      }
-#pragma unroll
-      for (int t = 0; t < kRouterTokTile; ++t) {
-        if (t < tb) {
-          float s = warp_sum(acc[t]);
-          if (lane == 0) p.logits[(size_t)(b0 + t) * p.E + e] = s;
+          for (int t = 0; t < kRouterTokTile; ++t)
+            if (t < tb) acc[t] = dot8_bf16(wv[u], reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
         }
       }
     }
+#pragma unroll
+    for (int t = 0; t < kRouterTokTile; ++t) {
+      if (t < tb) {
+        float sum = warp_sum(acc[t]);
+        if (lane == 0) p.logits[(size_t)(b0 + t) * p.E + e] = sum;
+      }
+    }
   }
-  // The last CTA to arrive selects for every token.
+  // The last CTA of this token tile to arrive selects for its tokens.
   __syncthreads();
   if (threadIdx.x == 0) {
     __threadfence();
-    unsigned t = atomicAdd(&p.ctrl->router_ticket, 1u);
+    unsigned t = atomicAdd(&p.ctrl->router_ticket[blockIdx.y], 1u);
     s_last = (t == gridDim.x - 1);
   }
   __syncthreads();
   if (!s_last) return;
   __threadfence();
-  float* lsm = reinterpret_cast<float*>(smem_raw);  // logits of up to kRouterTokTile tokens
-  for (int b0 = 0; b0 < p.B; b0 += kRouterTokTile) {
-    const int tb = min(kRouterTokTile, p.B - b0);
-    __syncthreads();
-    for (int i = threadIdx.x; i < tb * p.E; i += blockDim.x) lsm[i] = __ldcg(p.logits + (size_t)b0 * p.E + i);
-    __syncthreads();
-    for (int t = warp; t < tb; t += kRouterWarps) {
-      const int b = b0 + t;
-      topk_one_token(lsm + (size_t)t * p.E, p.E, p.K, p.renorm, p.forced ? p.forced + (size_t)b * p.K : nullptr,
-                     p.idx + (size_t)b * p.K, p.w + (size_t)b * p.K, p.ctrl);
-    }
+  float* lsm = reinterpret_cast<float*>(smem_raw);  // this tile's logits
+  for (int i = threadIdx.x; i < tb * p.E; i += blockDim.x) lsm[i] = __ldcg(p.logits + (size_t)b0 * p.E + i);
+  __syncthreads();
+  for (int t = warp; t < tb; t += kRouterWarps) {
+    const int b = b0 + t;
+    topk_one_token(lsm + (size_t)t * p.E, p.E, p.K, p.renorm, p.forced ? p.forced + (size_t)b * p.K : nullptr,
+                   p.idx + (size_t)b * p.K, p.w + (size_t)b * p.K, p.ctrl);
   }
   __syncthreads();
-  if (threadIdx.x == 0) p.ctrl->router_ticket = 0u;
+  if (threadIdx.x == 0) p.ctrl->router_ticket[blockIdx.y] = 0u;
 }
 
 }  // namespace moeq
