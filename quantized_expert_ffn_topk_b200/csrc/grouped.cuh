@@ -24,6 +24,7 @@
 namespace moeq {
 
 constexpr int kGrpWarps = 8;
+constexpr int kGrpCtasPerSm = 4;                   // resident CTAs per SM (64 registers a thread)
 constexpr int kGrpUnits = kGrpWarps / kFfnPieces;  // units per round (four warps each)
 constexpr int kGrpMaxTok = MOEQ_MAX_B;              // tokens of one expert at most
 
@@ -160,7 +161,7 @@ __device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int n
                                                 const unsigned char* const (&imgs)[4], int gs_off, float& acc0,
                                                 float& acc1) {
   using F = TileFmt<BITS, KS>;
-  constexpr int P = 4;
+  constexpr int P = 2;  // blocks in flight per warp (four CTAs per SM keep the bytes in flight)
   const int lane = threadIdx.x & 31, gid = lane >> 2, t = lane & 3;
   // B fragments of column gid: token gid/2, plane hi (gid even) or lo
   const uint2* planes = reinterpret_cast<const uint2*>(imgs[gid >> 1]) + (gid & 1) * 4 + t;
@@ -235,7 +236,7 @@ __device__ __forceinline__ void unit_token(const GrpParams& p, int a, int i, int
 // DOWN == false: gate/up tiles against x images, h per (token, slot).
 // DOWN == true: down tiles against h images, y per (token, slot).
 template <bool DOWN>
-__global__ void __launch_bounds__(kGrpWarps * 32, 2) k_ffn_grp(GrpParams p) {
+__global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpParams p) {
   __shared__ float part[kGrpUnits][kFfnPieces][kGrpMaxTok][kTileRows];
   __shared__ int s_tok[kGrpUnits][kGrpMaxTok][2];
   const FfnParams& f = p.f;

@@ -333,7 +333,7 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
                  reinterpret_cast<int*>((char*)ws + wl.list), reinterpret_cast<int*>((char*)ws + wl.act),
                  reinterpret_cast<int*>((char*)ws + wl.nact)};
     const int max_act = std::min(p.E, B * p.K) + kGrpExtraChunks;  // work items at most
-    const int ctas = 2 * num_sms();
+    const int ctas = kGrpCtasPerSm * num_sms();
     st = launch_pdl(k_group, dim3(1), dim3(256), (size_t)(p.E + 1) * 4, s, idx, B, p.K, p.E, p.H, gp.g, y_out,
                     p.ctrl);
     if (st != MOE_OK) return st;
