@@ -6,7 +6,7 @@
 
 namespace moeq {
 
-constexpr int kRouterWarps = 4;     // warps per CTA, one expert row per warp at a time
+constexpr int kRouterWarps = 8;     // warps per CTA, one expert row per warp at a time
 constexpr int kRouterTokTile = 8;   // tokens of one CTA (its x staged in shared memory)
 constexpr int kRouterUnroll = 8;    // 16-byte loads of one row in flight per lane (the rows were prefetched to L2)
 
