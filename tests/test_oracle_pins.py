@@ -337,3 +337,96 @@ def test_rmsnorm_closed_forms(ref):
     assert [int(v) for v in xb] == [int(ref.f64_to_bf16(v)[0]) for v in (3 / math.sqrt(12.5), -4 / math.sqrt(12.5),
                                                                           0.0, 5 / math.sqrt(12.5))]
     assert int(xb[2]) == 0 and int(xb[1]) & 0x8000
+
+
+# ---- the whole-layer glue (oracle/layer.py::layer_token) ---------------------
+
+def _rne_bf16_bits(v: float) -> int:
+    """bf16 bits nearest to v, ties to even, written from the format's
+    definition (8 significant bits) with Python integers, not the oracle."""
+    if v == 0.0:
+        return 0x8000 if math.copysign(1.0, v) < 0 else 0
+    m, e = math.frexp(abs(v))          # |v| = m * 2^e, 0.5 <= m < 1
+    q = round(m * 256)                  # round() on a float is ties-to-even
+    if q == 256:
+        q, e = 128, e + 1
+    f32 = np.float32(math.ldexp(q, e - 8)).view(np.uint32)
+    return int((f32 >> 16) | (0x8000 if v < 0 else 0))
+
+
+def _closed_form_layer(gate_w_on: bool, resid, forced, renorm, eps):
+    """A layer whose every expert has constant codes per matrix and whose
+    router rows are scaled one-hot vectors: logits, picks, expert outputs,
+    combine and RMSNorm follow by hand (Python floats)."""
+    H, I, G, E, K = 128, 64, 32, 6, 2
+    s, b = 0.0078125, 0.015625
+    xv = [1.0] * E + [((j * 7) % 11 - 5) / 8.0 for j in range(E, H)]
+    x_bits = np.array([_bf16(v) for v in xv], np.uint16)
+    alpha = [0.5, 2.0, -1.0, 1.5, 0.25, 3.0]          # logit of expert e = alpha_e * x_e = alpha_e
+    router = np.zeros((E, H), np.uint16)
+    for e in range(E):
+        router[e, e] = _bf16(alpha[e])
+    consts = {e: (1 + e, 14 - 2 * e, 3 + e) for e in range(E)}  # (gate, up, down) code per expert
+    consts[E] = (9, 5, 12)                                      # the shared expert
+
+    def mat(rows, cols, c, bb):
+        return (np.full((rows, cols), c, np.uint8), np.full((rows, cols // G), _bf16(s), np.uint16),
+                np.full((rows, cols // G), _bf16(bb), np.uint16))
+
+    def weights(e):
+        cg, cu, cd = consts[e]
+        return mat(I, H, cg, b), mat(I, H, cu, -b), mat(H, I, cd, b)
+
+    def y_const(e):
+        cg, cu, cd = consts[e]
+        sx = math.fsum(xv)
+        g, u = (cg * s + b) * sx, (cu * s - b) * sx
+        return (cd * s + b) * I * (g / (1.0 + math.exp(-g))) * u
+
+    wsg = None
+    gamma = 1.0
+    if gate_w_on:
+        wsg = np.zeros(H, np.uint16)
+        wsg[0] = _bf16(0.5)
+        gamma = 1.0 / (1.0 + math.exp(-0.5 * xv[0]))
+    z = math.fsum(math.exp(a) for a in alpha)
+    p = [math.exp(a) / z for a in alpha]
+    idx = list(forced) if forced is not None else sorted(range(E), key=lambda e: (-alpha[e], e))[:K]
+    w = [p[e] for e in idx]
+    if renorm:
+        t = sum(w)
+        w = [v / t for v in w]
+    r = list(xv) if resid is None else list(resid)
+    out = [r[i] + sum(w[k] * y_const(idx[k]) for k in range(K)) + gamma * y_const(E) for i in range(H)]
+    inv = 1.0 / math.sqrt(math.fsum(v * v for v in out) / H + eps)
+    xn = [_rne_bf16_bits(v * inv) for v in out]
+    ys = [y_const(e) for e in idx] + [y_const(E)]
+    args = (H, I, E, K, G, x_bits, router, weights, weights(E))
+    expect = dict(logits=alpha, idx=idx, w=w, y=ys, gamma=gamma, out=out, xn=xn)
+    return args, wsg, expect
+
+
+@pytest.mark.parametrize("gate_w_on,with_resid,forced,renorm,eps", [(False, False, None, False, 1e-6),
+                                                                    (True, True, None, True, 0.25),
+                                                                    (False, True, [2, 4], False, 1e-6),
+                                                                    (True, False, [0, 5], True, 0.5)])
+def test_layer_token_closed_form(ref, gate_w_on, with_resid, forced, renorm, eps):
+    """oracle/layer.py::layer_token against a layer computed by hand: the
+    residual default (r = widened x), the slot order (routed picks in rank
+    order, the shared expert in row K), the shared-expert gate, forced picks,
+    renormalisation and the RMSNorm hand-off to bf16 (an eps of the order of
+    the mean square makes eps itself visible in the bf16 result)."""
+    from oracle import layer as ref_layer
+    resid = [0.25 * ((i % 9) - 4) for i in range(128)] if with_resid else None
+    args, wsg, ex = _closed_form_layer(gate_w_on, resid, forced, renorm, eps)
+    got = ref_layer.layer_token(*args, renorm=renorm, forced=forced,
+                                resid=None if resid is None else np.array(resid), shared_gate_w=wsg, eps=eps)
+    assert np.allclose(got["logits"], ex["logits"], rtol=0, atol=0)
+    assert [int(v) for v in got["idx"]] == ex["idx"]
+    assert np.allclose(got["w"], ex["w"], rtol=1e-13, atol=0)
+    assert abs(got["gamma"] - ex["gamma"]) < 1e-15
+    H = len(ex["out"])
+    for k, v in enumerate(ex["y"]):
+        assert np.allclose(got["y"][k], np.full(H, v), rtol=1e-12, atol=0), k
+    assert np.allclose(got["out"], ex["out"], rtol=1e-12, atol=1e-15)
+    assert [int(v) for v in got["xn"]] == ex["xn"]
