@@ -299,3 +299,17 @@ void moe_ref_rmsnorm_bf16(const double* v, int H, double eps, uint16_t* out) {
   for (int i = 0; i < H; ++i) out[i] = moe_ref_f64_to_bf16(t[i]);
   free(t);
 }
+
+/* The RMS norm as a kernel of its own (Flash-MoE page, "Metal Compute
+ * Shaders"), with a per-element bf16 weight: out[i] = bf16(v[i] * inv * w[i]),
+ * inv = 1 / sqrt(mean(v^2) + eps), in fp64, rounded once to nearest-even
+ * bf16. w == NULL means unit weight. */
+void moe_ref_rmsnorm_weighted_bf16(const double* v, const uint16_t* w, int H, double eps, uint16_t* out) {
+  double ss = 0.0;
+  for (int i = 0; i < H; ++i) ss += v[i] * v[i];
+  double inv = 1.0 / sqrt(ss / H + eps);
+  for (int i = 0; i < H; ++i) {
+    double wi = w ? moe_ref_bf16_to_f64(w[i]) : 1.0;
+    out[i] = moe_ref_f64_to_bf16(v[i] * inv * wi);
+  }
+}

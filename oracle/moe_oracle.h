@@ -98,6 +98,8 @@ void moe_ref_combine(int H, int K, const double* y, const double* w, double gamm
 
 void moe_ref_rmsnorm(const double* v, int H, double eps, double* out);
 void moe_ref_rmsnorm_bf16(const double* v, int H, double eps, uint16_t* out);
+/* out[i] = bf16(v[i] / sqrt(mean(v^2) + eps) * w[i]); w == NULL: unit weight */
+void moe_ref_rmsnorm_weighted_bf16(const double* v, const uint16_t* w, int H, double eps, uint16_t* out);
 
 #ifdef __cplusplus
 }

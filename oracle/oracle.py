@@ -82,6 +82,8 @@ def lib():
         L.moe_ref_rmsnorm.argtypes = [_f64p, ctypes.c_int, ctypes.c_double, _f64p]
         L.moe_ref_rmsnorm_bf16.restype = None
         L.moe_ref_rmsnorm_bf16.argtypes = [_f64p, ctypes.c_int, ctypes.c_double, _u16p]
+        L.moe_ref_rmsnorm_weighted_bf16.restype = None
+        L.moe_ref_rmsnorm_weighted_bf16.argtypes = [_f64p, _u16p, ctypes.c_int, ctypes.c_double, _u16p]
         _lib = L
     return _lib
 
@@ -263,4 +265,17 @@ def rmsnorm_bf16(v, eps: float):
     v = _c(v, np.float64)
     out = np.zeros(v.shape[0], dtype=np.uint16)
     lib().moe_ref_rmsnorm_bf16(_p(v, _f64p), v.shape[0], float(eps), _p(out, _u16p))
+    return out
+
+
+def rmsnorm_weighted_bf16(v, w_bf16, eps: float):
+    """bf16 bits of v / rms(v) * w (w: bf16 bits [H], or None for unit weight)."""
+    v = _c(v, np.float64)
+    out = np.zeros(v.shape[0], dtype=np.uint16)
+    wp = None
+    if w_bf16 is not None:
+        w = _c(w_bf16, np.uint16)
+        assert w.shape == v.shape
+        wp = _p(w, _u16p)
+    lib().moe_ref_rmsnorm_weighted_bf16(_p(v, _f64p), wp, v.shape[0], float(eps), _p(out, _u16p))
     return out

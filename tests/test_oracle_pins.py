@@ -339,6 +339,27 @@ def test_rmsnorm_closed_forms(ref):
     assert int(xb[2]) == 0 and int(xb[1]) & 0x8000
 
 
+def test_rmsnorm_weighted_closed_forms(ref):
+    """The standalone RMS norm with a weight vector: unit weight (None, or all
+    ones) is the unweighted norm; [3, 4] with weights [0.5, 2] and a power of
+    two weight follow by hand."""
+    rng = np.random.default_rng(6)
+    v = rng.normal(size=96)
+    unit = ref.rmsnorm_bf16(v, 1e-6)
+    assert (ref.rmsnorm_weighted_bf16(v, None, 1e-6) == unit).all()
+    assert (ref.rmsnorm_weighted_bf16(v, np.full(96, _bf16(1.0), np.uint16), 1e-6) == unit).all()
+    # a power-of-two weight scales exactly: the bf16 pattern moves by its exponent
+    got = ref.rmsnorm_weighted_bf16(v, np.full(96, _bf16(4.0), np.uint16), 1e-6)
+    assert (got.astype(np.int32) - unit.astype(np.int32) == np.where(unit & 0x7FFF, 2 << 7, 0)).all()
+    w = np.array([_bf16(0.5), _bf16(2.0)], np.uint16)
+    got = ref.rmsnorm_weighted_bf16(np.array([3.0, 4.0]), w, 0.0)
+    rms = math.sqrt(12.5)
+    assert [int(b) for b in got] == [_rne_bf16_bits(3.0 / rms * 0.5), _rne_bf16_bits(4.0 / rms * 2.0)]
+    # a weight of -1 flips only the sign bit
+    neg = ref.rmsnorm_weighted_bf16(v, np.full(96, _bf16(-1.0), np.uint16), 1e-6)
+    assert (neg == (unit ^ 0x8000)).all()
+
+
 # ---- the whole-layer glue (oracle/layer.py::layer_token) ---------------------
 
 def _rne_bf16_bits(v: float) -> int:
