@@ -1,13 +1,15 @@
 #!/usr/bin/env python3
 """Benchmark of the decode-time quantized MoE FFN step on B200.
 
-Default workload ("layer4"): one batch-1 MoE layer per step (H=4096, E=512
-routed experts, I=1024, top-4 + 1 shared expert, 4-bit group-64 affine codes
-with bf16 scale/bias, bf16 router), i.e. router GEMV + softmax/top-K +
+Default workload ("layer4"): batch-1 MoE layers (H=4096, E=512 routed
+experts, I=1024, top-4 + 1 shared expert, 4-bit group-64 affine codes with
+bf16 scale/bias, bf16 router), i.e. per layer router GEMV + softmax/top-K +
 gate/up/down dequant mat-vecs + SwiGLU + combine with shared expert and
-residual + RMSNorm. A step is one layer-token; steps chain like decode
-(x_{t+1} = RMSNorm(r_{t+1}) of step t) and walk `--layers` distinct resident
-layers so that no weight byte is reused from L2 (126 MB) between visits.
+residual + RMSNorm. A step is one decode token through `--layers` distinct
+resident layers (one launch of the fused kernel); the metric counts
+layer-tokens (one token through one MoE layer). Steps chain like decode
+(x_{t+1} = RMSNorm(r_{t+1}) of step t), and every launch walks the whole
+resident stack, so no weight byte is reused from L2 (126 MB) between visits.
 
 Prints one JSON line (rank 0). `--impl reference` times the fp64 C oracle on
 the host cores instead, on a bounded sample of the same workload.
@@ -32,14 +34,18 @@ FALLBACK_HBM_GBS = 6650.0
 def parse():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
-    ap.add_argument("--steps", type=int, default=20000)
-    ap.add_argument("--warmup", type=int, default=200)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=20)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--workload", default="layer4", choices=["layer4", "layer2"])
     ap.add_argument("--layers", type=int, default=24, help="resident layers walked by the steps")
     ap.add_argument("--cpu-sample", type=int, default=12, help="tokens in the oracle CPU-baseline sample")
     ap.add_argument("--no-e2e", action="store_true")
     ap.add_argument("--no-extra", action="store_true", help="skip the C0/C2/C3/C4 report lines")
+    ap.add_argument("--stat-replays", type=int, default=200, help="individually timed launches for the distribution")
+    ap.add_argument("--profile-case", choices=["decode", "per_call", "batch"], default=None,
+                    help="run one path on --layers resident layers for --steps steps and print no JSON "
+                         "(a small case for ncu captures)")
     return ap.parse_args()
 
 
@@ -137,19 +143,37 @@ def oracle_tokens_per_s(w, n_tokens: int, layers: int = 2, seed_token: int = 1_0
     return n_tokens / total, total
 
 
+def workload_config(w, nlayers: int, world: int = 1) -> dict:
+    """The `config` object of both arms' JSON lines."""
+    import quantized_expert_ffn_topk_b200 as moeq
+    rec_r = moeq.moe_expert_bytes(w.H, w.I, w.bits_routed, w.group)
+    rec_s = moeq.moe_expert_bytes(w.H, w.I, w.bits_shared, w.group)
+    resident = nlayers * (w.E * rec_r + rec_s + w.E * w.H * 2)
+    return {"workload": "%s: batch-1 MoE layer H%d E%d I%d top-%d + shared, %d-bit routed / %d-bit shared, group %d"
+                        % (w.name, w.H, w.E, w.I, w.K, w.bits_routed, w.bits_shared, w.group),
+            "batch": 1, "layers_resident": nlayers, "resident_bytes": resident,
+            "step": "one decode token through the %d resident layers (%d layer-tokens)" % (nlayers, nlayers),
+            "l2": "inputs larger than L2: each step walks %d resident layers (%.1f GB)" % (nlayers, resident / 1e9),
+            "parallelism": "replicas" if world > 1 else "single GPU"}
+
+
 def run_reference(args, w, rank: int):
+    """The reference arm: the fp64 C oracle on the host cores (rank 0 only),
+    each step one layer-token of the same workload (a bounded sample of a
+    decode token through the stack), reported in the same unit."""
     if rank != 0:
         return
-    tps, secs = oracle_tokens_per_s(w, args.warmup + args.steps)
-    line = {"impl": "reference", "metric": "MoE-layer decode tokens/s", "value": tps, "unit": "tokens/s",
+    n = args.warmup + args.steps
+    tps, secs = oracle_tokens_per_s(w, n)
+    line = {"impl": "reference", "metric": "MoE-layer decode tokens/s", "value": tps, "unit": "layer-tokens/s",
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / tps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
-            "config": {"workload": w.name, "H": w.H, "E": w.E, "I": w.I, "K": w.K, "group": w.group,
-                       "bits_routed": w.bits_routed, "bits_shared": w.bits_shared, "batch": 1},
-            "cpu_baseline": {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
-                             "sample": "%d layer-token steps through the single-threaded fp64 C oracle "
-                                       "(router, top-K, 5 expert FFNs, combine, RMSNorm)" % (args.warmup + args.steps)},
-            "e2e": {"value": tps, "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+            "config": workload_config(w, args.layers, args.gpus),
+            "cpu_baseline": {"value": tps, "unit": "layer-tokens/s", "cores": 1, "kind": "oracle",
+                             "sample": "%d layer-token steps (router, top-K, 5 expert FFNs, combine, RMSNorm) of %s "
+                                       "through the single-threaded fp64 C oracle, %.1f s of oracle work"
+                                       % (n, w.name, secs)},
+            "e2e": {"value": tps, "unit": "layer-tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     print(json.dumps(line), flush=True)
 
 
@@ -167,10 +191,46 @@ def build_layers(w, nlayers, dev, s):
     return layers
 
 
-def per_call_path(w, layers, ws, dev, stream, steps):
+def dist_of(ms_list):
+    """median / p10 / p90 of per-replay times (ms)."""
+    import numpy as np
+    a = np.asarray(ms_list, dtype=np.float64)
+    return {"median_ms": float(np.median(a)), "p10_ms": float(np.percentile(a, 10)),
+            "p90_ms": float(np.percentile(a, 90)), "replays": int(a.size)}
+
+
+def replay_times(stream, graphs, n: int, nvtx: str = None):
+    """Replay the graphs in turn n times, each replay bracketed by its own
+    events on `stream`; returns the per-replay times (ms). `nvtx` names the
+    range (for profiler filters)."""
+    import torch
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(n)]
+    torch.cuda.synchronize()
+    if nvtx:
+        torch.cuda.nvtx.range_push(nvtx)
+    for i in range(n):
+        ev[i][0].record(stream)
+        graphs[i % len(graphs)].replay()
+        ev[i][1].record(stream)
+    torch.cuda.synchronize()
+    if nvtx:
+        torch.cuda.nvtx.range_pop()
+    return [a.elapsed_time(b) for (a, b) in ev]
+
+
+def capture(stream, fn):
+    import torch
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g, stream=stream):
+        fn()
+    return g
+
+
+def per_call_path(w, layers, ws, dev, stream, replays):
     """The four per-token calls (router+top-K, expert FFN, combine) chained
-    like decode, each step one CUDA graph of 4 kernels with PDL; also times
-    the expert-FFN call alone with events around it."""
+    like decode, one CUDA graph per layer (PDL between the kernels); each
+    replay is timed on its own. Also the expert-FFN call alone (events around
+    it, eager launches)."""
     import torch
 
     import quantized_expert_ffn_topk_b200 as moeq
@@ -192,27 +252,13 @@ def per_call_path(w, layers, ws, dev, stream, steps):
     for l in range(nl):
         step(l)
     torch.cuda.synchronize()
-    graphs = []
-    for l in range(nl):
-        g = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g, stream=stream):
-            step(l)
-        graphs.append(g)
+    graphs = [capture(stream, lambda l=l: step(l)) for l in range(nl)]
     for t in range(2 * nl):
         graphs[t % nl].replay()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    torch.cuda.synchronize()
-    torch.cuda.nvtx.range_push("per_call")
-    a.record(stream)
-    for t in range(steps):
-        graphs[t % nl].replay()
-    b.record(stream)
-    torch.cuda.synchronize()
-    torch.cuda.nvtx.range_pop()
-    ms = a.elapsed_time(b)
+    times = replay_times(stream, graphs, max(replays, nl), nvtx="per_call")
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(nl)]
     ffn_ms = []
-    for t in range(max(nl, min(steps, 1600))):
+    for t in range(max(nl, min(replays, 400))):
         l = t % nl
         L, o = layers[l], outs[l]
         xin = xbuf[l % 2]
@@ -229,14 +275,14 @@ def per_call_path(w, layers, ws, dev, stream, steps):
             ffn_ms += [x.elapsed_time(y) for (x, y) in ev]
     torch.cuda.synchronize()
     del graphs
-    return steps / (ms / 1e3), statistics.mean(ffn_ms)
+    return times, ffn_ms
 
 
 def replica_rate(ms: float, steps: int, world: int, device=None):
-    """Whole-job rate of `world` independent replicas, each having run `steps`
-    layer-token steps in `ms` milliseconds of its own device time: the job
-    takes the slowest replica's time (max over ranks), and processes
-    world * steps units in it. Returns (max ms, units per second)."""
+    """Whole-job rate of `world` independent replicas, each having processed
+    `steps` units in `ms` milliseconds of its own device time: the job takes
+    the slowest replica's time (max over ranks), and processes world * steps
+    units in it. Returns (max ms, units per second)."""
     if world > 1:
         import torch
         import torch.distributed as dist
@@ -246,29 +292,10 @@ def replica_rate(ms: float, steps: int, world: int, device=None):
     return ms, world * steps / (ms / 1e3)
 
 
-def timed_graph(stream, fn, reps: int = 2):
-    """Capture fn() (a sequence of launches on `stream`) in a CUDA graph, replay
-    it once to warm up, then time `reps` replays with events. Returns ms per replay."""
-    import torch
-    g = torch.cuda.CUDAGraph()
-    with torch.cuda.graph(g, stream=stream):
-        fn()
-    g.replay()
-    torch.cuda.synchronize()
-    a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-    a.record(stream)
-    for _ in range(reps):
-        g.replay()
-    b.record(stream)
-    torch.cuda.synchronize()
-    ms = a.elapsed_time(b) / reps
-    del g
-    return ms
-
-
-def extra_configs(layers, ws, dev, stream, peak):
-    """The other workloads, each timed on the device with the data resident:
-    C0 (tiny, fused), C2 (2-bit routed experts, fused, own arena), C3 (256
+def extra_configs(layers, dev, stream, peak):
+    """The other workloads, each timed on the device with the data resident,
+    as a distribution over individually timed CUDA-graph replays: C0 (tiny,
+    fused), C2 (2-bit routed experts, fused, own 8-layer arena), C3 (256
     tokens through all resident layer4 layers with forced 27 %-overlap
     routing), C4 (32 tokens per step, forced Zipf routing, grouped per-call
     path). Returns a dict of report lines."""
@@ -281,60 +308,70 @@ def extra_configs(layers, ws, dev, stream, peak):
     out = {}
     eps = 1e-6
 
-    def decode_rate(w, Ls, steps_layers):
+    def decode_stats(w, Ls, launches_per_graph, replays):
+        ws_w = moeq.Workspace(1, w.K, w.H, w.I, w.E, device=dev, stream=s)
         x = torch.empty(w.H, dtype=torch.bfloat16, device=dev)
         synth.x_dev(w, 7, 1, x.data_ptr(), s)
         r = x.float().clone()
-        structs = [L.struct for L in Ls]
-        reps = max(1, steps_layers // len(Ls))
-        ms = timed_graph(stream, lambda: [moeq.moe_decode_layers(structs, x, r, False, None, None, None, r, x, eps,
-                                                                 ws_w.buf, ws_w.nbytes, s) for _ in range(reps)])
-        return reps * len(Ls) / (ms / 1e3)
+        table = moeq.layer_table([L.struct for L in Ls])
+        g = capture(stream, lambda: [moeq.moe_decode_layers(table, x, r, False, None, None, None, r, x, eps,
+                                                            ws_w.buf, ws_w.nbytes, s)
+                                     for _ in range(launches_per_graph)])
+        for _ in range(3):
+            g.replay()
+        d = dist_of(replay_times(stream, [g], replays))
+        units = launches_per_graph * len(Ls)
+        return units / (d["median_ms"] / 1e3), d
 
     # C0: tiny, one layer, fused (parity workload; a latency figure)
     w0 = synth.WORKLOADS["tiny"]
     L0 = build_layers(w0, 1, dev, s)
-    ws_w = moeq.Workspace(1, w0.K, w0.H, w0.I, w0.E, device=dev, stream=s)
-    tps0 = decode_rate(w0, L0, 256)
+    tps0, d0 = decode_stats(w0, L0, 64, 50)
     b0 = algorithmic_bytes(w0)[0]
     out["C0"] = {"workload": "tiny H256 E8 I128 top-2 + shared, 4-bit, group 32", "tokens_per_s": tps0,
-                 "step_bytes": b0, "gbs": b0 * tps0 / 1e9}
+                 "step_bytes": b0, "gbs": b0 * tps0 / 1e9, "timing": d0, "graph": "64 one-layer launches"}
     del L0
 
     # C2: 2-bit routed experts (4-bit shared), own 8-layer arena
     w2 = synth.WORKLOADS["layer2"]
     L2 = build_layers(w2, 8, dev, s)
-    ws_w = moeq.Workspace(1, w2.K, w2.H, w2.I, w2.E, device=dev, stream=s)
-    tps2 = decode_rate(w2, L2, 8 * 64)
+    tps2, d2 = decode_stats(w2, L2, 4, 100)
     b2 = algorithmic_bytes(w2)[0]
     out["C2"] = {"workload": "layer2: as layer4 with 2-bit routed experts (shared 4-bit)", "tokens_per_s": tps2,
-                 "step_bytes": b2, "gbs": b2 * tps2 / 1e9, "frac_of_measured_hbm": b2 * tps2 / 1e9 / peak,
-                 "layers_resident": 8}
+                 "step_bytes": b2, "gbs": b2 * tps2 / 1e9, "frac_of_peak": b2 * tps2 / 1e9 / peak,
+                 "layers_resident": 8, "timing": d2, "graph": "4 launches over the 8 resident layers"}
     del L2
     torch.cuda.empty_cache()
 
     # C3: 256 tokens x all resident layer4 layers, forced routing with 27 % overlap
     w = synth.WORKLOADS["layer4"]
     nl = len(layers)
-    T = 256
+    T, per = 256, 32
     routing = synth.overlap_routing(w.E, w.K, T, nl, 0.27, seed=3)
     rd = torch.from_numpy(np.ascontiguousarray(routing)).to(dev)
     xs = torch.empty((T, w.H), dtype=torch.bfloat16, device=dev)
     synth.x_dev(w, 9000, T, xs.data_ptr(), s)
     r3 = torch.empty(w.H, dtype=torch.float32, device=dev)
-    structs = [L.struct for L in layers]
-    ws_w = ws
-    ms3 = timed_graph(stream, lambda: [moeq.moe_decode_layers(structs, xs[t], None, False, rd[t], None, None, r3, None,
-                                                              eps, ws.buf, ws.nbytes, s) for t in range(T)])
-    tps3 = T / (ms3 / 1e3)
+    table = moeq.layer_table([L.struct for L in layers])
+    ws3 = moeq.Workspace(1, w.K, w.H, w.I, w.E, device=dev, stream=s)
+    graphs3 = [capture(stream, lambda g0=g0: [moeq.moe_decode_layers(table, xs[t], None, False, rd[t], None, None, r3,
+                                                                      None, eps, ws3.buf, ws3.nbytes, s)
+                                              for t in range(g0, g0 + per)])
+               for g0 in range(0, T, per)]
+    graphs3[0].replay()
+    d3 = dist_of(replay_times(stream, graphs3, 3 * len(graphs3)))
+    tps3 = per / (d3["median_ms"] / 1e3)
     b3 = algorithmic_bytes(w)[0] * nl
     out["C3"] = {"workload": "%d layer4 layers resident, %d tokens, forced routing (overlap %.3f measured)" %
                              (nl, T, synth.measured_overlap(routing)),
-                 "tokens_per_s": tps3, "token_bytes": b3, "gbs": b3 * tps3 / 1e9,
-                 "frac_of_measured_hbm": b3 * tps3 / 1e9 / peak}
+                 "tokens_per_s": tps3, "layer_tokens_per_s": tps3 * nl, "token_bytes": b3, "gbs": b3 * tps3 / 1e9,
+                 "frac_of_peak": b3 * tps3 / 1e9 / peak, "timing": d3,
+                 "graph": "%d graphs of %d tokens (one launch per token over %d layers), replayed in turn" %
+                          (len(graphs3), per, nl)}
+    del graphs3
 
     # C4: 32 tokens per step, forced Zipf(1.1) routing, grouped per-call path
-    B, S = 32, 2 * nl
+    B, S = 32, nl
     zr = synth.zipf_routing(w.E, w.K, B, S, 1.1, seed=5)
     zd = torch.from_numpy(np.ascontiguousarray(zr)).to(dev)
     wsb = moeq.Workspace(B, w.K, w.H, w.I, w.E, device=dev, stream=s)
@@ -343,23 +380,26 @@ def extra_configs(layers, ws, dev, stream, peak):
     resid = xb.float().clone()
     outs = [L.alloc_outputs(B, logits=False, xnorm=True) for L in layers]
 
-    def c4():
-        for st in range(S):
-            l = st % nl
-            L, o = layers[l], outs[l]
-            moeq.moe_router_topk(xb, L.router_w, B, w.H, w.E, w.K, False, zd[st], o["idx"], o["w"], None, wsb.buf,
-                                 wsb.nbytes, s)
-            moeq.moe_expert_ffn_q(L.struct, xb, B, o["idx"], o["y"], wsb.buf, wsb.nbytes, s)
-            moeq.moe_combine_residual(L.struct, o["y"], o["w"], xb, resid, B, resid, o["xnorm"], eps, s)
+    def c4_step(st):
+        L, o = layers[st], outs[st]
+        moeq.moe_router_topk(xb, L.router_w, B, w.H, w.E, w.K, False, zd[st], o["idx"], o["w"], None, wsb.buf,
+                             wsb.nbytes, s)
+        moeq.moe_expert_ffn_q(L.struct, xb, B, o["idx"], o["y"], wsb.buf, wsb.nbytes, s)
+        moeq.moe_combine_residual(L.struct, o["y"], o["w"], xb, resid, B, resid, o["xnorm"], eps, s)
 
-    ms4 = timed_graph(stream, c4)
-    tps4 = B * S / (ms4 / 1e3)
+    graphs4 = [capture(stream, lambda st=st: c4_step(st)) for st in range(S)]
+    for g in graphs4:
+        g.replay()
+    d4 = dist_of(replay_times(stream, graphs4, max(200, 4 * S), nvtx="batch"))
+    step_s = d4["median_ms"] / 1e3
     rec = algorithmic_bytes(w)[1]
     distinct = float(np.mean([len(np.unique(zr[st])) for st in range(S)]))
     b4 = w.E * w.H * 2 + (1 + distinct) * rec
     out["C4"] = {"workload": "layer4, 32 tokens per step, forced Zipf(1.1) routing, grouped per expert",
-                 "tokens_per_s": tps4, "distinct_experts_per_step": distinct, "step_bytes": b4,
-                 "gbs": b4 * (S / (ms4 / 1e3)) / 1e9, "frac_of_measured_hbm": b4 * (S / (ms4 / 1e3)) / 1e9 / peak}
+                 "tokens_per_s": B / step_s, "distinct_experts_per_step": distinct, "step_bytes": b4,
+                 "gbs": b4 / step_s / 1e9, "frac_of_peak": b4 / step_s / 1e9 / peak, "timing": d4,
+                 "graph": "one graph per layer (router + grouped expert FFN + combine), layers in turn"}
+    del graphs4
     return out
 
 
@@ -390,6 +430,57 @@ def measured_traffic(w, nlayers):
     return rec["dram_bytes_per_layer"] * nlayers
 
 
+def profile_case(args, w, dev, stream):
+    """A small run of one path for ncu (no JSON): `decode` (the fused kernel),
+    `per_call` (router, expert FFN, combine per token) or `batch` (32 tokens
+    per step, grouped), each over --layers resident layers for --steps steps."""
+    import numpy as np
+    import torch
+
+    import quantized_expert_ffn_topk_b200 as moeq
+    from synth import synth
+    s = stream.cuda_stream
+    with torch.cuda.stream(stream):
+        layers = build_layers(w, args.layers, dev, s)
+        nl = len(layers)
+        if args.profile_case == "decode":
+            ws = moeq.Workspace(1, w.K, w.H, w.I, w.E, device=dev, stream=s)
+            x = torch.empty(w.H, dtype=torch.bfloat16, device=dev)
+            synth.x_dev(w, 1, 1, x.data_ptr(), s)
+            r = x.float().clone()
+            table = moeq.layer_table([L.struct for L in layers])
+            for _ in range(args.warmup + args.steps):
+                moeq.moe_decode_layers(table, x, r, False, None, None, None, r, x, 1e-6, ws.buf, ws.nbytes, s)
+        elif args.profile_case == "per_call":
+            ws = moeq.Workspace(1, w.K, w.H, w.I, w.E, device=dev, stream=s)
+            x = torch.empty((1, w.H), dtype=torch.bfloat16, device=dev)
+            synth.x_dev(w, 1, 1, x.data_ptr(), s)
+            r = x.float().clone()
+            outs = [L.alloc_outputs(1, logits=False, xnorm=True) for L in layers]
+            for t in range(args.warmup + args.steps):
+                l = t % nl
+                layers[l].forward(x, ws, outs[l], resid_in=r, eps=1e-6, stream=s)
+                x.copy_(outs[l]["xnorm"])
+        else:
+            B = 32
+            zr = synth.zipf_routing(w.E, w.K, B, args.warmup + args.steps, 1.1, seed=5)
+            zd = torch.from_numpy(np.ascontiguousarray(zr)).to(dev)
+            ws = moeq.Workspace(B, w.K, w.H, w.I, w.E, device=dev, stream=s)
+            xb = torch.empty((B, w.H), dtype=torch.bfloat16, device=dev)
+            synth.x_dev(w, 12000, B, xb.data_ptr(), s)
+            resid = xb.float().clone()
+            outs = [L.alloc_outputs(B, logits=False, xnorm=True) for L in layers]
+            for t in range(args.warmup + args.steps):
+                l = t % nl
+                layers[l].forward(xb, ws, outs[l], resid_in=resid, forced_idx=zd[t], eps=1e-6, stream=s)
+        torch.cuda.synchronize()
+        err = moeq.moe_get_device_error(ws.buf, s)
+    print("profile case %s: %d layers, %d steps, device status %s" %
+          (args.profile_case, nl, args.warmup + args.steps, moeq.status_str(err)), flush=True)
+    if err != moeq.MOE_OK:
+        raise SystemExit(1)
+
+
 def run_ours(args, w, rank: int, world: int, local_rank: int):
     import torch
     import torch.distributed as dist
@@ -400,8 +491,13 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
     dev = torch.device("cuda", local_rank)
     torch.cuda.set_device(dev)
     stream = torch.cuda.Stream(device=dev)
+    if args.profile_case:
+        profile_case(args, w, dev, stream)
+        return None
     nlayers = args.layers
     eps = 1e-6
+    peak, peak_src = peaks()
+    K, W = args.steps, args.warmup
     with torch.cuda.stream(stream):
         s = stream.cuda_stream
         layers = build_layers(w, nlayers, dev, s)
@@ -409,63 +505,55 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
         x = torch.empty(w.H, dtype=torch.bfloat16, device=dev)
         synth.x_dev(w, 1000 * rank, 1, x.data_ptr(), s)
         resid = x.float().clone()
-        structs = [L.struct for L in layers]
+        table = moeq.layer_table([L.struct for L in layers])
         torch.cuda.synchronize()
 
-        # a step is one layer-token; one launch walks all resident layers
-        # (x <- RMSNorm(r) of the last layer, so passes chain like decode)
-        def launch(n):
-            moeq.moe_decode_layers(structs[:n], x, resid, False, None, None, None, resid, x, eps, ws.buf, ws.nbytes, s)
+        # a step is one decode token through all resident layers: one launch
+        # (x <- RMSNorm(r) of the last layer, so steps chain like decode)
+        def launch():
+            moeq.moe_decode_layers(table, x, resid, False, None, None, None, resid, x, eps, ws.buf, ws.nbytes, s)
 
-        launch(nlayers)
+        launch()
         torch.cuda.synchronize()
         if moeq.moe_get_device_error(ws.buf, s) != moeq.MOE_OK:
             raise RuntimeError("device error in the first launch")
-        full, rem = divmod(args.steps, nlayers)
-        g_full = torch.cuda.CUDAGraph()
-        with torch.cuda.graph(g_full, stream=stream):
-            launch(nlayers)
-        g_rem = None
-        if rem:
-            g_rem = torch.cuda.CUDAGraph()
-            with torch.cuda.graph(g_rem, stream=stream):
-                launch(rem)
+        g = capture(stream, launch)
         synth.x_dev(w, 1000 * rank, 1, x.data_ptr(), s)
         resid.copy_(x.float())
-        for _ in range(max(1, args.warmup // nlayers)):
-            g_full.replay()
+        for _ in range(W):
+            g.replay()
         start, end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
-        if world > 1:
-            dist.barrier()
-        torch.cuda.synchronize()
         with ClockSampler(local_rank) as clk:
+            if world > 1:
+                dist.barrier()
+            torch.cuda.synchronize()
             torch.cuda.nvtx.range_push("decode")
             start.record(stream)
-            for _ in range(full):
-                g_full.replay()
-            if g_rem is not None:
-                g_rem.replay()
+            for _ in range(K):
+                g.replay()
             end.record(stream)
             torch.cuda.synchronize()
             torch.cuda.nvtx.range_pop()
-        if world > 1:
-            dist.barrier()
-        ms = start.elapsed_time(end)
+            if world > 1:
+                dist.barrier()
+            ms = start.elapsed_time(end)
+            # the distribution: launches timed one by one, at least --stat-replays of them
+            dist_ms = replay_times(stream, [g], max(args.stat_replays, 1), nvtx="decode_dist")
         err = moeq.moe_get_device_error(ws.buf, s)
         if err != moeq.MOE_OK:
             raise RuntimeError("device error in timed region: %s" % moeq.status_str(err))
-        ms, tps = replica_rate(ms, args.steps, world, dev)
-        launches = full + (1 if rem else 0)
-        del g_full, g_rem
+        ms, tps = replica_rate(ms, K * nlayers, world, dev)
+        del g
 
         # the per-call path (router_topk, expert_ffn_q, combine_residual)
-        pc_tps, ffn_avg_ms = per_call_path(w, layers, ws, dev, stream, min(args.steps, 4000))
+        pc_times, ffn_ms = per_call_path(w, layers, ws, dev, stream, args.stat_replays)
 
         # end to end through the public call with host buffers: per step one
-        # layer-token, x copied in from pinned memory and r copied back out
+        # token through all resident layers (one call, prebuilt layer table),
+        # x copied in from pinned memory and r copied back out
         e2e = None
         if not args.no_e2e:
-            n_e2e = min(args.steps, 4000)
+            n_e2e = max(K, 100)
             tmp = torch.empty((n_e2e, w.H), dtype=torch.bfloat16, device=dev)
             synth.x_dev(w, 50_000, n_e2e, tmp.data_ptr(), s)
             torch.cuda.synchronize()
@@ -479,48 +567,52 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
             e0.record(stream)
             for t in range(n_e2e):
                 xd.copy_(xh[t], non_blocking=True)
-                moeq.moe_decode_layers(structs[t % nlayers: t % nlayers + 1], xd, None, False, None, None, None, rd,
-                                       None, eps, ws.buf, ws.nbytes, s)
+                moeq.moe_decode_layers(table, xd, None, False, None, None, None, rd, None, eps, ws.buf, ws.nbytes, s)
                 outh[t].copy_(rd, non_blocking=True)
             e1.record(stream)
             torch.cuda.synchronize()
             torch.cuda.nvtx.range_pop()
-            e2e_ms = e0.elapsed_time(e1)
-            e2e = {"value": n_e2e / (e2e_ms / 1e3), "unit": "tokens/s", "h2d_bytes_per_step": w.H * 2,
-                   "d2h_bytes_per_step": w.H * 4, "steps": n_e2e,
-                   "path": "moe_decode_layers (1 layer per call) with pinned host input/output copies"}
+            e2e_ms, e2e_rate = replica_rate(e0.elapsed_time(e1), n_e2e * nlayers, world, dev)
+            e2e = {"value": e2e_rate, "unit": "layer-tokens/s", "tokens_per_s": e2e_rate / nlayers,
+                   "h2d_bytes_per_step": w.H * 2, "d2h_bytes_per_step": w.H * 4, "steps": n_e2e,
+                   "path": "moe_decode_layers over the %d resident layers per call (one token per call), "
+                           "pinned host input and output copies on the stream" % nlayers}
 
         # the other workloads (report lines), on one GPU only
         extra = None
         if not args.no_extra and world == 1 and w.name == "layer4":
-            extra = extra_configs(layers, ws, dev, stream, peaks()[0])
+            extra = extra_configs(layers, dev, stream, peak)
 
     step_bytes, rec_r, rec_s = algorithmic_bytes(w)
-    peak, peak_src = peaks()
-    achieved = step_bytes * args.steps / (ms / 1e3) / 1e9
+    launches = K
+    bytes_per_launch = step_bytes * nlayers
+    avg_launch_us = ms * 1e3 / launches
+    achieved = bytes_per_launch / (avg_launch_us / 1e6) / 1e9
+    dd = dist_of(dist_ms)
     ffn_bytes = w.K * rec_r + rec_s
-    resident = sum(L.nbytes() for L in layers)
+    pc = dist_of(pc_times)
+    ffn_mean = statistics.mean(ffn_ms)
+    cfg = workload_config(w, nlayers, world)
     line = {
-        "metric": "MoE-layer decode tokens/s", "value": tps, "unit": "tokens/s", "n_gpus": world,
-        "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms / args.steps, "higher_is_better": True,
+        "metric": "MoE-layer decode tokens/s", "value": tps, "unit": "layer-tokens/s", "n_gpus": world,
+        "steps": K, "warmup": W, "ms_per_step": ms / K, "higher_is_better": True,
         "scaling": "weak", "vs_baseline": None, "dtype": "u8xs8-mma+f32", "data": "synthetic",
-        "config": {"workload": "%s: batch-1 MoE layer H%d E%d I%d top-%d + shared, %d-bit routed / %d-bit shared, "
-                               "group %d" % (w.name, w.H, w.E, w.I, w.K, w.bits_routed, w.bits_shared, w.group),
-                   "batch": 1, "layers_resident": nlayers, "resident_bytes": resident,
-                   "l2": "inputs larger than L2: each launch walks %d resident layers (%.1f GB)" %
-                         (nlayers, resident / 1e9),
-                   "parallelism": "replicas" if world > 1 else "single GPU",
-                   "launch": "moe_decode_layers: one persistent kernel per %d layer-token steps, CUDA graph" % nlayers},
-        "step_bytes": step_bytes,
+        "config": cfg,
+        "launch": "moe_decode_layers: one persistent kernel per step (%d layers), CUDA graph replay" % nlayers,
+        "tokens_per_s": tps / nlayers,
+        "step_bytes": bytes_per_launch,
         "effective_gbs": achieved,
         "frac_of_8tbs": achieved * 1e9 / 8e12,
         "roofline": {"bound": "hbm", "achieved": achieved, "peak": peak, "unit": "GB/s", "frac": achieved / peak,
                      "traffic": measured_traffic(w, nlayers), "kernel": "k_decode_layers",
-                     "bytes_per_launch": step_bytes * nlayers, "avg_launch_us": ms * 1e3 / launches,
-                     "peak_source": peak_src},
-        "per_call": {"value": pc_tps, "unit": "tokens/s",
-                     "path": "moe_router_topk + moe_expert_ffn_q + moe_combine_residual, graph per step",
-                     "ffn_call_us": ffn_avg_ms * 1e3, "ffn_call_gbs": ffn_bytes / (ffn_avg_ms / 1e3) / 1e9},
+                     "layers_per_launch": nlayers, "bytes_per_layer": step_bytes,
+                     "bytes_per_launch": bytes_per_launch, "avg_launch_us": avg_launch_us,
+                     "launches_timed": launches, "peak_source": peak_src,
+                     "launch_distribution_us": {k: v * 1e3 if k.endswith("_ms") else v for k, v in dd.items()}},
+        "per_call": {"value": 1.0 / (pc["median_ms"] / 1e3), "unit": "layer-tokens/s",
+                     "path": "moe_router_topk + moe_expert_ffn_q + moe_combine_residual, one graph per layer",
+                     "timing": pc, "ffn_call_us": ffn_mean * 1e3,
+                     "ffn_call_gbs": ffn_bytes / (ffn_mean / 1e3) / 1e9},
         "gpu_launches": launches,
         "clocks": clk.summary(),
     }
@@ -547,9 +639,9 @@ def main():
         import datetime
         dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120))
     line = run_ours(args, w, rank, world, local_rank)
-    if rank == 0:
+    if rank == 0 and line is not None:
         tps, secs = oracle_tokens_per_s(w, args.cpu_sample)
-        line["cpu_baseline"] = {"value": tps, "unit": "tokens/s", "cores": 1, "kind": "oracle",
+        line["cpu_baseline"] = {"value": tps, "unit": "layer-tokens/s", "cores": 1, "kind": "oracle",
                                 "sample": "%d layer-token steps of %s through the single-threaded fp64 C oracle "
                                           "(%.1f s of oracle work)" % (args.cpu_sample, w.name, secs)}
         print(json.dumps(line), flush=True)

@@ -127,7 +127,27 @@ size_t moe_workspace_bytes(int B, int K, int H, int I, int E);
 moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream);
 
 /*
- * moe_pack_q -- pack one code matrix into the layout of moe_layer_q.
+ * moe_workspace_debug -- testing hook for the bounded waits (the pages have
+ * no counterpart). Sets two words of the workspace control block, in stream
+ * order, for the calls that use the workspace afterwards:
+ *   wait_budget_us  every bounded wait gives up after about this many
+ *                   microseconds (0: the default, about one second)
+ *   withhold_cta    c + 1: CTA c of moe_decode_layers skips its arrival on
+ *                   the first layer's logits exchange, so every CTA's wait on
+ *                   it runs out: the kernel then sets MOE_ERR_TIMEOUT, lets
+ *                   its bulk copies land and exits; 0: off
+ * moe_workspace_init clears both. MOE_ERR_WORKSPACE for a missing or short
+ * workspace, MOE_ERR_ALIGN, MOE_ERR_INVALID_ARG for withhold_cta < 0.
+ */
+moe_status moe_workspace_debug(void* ws, size_t ws_bytes, unsigned wait_budget_us, int withhold_cta, void* stream);
+
+/*
+ * moe_pack_q -- pack one code matrix into the plain row-major interchange
+ * image: code j of a row at bit offset (j*bits) mod 8 of byte j*bits/8 of
+ * the row (low bits first), and the (scale, bias) bf16 pair of each (row,
+ * group) interleaved, scale first. This image is for storage and exchange;
+ * the resident expert record that moe_expert_ffn_q and moe_decode_layers
+ * read is tile-major and is written by moe_pack_expert.
  *   codes      u8 [rows, cols], one code per byte, values < 2^bits
  *   scale_bf16 bf16 [rows, cols/group]
  *   bias_bf16  bf16 [rows, cols/group]
@@ -147,8 +167,10 @@ moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* 
 /*
  * moe_pack_expert -- pack the gate [I,H], up [I,H] and down [H,I] code
  * matrices of one expert (u8 codes, bf16 scale/bias [rows, cols/group]) into
- * one expert record at record_out (moe_expert_bytes(H, I, bits, group)
- * bytes), with the same packing as moe_pack_q. ws as in moe_pack_q.
+ * one resident expert record at record_out (moe_expert_bytes(H, I, bits,
+ * group) bytes) in the tile-major layout described at moe_layer_q. The
+ * record holds the same codes and (scale, bias) pairs as the row-major image
+ * of moe_pack_q, in a different order. ws as in moe_pack_q.
  */
 moe_status moe_pack_expert(const uint8_t* codes_gate, const void* scale_gate_bf16, const void* bias_gate_bf16,
                            const uint8_t* codes_up, const void* scale_up_bf16, const void* bias_up_bf16,
@@ -168,7 +190,8 @@ moe_status moe_pack_expert(const uint8_t* codes_gate, const void* scale_gate_bf1
  *   logits_out    fp32 [B, E] or NULL
  * Logits accumulate in fp32 (bf16 products are exact in fp32). NaN logits
  * rank as -inf; a pick left with no finite logit is -1 and sets
- * MOE_ERR_INDEX (its weight is 0).
+ * MOE_ERR_INDEX (its weight is 0). E <= 1024 (MOE_ERR_UNSUPPORTED above:
+ * the selection holds 32 logits per lane of a warp).
  * Source: "Kien truc mo hinh" (512 experts, K active per token).
  */
 moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B, int H, int E, int K,
@@ -235,6 +258,21 @@ moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers, const void
                              float* resid_out, void* xnorm_bf16_out, float eps, void* ws, size_t ws_bytes,
                              void* stream);
 
+/*
+ * moe_rmsnorm -- x[b] = bf16(r[b] / sqrt(mean(r[b]^2) + eps) * weight), the
+ * RMS norm of the Flash-MoE page ("Metal Compute Shaders": a kernel of its
+ * own between the MoE block and the next layer), rounded to nearest-even
+ * bf16.
+ *   r            fp32 [B, H]
+ *   weight_bf16  bf16 [H], or NULL for unit weight
+ *   xnorm_bf16_out  bf16 [B, H]
+ * H a multiple of 8 (MOE_ERR_UNSUPPORTED otherwise); eps >= 0. The same
+ * norm is fused into moe_combine_residual and moe_decode_layers (unit
+ * weight there).
+ */
+moe_status moe_rmsnorm(const float* r, const void* weight_bf16, int B, int H, float eps, void* xnorm_bf16_out,
+                       void* stream);
+
 /* Read (and clear) the workspace error word. Synchronises `stream`.
  * Returns MOE_OK, MOE_ERR_INDEX, MOE_ERR_RANGE, MOE_ERR_TIMEOUT, or
  * MOE_ERR_CUDA if the copy itself failed. */
@@ -253,7 +291,8 @@ moe_status moe_get_device_error(void* ws, void* stream);
  * Scratch is a MOEQ_STATIC_SCRATCH_BYTES array inside the library, held by
  * every GPU that loads it until the process exits. A shape whose
  * moe_workspace_bytes(B, K, H, I, E) exceeds that size is rejected with
- * MOE_ERR_WORKSPACE before anything is launched. The call allocates nothing:
+ * MOE_ERR_WORKSPACE; every argument error (those of moe_expert_ffn_q first)
+ * returns before anything is queued. The call allocates nothing:
  * it clears the array's control block with cudaMemsetAsync and runs the
  * kernels of moe_expert_ffn_q on the array. All calls on a device share the
  * array and it keeps the last call's contents, so calls that overlap on the

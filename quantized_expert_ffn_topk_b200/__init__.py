@@ -49,6 +49,8 @@ _SIGS = {
     "moe_expert_layout": (_INT, [_INT, _INT, _INT, _INT, ctypes.POINTER(_SZ)]),
     "moe_workspace_bytes": (_SZ, [_INT, _INT, _INT, _INT, _INT]),
     "moe_workspace_init": (_INT, [_VP, _SZ, _VP]),
+    "moe_workspace_debug": (_INT, [_VP, _SZ, ctypes.c_uint, _INT, _VP]),
+    "moe_rmsnorm": (_INT, [_VP, _VP, _INT, _INT, _FLT, _VP, _VP]),
     "moe_pack_q": (_INT, [_VP, _VP, _VP, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP]),
     "moe_pack_expert": (_INT, [_VP] * 9 + [_INT, _INT, _INT, _INT, _VP, _VP, _VP]),
     "moe_router_topk": (_INT, [_VP, _VP, _INT, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
@@ -127,6 +129,12 @@ def moe_workspace_init(ws, ws_bytes: int = None, stream=None) -> None:
     _check(lib().moe_workspace_init(_ptr(ws), n, _stream(stream)), "moe_workspace_init")
 
 
+def moe_workspace_debug(ws, ws_bytes: int, wait_budget_us: int, withhold_cta: int, stream=None) -> None:
+    """Testing hook of the bounded waits (see include/moeq.h)."""
+    _check(lib().moe_workspace_debug(_ptr(ws), ws_bytes, int(wait_budget_us), int(withhold_cta), _stream(stream)),
+           "moe_workspace_debug")
+
+
 # ---- the four calls ---------------------------------------------------------
 
 def moe_pack_q(codes, scale_bf16, bias_bf16, rows: int, cols: int, bits: int, group: int, packed_out, sb_out,
@@ -161,10 +169,22 @@ def moe_combine_residual(layer: moe_layer_q, y, w, x_bf16, resid_in, B: int, res
            "moe_combine_residual")
 
 
+def moe_rmsnorm(r, weight_bf16, B: int, H: int, eps: float, xnorm_bf16_out, stream=None) -> None:
+    _check(lib().moe_rmsnorm(_ptr(r), _ptr(weight_bf16), B, H, float(eps), _ptr(xnorm_bf16_out), _stream(stream)),
+           "moe_rmsnorm")
+
+
+def layer_table(layers):
+    """A C array of moe_layer_q for moe_decode_layers, built once and reused
+    across calls (saves rebuilding it on every token)."""
+    return (moe_layer_q * len(layers))(*layers)
+
+
 def moe_decode_layers(layers, x_bf16, resid_in, renorm: bool, forced_idx, idx_out, w_out, resid_out, xnorm_bf16_out,
                       eps: float, ws, ws_bytes: int, stream=None) -> None:
-    """layers: a sequence of moe_layer_q (one token through all of them)."""
-    arr = (moe_layer_q * len(layers))(*layers)
+    """layers: a sequence of moe_layer_q (one token through all of them), or
+    a table from layer_table()."""
+    arr = layers if isinstance(layers, ctypes.Array) else (moe_layer_q * len(layers))(*layers)
     _check(lib().moe_decode_layers(arr, len(layers), _ptr(x_bf16), _ptr(resid_in), int(bool(renorm)),
                                    _ptr(forced_idx), _ptr(idx_out), _ptr(w_out), _ptr(resid_out),
                                    _ptr(xnorm_bf16_out), float(eps), _ptr(ws), ws_bytes, _stream(stream)),

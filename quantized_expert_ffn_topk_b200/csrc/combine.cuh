@@ -88,4 +88,38 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(CombineParams p) {
   }
 }
 
+// moe_rmsnorm: grid B, one token per CTA. xn = bf16(r * rsqrt(mean(r^2) +
+// eps) * weight) with unit weight when none is given (the RMS norm kernel of
+// the Flash-MoE page, "Metal Compute Shaders"). H a multiple of 8; r is read
+// twice (the second time from L1/L2).
+__global__ void __launch_bounds__(kCombineThreads) k_rmsnorm(const float* r, const uint16_t* weight, int H, float eps,
+                                                             uint16_t* out) {
+  __shared__ float red[32];
+  pdl_trigger();
+  pdl_wait();
+  const int b = blockIdx.x, n4 = H / 4;
+  const float4* rb = reinterpret_cast<const float4*>(r + (size_t)b * H);
+  float ss = 0.f;
+  for (int j = threadIdx.x; j < n4; j += blockDim.x) {
+    const float4 v = rb[j];
+    ss += v.x * v.x + v.y * v.y + v.z * v.z + v.w * v.w;
+  }
+  ss = block_sum(ss, red);
+  const float inv = rsqrtf(ss / (float)H + eps);
+  uint2* ob = reinterpret_cast<uint2*>(out + (size_t)b * H);
+  for (int j = threadIdx.x; j < n4; j += blockDim.x) {
+    const float4 v = rb[j];
+    float f[4] = {v.x * inv, v.y * inv, v.z * inv, v.w * inv};
+    if (weight) {
+      const uint2 wv = reinterpret_cast<const uint2*>(weight)[j];
+      f[0] *= bf16_bits_to_f32(wv.x & 0xFFFFu);
+      f[1] *= bf16_bits_to_f32(wv.x >> 16);
+      f[2] *= bf16_bits_to_f32(wv.y & 0xFFFFu);
+      f[3] *= bf16_bits_to_f32(wv.y >> 16);
+    }
+    ob[j] = make_uint2((uint32_t)f32_to_bf16_bits(f[0]) | ((uint32_t)f32_to_bf16_bits(f[1]) << 16),
+                       (uint32_t)f32_to_bf16_bits(f[2]) | ((uint32_t)f32_to_bf16_bits(f[3]) << 16));
+  }
+}
+
 }  // namespace moeq

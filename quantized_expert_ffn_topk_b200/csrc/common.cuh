@@ -12,10 +12,12 @@ namespace moeq {
 // Workspace control block: the first 256 bytes of every workspace.
 struct WsCtrl {
   int error;                // first device-side moe_status (0 = none)
-  unsigned router_ticket[8];  // last-CTA tickets of the router kernel, one per 8-token tile (0 between calls)
+  unsigned router_ticket[16]; // last-CTA tickets of the router kernel, one per 8-token tile (0 between calls)
   unsigned exit_count;      // CTAs that left the fused decode kernel (0 between calls)
   unsigned sync[4];         // arrival counters of the fused decode kernel (0 between calls)
-  unsigned pad[50];
+  unsigned wait_us;         // budget of every bounded wait in microseconds (0: about one second)
+  int withhold_cta;         // c + 1: CTA c of the fused kernel withholds its first logits arrival (0: none)
+  unsigned pad[40];
 };
 static_assert(sizeof(WsCtrl) == 256, "control block is 256 bytes");
 
@@ -199,30 +201,38 @@ __device__ __forceinline__ void arrive_release_gpu(unsigned* counter) {
   asm volatile("red.release.gpu.global.add.u32 [%0], 1;" ::"l"(counter) : "memory");
 }
 
-// Wait budget for every spin in the library: ~1 s of SM clock cycles.
+// Default budget of every spin in the library: ~1 s of SM clock cycles.
 constexpr long long kWaitBudgetCycles = 2000000000LL;
 
-// Bounded wait for an mbarrier phase; false on timeout or when `abort` is set.
-// Waiting warps back off with __nanosleep so that they leave the issue slots
-// to the warps that have work.
-__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort) {
+// The budget a kernel's waits use: the workspace's wait_us (a testing hook,
+// about 2000 cycles per microsecond) or the default. Read once per kernel.
+__device__ __forceinline__ long long wait_budget(const WsCtrl* c) {
+  const unsigned us = c ? *reinterpret_cast<const volatile unsigned*>(&c->wait_us) : 0u;
+  return us ? (long long)us * 2000LL : kWaitBudgetCycles;
+}
+
+// Bounded wait for an mbarrier phase; false after `budget` cycles or when
+// `abort` is set. Waiting warps back off with __nanosleep so that they leave
+// the issue slots to the warps that have work.
+__device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const volatile int* abort, long long budget) {
   if (mbar_try_wait(bar, parity)) return true;
   const long long t0 = clock64();
   while (true) {
     __nanosleep(64);
     if (mbar_try_wait(bar, parity)) return true;
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) return false;
+    if (clock64() - t0 > budget) return false;
   }
 }
 
 // Bounded wait until *counter >= target (gpu-scope acquire).
-__device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned target, const volatile int* abort) {
+__device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned target, const volatile int* abort,
+                                             long long budget) {
   if (ld_acquire_gpu(counter) >= target) return true;
   const long long t0 = clock64();
   while (ld_acquire_gpu(counter) < target) {
     if (*abort) return false;
-    if (clock64() - t0 > kWaitBudgetCycles) return false;
+    if (clock64() - t0 > budget) return false;
     __nanosleep(32);
   }
   return true;

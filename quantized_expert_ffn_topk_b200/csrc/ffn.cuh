@@ -67,8 +67,9 @@ __device__ __forceinline__ void ffn_issue(unsigned char* tiles, int stride, uint
 
 // Bounded wait for buffer j of the current round; on a timeout the CTA
 // records MOE_ERR_TIMEOUT and stops.
-__device__ __forceinline__ bool ffn_wait(uint64_t* bar, int j, int round, WsCtrl* ctrl, volatile int* abort) {
-  const bool ok = mbar_wait(&bar[j], (uint32_t)(round & 1), abort);
+__device__ __forceinline__ bool ffn_wait(uint64_t* bar, int j, int round, WsCtrl* ctrl, volatile int* abort,
+                                         long long budget) {
+  const bool ok = mbar_wait(&bar[j], (uint32_t)(round & 1), abort, budget);
   if (!ok && (threadIdx.x & 31) == 0) {
     if (!*abort) set_error(ctrl, MOE_ERR_TIMEOUT);
     *abort = 1;
@@ -78,10 +79,10 @@ __device__ __forceinline__ bool ffn_wait(uint64_t* bar, int j, int round, WsCtrl
 
 // Before the CTA leaves after a timeout: every copy it issued must have
 // landed (bounded).
-__device__ __forceinline__ void ffn_drain(uint64_t* bar, int nt, int round) {
+__device__ __forceinline__ void ffn_drain(uint64_t* bar, int nt, int round, long long budget) {
   if (threadIdx.x < nt) {
     const long long t0 = clock64();
-    while (!mbar_try_wait(&bar[threadIdx.x], (uint32_t)(round & 1)) && clock64() - t0 < kWaitBudgetCycles) {
+    while (!mbar_try_wait(&bar[threadIdx.x], (uint32_t)(round & 1)) && clock64() - t0 < budget) {
     }
   }
 }
@@ -120,6 +121,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
   // the shared expert's tiles do not depend on the previous kernel
   if (warp == 0 && t_lo < t_hi) ffn_issue(tiles, p.gu_stride, bar, t_lo, min(p.gu_nbuf, t_hi - t_lo), src, is_shared);
   pdl_wait();
+  const long long budget = wait_budget(p.ctrl);
   int round = 0, nt = 0;
   for (int r0 = t_lo; r0 < t_hi; r0 += p.gu_nbuf, ++round) {
     nt = min(p.gu_nbuf, t_hi - r0);
@@ -135,7 +137,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
       const int j = pc / kFfnPieces, q = pc % kFfnPieces, k = (r0 + j) / tps;
       const bool routed = k < p.K;
       float acc0 = 0.f, acc1 = 0.f;
-      if (ffn_wait(bar, j, round, p.ctrl, &s_abort) && ffn_slot_rec(p, k)) {
+      if (ffn_wait(bar, j, round, p.ctrl, &s_abort, budget) && ffn_slot_rec(p, k)) {
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
         const int g0 = piece_lo(q, (int)g.ng_h), g1 = piece_lo(q + 1, (int)g.ng_h);
         const unsigned char* blk = tiles + (size_t)j * p.gu_stride + (size_t)g0 * g.blk;
@@ -164,7 +166,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
     __syncthreads();  // buffers and partials free for the next round
     if (s_abort) break;
   }
-  if (s_abort) ffn_drain(bar, nt, round);
+  if (s_abort) ffn_drain(bar, nt, round, budget);
 }
 
 // Down: job u = (slot u / (H/16), down tile u % (H/16)); 16 threads per job
@@ -204,6 +206,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
   // the shared expert's tiles do not depend on the previous kernels
   if (warp == 0 && t_lo < t_hi) ffn_issue(tiles, p.dn_stride, bar, t_lo, min(p.dn_nbuf, t_hi - t_lo), src, is_shared);
   pdl_wait();
+  const long long budget = wait_budget(p.ctrl);
   int round = 0, nt = 0;
   for (int r0 = t_lo; r0 < t_hi; r0 += p.dn_nbuf, ++round) {
     nt = min(p.dn_nbuf, t_hi - r0);
@@ -223,7 +226,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
       const int j = pc / kFfnPieces, q = pc % kFfnPieces, k = (r0 + j) / tpd;
       const bool routed = k < p.K;
       float acc0 = 0.f, acc1 = 0.f;
-      if (ffn_wait(bar, j, round, p.ctrl, &s_abort) && ffn_slot_rec(p, k)) {
+      if (ffn_wait(bar, j, round, p.ctrl, &s_abort, budget) && ffn_slot_rec(p, k)) {
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
         const int g0 = piece_lo(q, (int)g.ng_i), g1 = piece_lo(q + 1, (int)g.ng_i);
         const unsigned char* blk = tiles + (size_t)j * p.dn_stride + (size_t)g0 * g.blk;
@@ -248,7 +251,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
     __syncthreads();
     if (s_abort) break;
   }
-  if (s_abort) ffn_drain(bar, nt, round);
+  if (s_abort) ffn_drain(bar, nt, round, budget);
 }
 
 }  // namespace moeq

@@ -4,6 +4,7 @@
 
 #include <algorithm>
 #include <cstring>
+#include <mutex>
 
 #include "combine.cuh"
 #include "common.cuh"
@@ -64,14 +65,33 @@ moe_status launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem
   return MOE_OK;
 }
 
+// Raise a kernel's dynamic shared-memory limit to `bytes` once per (kernel,
+// device): the attribute is set only when a call needs more than before.
 template <typename K>
 moe_status ensure_smem(K kern, size_t bytes) {
   if (bytes <= 48 * 1024) return MOE_OK;
   if (bytes > 227 * 1024) return MOE_ERR_UNSUPPORTED;
+  struct Seen { const void* fn; int dev; size_t bytes; };
+  static std::mutex mu;
+  static Seen seen[64];
+  static int nseen = 0;
+  int dev = 0;
+  if (cudaGetDevice(&dev) != cudaSuccess) {
+    (void)cudaGetLastError();
+    return MOE_ERR_CUDA;
+  }
+  const void* fn = reinterpret_cast<const void*>(kern);
+  std::lock_guard<std::mutex> lock(mu);
+  Seen* e = nullptr;
+  for (int i = 0; i < nseen; ++i)
+    if (seen[i].fn == fn && seen[i].dev == dev) e = &seen[i];
+  if (e && e->bytes >= bytes) return MOE_OK;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)bytes) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
   }
+  if (e) e->bytes = bytes;
+  else if (nseen < 64) seen[nseen++] = Seen{fn, dev, bytes};
   return MOE_OK;
 }
 
@@ -133,7 +153,24 @@ moe_status check_layer(const moe_layer_q* L) {
 
 bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes);  // below
 
+__global__ void k_ws_debug(WsCtrl* c, unsigned wait_us, int withhold_cta) {
+  c->wait_us = wait_us;
+  c->withhold_cta = withhold_cta;
+}
+
 }  // namespace
+
+// Arguments of moe_expert_ffn_q other than the workspace (layer, pointers,
+// batch, alignment); MOE_OK or the status the call returns.
+moe_status ffn_check_args(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx, const float* y_out) {
+  moe_status st = check_layer(L);
+  if (st != MOE_OK) return st;
+  if (!x_bf16 || !idx || !y_out) return MOE_ERR_INVALID_ARG;
+  if (B <= 0 || B > MOEQ_MAX_B) return MOE_ERR_INVALID_ARG;
+  if (!aligned16(x_bf16) || !aligned16(y_out) || !aligned16(idx)) return MOE_ERR_ALIGN;
+  return MOE_OK;
+}
+
 }  // namespace moeq
 
 using namespace moeq;
@@ -191,6 +228,25 @@ moe_status moe_workspace_init(void* ws, size_t ws_bytes, void* stream) {
     return MOE_ERR_CUDA;
   }
   return MOE_OK;
+}
+
+moe_status moe_workspace_debug(void* ws, size_t ws_bytes, unsigned wait_budget_us, int withhold_cta, void* stream) {
+  if (!ws || ws_bytes < sizeof(WsCtrl)) return MOE_ERR_WORKSPACE;
+  if (!aligned16(ws)) return MOE_ERR_ALIGN;
+  if (withhold_cta < 0) return MOE_ERR_INVALID_ARG;
+  k_ws_debug<<<1, 1, 0, (cudaStream_t)stream>>>(reinterpret_cast<WsCtrl*>(ws), wait_budget_us, withhold_cta);
+  return launch_status();
+}
+
+moe_status moe_rmsnorm(const float* r, const void* weight_bf16, int B, int H, float eps, void* xnorm_bf16_out,
+                       void* stream) {
+  if (!r || !xnorm_bf16_out) return MOE_ERR_INVALID_ARG;
+  if (B <= 0 || H <= 0 || !(eps >= 0.f)) return MOE_ERR_INVALID_ARG;
+  if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(r) || !aligned16(xnorm_bf16_out) || (weight_bf16 && !aligned16(weight_bf16))) return MOE_ERR_ALIGN;
+  return launch_pdl(k_rmsnorm, dim3(B), dim3(kCombineThreads), 0, (cudaStream_t)stream, r,
+                    reinterpret_cast<const uint16_t*>(weight_bf16), H, eps,
+                    reinterpret_cast<uint16_t*>(xnorm_bf16_out));
 }
 
 moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* bias_bf16, int rows, int cols,
@@ -268,6 +324,7 @@ moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B,
   if (!x_bf16 || !router_w_bf16 || !idx_out || !w_out) return MOE_ERR_INVALID_ARG;
   if (B <= 0 || B > MOEQ_MAX_B || H <= 0 || E <= 0 || K <= 0 || K > MOEQ_MAX_K || K > E) return MOE_ERR_INVALID_ARG;
   if (H % 8 != 0) return MOE_ERR_UNSUPPORTED;
+  if (E > kRouterMaxE) return MOE_ERR_UNSUPPORTED;  // the selection holds 32 logits per lane
   if (!ws) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_workspace_bytes(B, K, H, 32, E)) return MOE_ERR_WORKSPACE;
   if (!aligned16(x_bf16) || !aligned16(router_w_bf16) || !aligned16(ws)) return MOE_ERR_ALIGN;
@@ -296,13 +353,11 @@ moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B,
 
 moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx, float* y_out,
                             void* ws, size_t ws_bytes, void* stream) {
-  moe_status st = check_layer(L);
+  moe_status st = ffn_check_args(L, x_bf16, B, idx, y_out);
   if (st != MOE_OK) return st;
-  if (!x_bf16 || !idx || !y_out) return MOE_ERR_INVALID_ARG;
-  if (B <= 0 || B > MOEQ_MAX_B) return MOE_ERR_INVALID_ARG;
   if (!ws) return MOE_ERR_WORKSPACE;
   if (ws_bytes < moe_workspace_bytes(B, L->K, L->H, L->I, L->E)) return MOE_ERR_WORKSPACE;
-  if (!aligned16(x_bf16) || !aligned16(y_out) || !aligned16(ws) || !aligned16(idx)) return MOE_ERR_ALIGN;
+  if (!aligned16(ws)) return MOE_ERR_ALIGN;
   FfnParams p{};
   p.experts = reinterpret_cast<const uint8_t*>(L->experts);
   p.shared = reinterpret_cast<const uint8_t*>(L->shared);

@@ -23,6 +23,10 @@
 #include "common.cuh"
 #include "moeq.h"
 
+namespace moeq {
+moe_status ffn_check_args(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx, const float* y_out);
+}
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -60,13 +64,15 @@ moe_status scratch_address(void** out) {
 
 extern "C" moe_status moe_expert_ffn_q_static(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx,
                                               float* y_out, int32_t* error_out, void* stream) {
-  if (!L || B <= 0 || B > MOEQ_MAX_B) return MOE_ERR_INVALID_ARG;
+  // every argument error returns before anything is queued
+  moe_status st = moeq::ffn_check_args(L, x_bf16, B, idx, y_out);
+  if (st != MOE_OK) return st;
+  if (error_out && (reinterpret_cast<uintptr_t>(error_out) & 3u)) return MOE_ERR_ALIGN;
   const size_t need = moe_workspace_bytes(B, L->K, L->H, L->I, L->E);
   if (need == 0) return MOE_ERR_INVALID_ARG;
   if (need > (size_t)MOEQ_STATIC_SCRATCH_BYTES) return MOE_ERR_WORKSPACE;
-  if (error_out && (reinterpret_cast<uintptr_t>(error_out) & 3u)) return MOE_ERR_ALIGN;
   void* ws = nullptr;
-  moe_status st = scratch_address(&ws);
+  st = scratch_address(&ws);
   if (st != MOE_OK) return st;
   cudaStream_t s = (cudaStream_t)stream;
   if (cudaMemsetAsync(ws, 0, sizeof(moeq::WsCtrl), s) != cudaSuccess) {

@@ -9,6 +9,7 @@ namespace moeq {
 constexpr int kRouterWarps = 8;     // warps per CTA, one expert row per warp at a time
 constexpr int kRouterTokTile = 8;   // tokens of one CTA (its x staged in shared memory)
 constexpr int kRouterUnroll = 8;    // 16-byte loads of one row in flight per lane (the rows were prefetched to L2)
+constexpr int kRouterMaxE = 1024;   // experts the selection holds: 32 keys per lane
 
 struct RouterParams {
   const uint16_t* x;       // [B, H] bf16
@@ -53,7 +54,7 @@ __device__ __forceinline__ float key_logit(uint32_t k) {
 __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const int32_t* forced, int32_t* idx_out,
                                float* w_out, WsCtrl* ctrl) {
   const int lane = threadIdx.x & 31;
-  constexpr int NV = 32;
+  constexpr int NV = kRouterMaxE / 32;
   uint32_t key[NV];
   uint32_t lk = 0u;
 #pragma unroll

@@ -216,7 +216,7 @@ __device__ __forceinline__ uint32_t item_source(const StackParams& p, const Item
 // are already free (lane j -> item next + j); if none is, lane 0 waits for
 // the first. Returns false if a wait gave up.
 __device__ bool issue_items(const StackParams& p, const ItemPlan& P, Ring& R, int l, int it0, int it1, uint32_t seq0,
-                            const int* s_idx, const volatile int* abort) {
+                            const int* s_idx, const volatile int* abort, long long budget) {
   const int lane = threadIdx.x & 31;
   const int width = min(32, R.nslot);
   for (int next = it0; next < it1;) {
@@ -229,7 +229,7 @@ __device__ bool issue_items(const StackParams& p, const ItemPlan& P, Ring& R, in
     nr = min(nr, n);
     if (nr == 0) {
       bool ok = true;
-      if (lane == 0) ok = mbar_wait(&R.empty[slot], (fill - 1) & 1, abort);
+      if (lane == 0) ok = mbar_wait(&R.empty[slot], (fill - 1) & 1, abort, budget);
       if (!__shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0)) return false;
       nr = 1;
     }
@@ -374,11 +374,12 @@ __device__ void block_topk(const StackParams& p, int l, TopkScratch& S, int* s_i
 }
 
 // Bounded wait until the shared-memory flag reaches target.
-__device__ __forceinline__ bool flag_wait(const volatile int* f, int target, const volatile int* abort) {
+__device__ __forceinline__ bool flag_wait(const volatile int* f, int target, const volatile int* abort,
+                                          long long budget) {
   if (*f >= target) return true;
   const long long t0 = clock64();
   while (*f < target) {
-    if (*abort || clock64() - t0 > kWaitBudgetCycles) return false;
+    if (*abort || clock64() - t0 > budget) return false;
     __nanosleep(32);
   }
   return true;
@@ -389,12 +390,13 @@ __device__ __forceinline__ bool flag_wait(const volatile int* f, int target, con
 // Bounded wait until the producer has issued ring sequence number seq into
 // `slot` (it records that before arming the slot's full barrier). The copy
 // still has to land after that, so the pause between looks can be long.
-__device__ __forceinline__ bool slot_issued(const int* last, int slot, int seq, const volatile int* abort) {
+__device__ __forceinline__ bool slot_issued(const int* last, int slot, int seq, const volatile int* abort,
+                                            long long budget) {
   const volatile int* v = last;
   if (v[slot] == seq) return true;
   const long long t0 = clock64();
   while (v[slot] != seq) {
-    if (*abort || clock64() - t0 > kWaitBudgetCycles) return false;
+    if (*abort || clock64() - t0 > budget) return false;
     __nanosleep(200);
   }
   return true;
@@ -422,6 +424,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;
+  const long long budget = wait_budget(p.ctrl);
+  // testing hook: this CTA skips its first logits arrival, so every CTA's
+  // logits wait runs out of budget (a fault made on the host, never on the GPU)
+  const bool withhold = *reinterpret_cast<const volatile int*>(&p.ctrl->withhold_cta) == (int)blockIdx.x + 1;
 
   if (tid == 0) {
     make_plan(p, P);
@@ -448,19 +454,19 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
   if (warp == kCWarps) {
     // ===================== producer warp =====================
     Ring R{full_bar, empty_bar, s_last, sm + p.sm_ring, p.slot_bytes, p.nslot};
-    if (!issue_items(p, P, R, 0, 0, P.n_pre_items, 0u, s_idx, &s_abort) && lane == 0) fail();
+    if (!issue_items(p, P, R, 0, 0, P.n_pre_items, 0u, s_idx, &s_abort, budget) && lane == 0) fail();
     for (int l = 0; l < p.n_layers; ++l) {
       // routing: the compute warps publish layer l's picks in s_idx/s_w
-      if (lane == 0 && !s_abort && !flag_wait(&s_topk_ready, l + 1, &s_abort) && !s_abort) fail();
+      if (lane == 0 && !s_abort && !flag_wait(&s_topk_ready, l + 1, &s_abort, budget) && !s_abort) fail();
       __syncwarp();
       __threadfence_block();
       // routed gate/up items (they gate the h exchange), the routed down
       // items (needed only after it), then the next layer's router, shared
       // gate/up and shared down items
       const uint32_t seq_l = (uint32_t)(l * n_items);
-      bool ok = !s_abort && issue_items(p, P, R, l, P.n_pre_items, n_items, seq_l + P.n_pre_items, s_idx, &s_abort);
+      bool ok = !s_abort && issue_items(p, P, R, l, P.n_pre_items, n_items, seq_l + P.n_pre_items, s_idx, &s_abort, budget);
       if (ok && l + 1 < p.n_layers)
-        ok = issue_items(p, P, R, l + 1, 0, P.n_pre_items, (uint32_t)((l + 1) * n_items), s_idx, &s_abort);
+        ok = issue_items(p, P, R, l + 1, 0, P.n_pre_items, (uint32_t)((l + 1) * n_items), s_idx, &s_abort, budget);
       if (!ok && lane == 0 && !s_abort) fail();
       __syncwarp();
     }
@@ -469,7 +475,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       const int j = s_last[lane];
       if (j >= 0) {
         const long long t0 = clock64();
-        while (!mbar_try_wait(&full_bar[lane], (j / p.nslot) & 1) && clock64() - t0 < kWaitBudgetCycles) {
+        while (!mbar_try_wait(&full_bar[lane], (j / p.nslot) & 1) && clock64() - t0 < budget) {
         }
       }
     }
@@ -496,8 +502,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       const int pos = pc - P.piece0[it];
       const uint32_t seq = (uint32_t)(l * n_items + it);
       const int slot = seq % p.nslot;
-      bool ok = slot_issued(s_last, slot, (int)seq, &s_abort);
-      ok = ok && mbar_wait(&full_bar[slot], (seq / p.nslot) & 1, &s_abort);
+      bool ok = slot_issued(s_last, slot, (int)seq, &s_abort, budget);
+      ok = ok && mbar_wait(&full_bar[slot], (seq / p.nslot) & 1, &s_abort, budget);
       if (!ok && lane == 0 && !s_abort) fail();
       const unsigned char* sl = ring + (size_t)slot * p.slot_bytes;
       if (P.kind[it] == kItemRouter) {
@@ -585,7 +591,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     // segment into its own slot's image; a group's lanes are adjacent and
     // share a slot (I is a multiple of G).
     auto stage_h = [&](int k0, int k1, int c, unsigned target) {
-      if (tid == 0 && !counter_wait(p.sync + c, target, &s_abort) && !s_abort) fail();
+      if (tid == 0 && !counter_wait(p.sync + c, target, &s_abort, budget) && !s_abort) fail();
       named_sync(1, kCThreads);
       const int spk = I / 16;  // segments per slot
       for (int s0 = tid - lane; s0 < (k1 - k0) * spk; s0 += kCThreads) {
@@ -612,7 +618,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         float v[16];
         const bool active = tid < nseg;
         if (l > 0) {
-          if (tid == 0 && !counter_wait(p.sync + kSyncResid, (unsigned)l * G1, &s_abort) && !s_abort) fail();
+          if (tid == 0 && !counter_wait(p.sync + kSyncResid, (unsigned)l * G1, &s_abort, budget) && !s_abort) fail();
           named_sync(1, kCThreads);
           float ss = 0.f;
           if (active) {
@@ -676,14 +682,14 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
           __stcg(p.logits + P.r0 + lane, lg);
         }
         __syncwarp();
-        if (lane == 0) arrive_release_gpu(p.sync + kSyncLogits);
+        if (lane == 0 && !(withhold && l == 0)) arrive_release_gpu(p.sync + kSyncLogits);
       }
       run_items(l, P.n_router_items, P.n_sgu_items);
       named_sync(1, kCThreads);
       if (tid == 0) arrive_release_gpu(p.sync + kSyncSharedH);
 
       // ---- softmax / top-K over every CTA's logits (the producer waits for it) ----
-      if (tid == 0 && !counter_wait(p.sync + kSyncLogits, (unsigned)(l + 1) * G1, &s_abort) && !s_abort) fail();
+      if (tid == 0 && !counter_wait(p.sync + kSyncLogits, (unsigned)(l + 1) * G1, &s_abort, budget) && !s_abort) fail();
       named_sync(1, kCThreads);
       block_topk(p, l, s_topk, s_idx, s_w, &s_topk_ready);
 
@@ -727,7 +733,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     if (p.xnorm_out) {
       const int nseg = H / 16;
       float ss = 0.f;
-      if (tid == 0 && !counter_wait(p.sync + kSyncResid, (unsigned)p.n_layers * G1, &s_abort) && !s_abort) fail();
+      if (tid == 0 && !counter_wait(p.sync + kSyncResid, (unsigned)p.n_layers * G1, &s_abort, budget) && !s_abort) fail();
       named_sync(1, kCThreads);
       if (tid < nseg) {
         float v[16];

@@ -135,3 +135,43 @@ def test_ffn_and_combine_reject_bad_layers(moeq):
     assert L.moe_combine_residual(ctypes.byref(s), None, A, A, None, 1, A, None, 1e-6, None) == moeq.MOE_ERR_INVALID_ARG
     assert L.moe_get_device_error(None, None) == moeq.MOE_ERR_WORKSPACE
     assert L.moe_workspace_init(None, 0, None) == moeq.MOE_ERR_WORKSPACE
+
+
+def test_router_rejects_more_experts_than_the_selection_holds(moeq):
+    """The router's selection keeps 32 logits per lane of a warp: E > 1024
+    is refused on the host instead of silently never picking experts >= 1024."""
+    L = moeq.lib()
+    n = moeq.moe_workspace_bytes(1, 4, 4096, 1024, 2048)
+    assert L.moe_router_topk(A, A, 1, 4096, 2048, 4, 0, None, A, A, None, A, n, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_router_topk(A, A, 1, 4096, 1025, 4, 0, None, A, A, None, A, n, None) == moeq.MOE_ERR_UNSUPPORTED
+
+
+def test_rmsnorm_and_debug_hook_reject_bad_arguments(moeq):
+    L = moeq.lib()
+    assert L.moe_rmsnorm(None, None, 1, 4096, 1e-6, A, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(A, None, 1, 4096, 1e-6, None, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(A, None, 0, 4096, 1e-6, A, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(A, None, 1, 4096, -1.0, A, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_rmsnorm(A, None, 1, 4092, 1e-6, A, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_rmsnorm(M, None, 1, 4096, 1e-6, A, None) == moeq.MOE_ERR_ALIGN
+    assert L.moe_rmsnorm(A, M, 1, 4096, 1e-6, A, None) == moeq.MOE_ERR_ALIGN
+    assert L.moe_workspace_debug(None, 4096, 1000, 1, None) == moeq.MOE_ERR_WORKSPACE
+    assert L.moe_workspace_debug(A, 100, 1000, 1, None) == moeq.MOE_ERR_WORKSPACE
+    assert L.moe_workspace_debug(M, 4096, 1000, 1, None) == moeq.MOE_ERR_ALIGN
+    assert L.moe_workspace_debug(A, 4096, 1000, -1, None) == moeq.MOE_ERR_INVALID_ARG
+
+
+def test_static_call_checks_arguments_before_its_size(moeq):
+    """Every argument error of the static-scratch call returns before the
+    scratch-size test (and before anything is queued)."""
+    L = moeq.lib()
+    good = dict(H=4096, I=1024, E=512, K=4, group=64, bits_routed=4, bits_shared=4, experts=A, shared=A, router_w=A,
+                shared_gate_w=None)
+    s = moeq.moe_layer_q(**dict(good, K=9))
+    assert L.moe_expert_ffn_q_static(ctypes.byref(s), A, 1, A, A, None, None) == moeq.MOE_ERR_INVALID_ARG
+    s = moeq.moe_layer_q(**good)
+    assert L.moe_expert_ffn_q_static(ctypes.byref(s), None, 1, A, A, None, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_expert_ffn_q_static(ctypes.byref(s), M, 1, A, A, None, None) == moeq.MOE_ERR_ALIGN
+    # a batch too large for the scratch, with a bad pointer: the pointer is reported
+    assert L.moe_expert_ffn_q_static(ctypes.byref(s), M, 64, A, A, None, None) == moeq.MOE_ERR_ALIGN
+    assert L.moe_expert_ffn_q_static(ctypes.byref(s), A, 64, A, A, None, None) == moeq.MOE_ERR_WORKSPACE

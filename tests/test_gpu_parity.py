@@ -1,10 +1,10 @@
 """GPU parity: every call of libmoeq.so against the oracle, through the C ABI.
 
-Bars: packed bytes and router indices bit-exact (indices compared where the
-oracle's ranking is decided by more than twice the observed logit error, else
-checked to be the exact top-K of the GPU's own logits); router weights within
-1e-5; expert and layer outputs within max|err| <= 2e-3 * ||y_oracle||_inf;
-combine within 1e-6 relative.
+Bars: packed bytes and router indices bit-exact; router weights within 1e-5;
+expert and layer outputs within max|err| <= 2e-3 * ||y_oracle||_inf; combine
+within 1e-6 relative. Router tests run on tokens whose oracle ranking is
+decided by more than twice the a-priori fp32 error bound of the GPU logits
+(tests/harness.py::logit_bound); the indices are then compared exactly.
 """
 import numpy as np
 import pytest
@@ -176,8 +176,13 @@ def test_packed_arena_matches_generator(name, over):
 @pytest.mark.parametrize("name,B,renorm", [("tiny", 1, False), ("tiny", 3, True), ("layer4", 1, False),
                                            ("layer4", 5, True), ("layer4", 32, False)])
 def test_router_topk(name, B, renorm):
+    """Router indices bit-exact on every token: the tokens are the first ones
+    whose oracle ranking is decided by more than twice the a-priori fp32
+    error bound of the GPU logits (tokens with a near tie are skipped and
+    reported, never compared loosely)."""
     w, L = get_layer(name)
-    x = hz.x_device(w, 100, B)
+    toks, skipped = hz.decided_tokens(w, 0, B, 100, ref.router_logits)
+    x = hz.x_tokens_device(w, toks)
     ws = moeq.Workspace(B, w.K, w.H, w.I, w.E)
     idx = torch.empty((B, w.K), dtype=torch.int32, device="cuda")
     wt = torch.empty((B, w.K), dtype=torch.float32, device="cuda")
@@ -185,15 +190,15 @@ def test_router_topk(name, B, renorm):
     moeq.moe_router_topk(x, L.router_w, B, w.H, w.E, w.K, renorm, None, idx, wt, lg, ws.buf, ws.nbytes)
     torch.cuda.synchronize()
     wr = synth.router_host(w, 0)
-    xb = synth.x_host(w, 100, B)
-    exact = 0
-    for b in range(B):
-        rl = ref.router_logits(xb[b], wr)
-        tol = 1e-5 * float(np.abs(ref.bf16_to_f64(wr) * hz.bf16_to_f64(xb[b])[None, :]).sum(axis=1).max())
-        exact += hz.check_topk(idx[b].cpu().numpy(), lg[b].cpu().numpy(), rl, w.K, tol)
-        ri, rw = ref.topk(rl, w.K, renorm=renorm, forced=idx[b].cpu().numpy())
+    for b, t in enumerate(toks):
+        xb = synth.x_host(w, t)[0]
+        rl = ref.router_logits(xb, wr)
+        bound = hz.logit_bound(xb, wr)
+        assert (np.abs(lg[b].cpu().numpy() - rl) <= bound).all()
+        ri, rw = ref.topk(rl, w.K, renorm=renorm)
+        assert list(idx[b].cpu().numpy()) == list(ri), (t, idx[b].tolist(), list(ri))
         assert np.abs(wt[b].cpu().numpy() - rw).max() <= W_TOL
-    assert exact >= B - 1  # near ties are rare; never all of them
+    print("near-tie tokens skipped:", skipped)
 
 
 def test_router_forced_and_bad_index():
@@ -339,35 +344,42 @@ def test_combine_residual(with_gate, with_resid):
 
 # ---- A1..A6 whole layer -----------------------------------------------------------
 
-@pytest.mark.parametrize("name,B", [("tiny", 1), ("tiny", 4), ("layer4", 1), ("layer2", 1)])
+@pytest.mark.parametrize("name,B", [("tiny", 1), ("tiny", 4), ("layer4", 1), ("layer2", 1), ("layer4", 3)])
 def test_layer_end_to_end(name, B):
+    """The three per-token calls against the oracle layer: indices exact on
+    tokens whose ranking is decided (near-tie tokens are skipped, reported),
+    weights, every expert slot and the residual output within the bars."""
     w, L = get_layer(name)
-    x = hz.x_device(w, 500, B)
+    toks, skipped = hz.decided_tokens(w, 0, B, 500, ref.router_logits)
+    x = hz.x_tokens_device(w, toks)
     out = run_layer(w, L, x, eps=1e-6)
-    xb = synth.x_host(w, 500, B)
-    for b in range(B):
-        ro = oracle_token(w, 0, xb[b], eps=1e-6)
-        got_idx = out["idx"][b].cpu().numpy()
-        if list(got_idx) != list(ro["idx"]):  # a near tie: evaluate the oracle on the GPU's picks
-            hz.check_topk(got_idx, out["logits"][b].cpu().numpy(), ro["logits"], w.K, 1e-3)
-            ro = oracle_token(w, 0, xb[b], forced=got_idx, eps=1e-6)
+    for b, t in enumerate(toks):
+        ro = oracle_token(w, 0, synth.x_host(w, t)[0], eps=1e-6)
+        assert list(out["idx"][b].cpu().numpy()) == list(ro["idx"]), (t, out["idx"][b].tolist(), list(ro["idx"]))
         assert np.abs(out["w"][b].cpu().numpy() - ro["w"]).max() <= W_TOL
         yg = out["y"][b].cpu().numpy()
         for k in range(w.K + 1):
             assert hz.max_rel_err(yg[k], ro["y"][k]) <= FFN_TOL
         assert hz.max_rel_err(out["resid"][b].cpu().numpy(), ro["out"]) <= FFN_TOL
+    print("near-tie tokens skipped:", skipped)
 
 
 def test_batched_zipf_routing_layer():
+    """The batched workload (32 tokens, forced Zipf(1.1) picks, grouped per
+    expert): every token's weights, every expert slot of y and every
+    residual row against the oracle."""
     w, L = get_layer("batch32")
     routing = synth.zipf_routing(w.E, w.K, w.B, 1, w.zipf_s, w.seed)[0]
     x = hz.x_device(w, 900, w.B)
     out = run_layer(w, L, x, forced=routing)
     xb = synth.x_host(w, 900, w.B)
-    for b in range(0, w.B, 7):
+    yg = out["y"].cpu().numpy()
+    for b in range(w.B):
         ro = oracle_token(w, 0, xb[b], forced=routing[b])
         assert (out["idx"][b].cpu().numpy() == routing[b]).all()
         assert np.abs(out["w"][b].cpu().numpy() - ro["w"]).max() <= W_TOL
+        for k in range(w.K + 1):
+            assert hz.max_rel_err(yg[b, k], ro["y"][k]) <= FFN_TOL, (b, k)
         assert hz.max_rel_err(out["resid"][b].cpu().numpy(), ro["out"]) <= FFN_TOL
 
 
@@ -378,14 +390,41 @@ def test_batched_zipf_routing_layer():
 def test_ragged_and_edge_shapes(over, B):
     w = synth.WORKLOADS["tiny"].with_(**over)
     L = hz.build_layer(w, 2)
-    x = hz.x_device(w, 77, B)
+    toks, _ = hz.decided_tokens(w, 2, B, 77, ref.router_logits)
+    x = hz.x_tokens_device(w, toks)
     out = run_layer(w, L, x, eps=1e-6)
-    xb = synth.x_host(w, 77, B)
-    for b in range(B):
-        got_idx = out["idx"][b].cpu().numpy()
-        ro = oracle_token(w, 2, xb[b], forced=got_idx, eps=1e-6)
-        if w.K < w.E:
-            hz.check_topk(got_idx, out["logits"][b].cpu().numpy(), ro["logits"], w.K, 1e-3)
+    for b, t in enumerate(toks):
+        ro = oracle_token(w, 2, synth.x_host(w, t)[0], eps=1e-6)
+        assert list(out["idx"][b].cpu().numpy()) == list(ro["idx"])
+        assert np.abs(out["w"][b].cpu().numpy() - ro["w"]).max() <= W_TOL
         assert hz.max_rel_err(out["resid"][b].cpu().numpy(), ro["out"]) <= FFN_TOL
         for k in range(w.K + 1):
             assert hz.max_rel_err(out["y"][b, k].cpu().numpy(), ro["y"][k]) <= FFN_TOL
+
+
+# ---- standalone RMS norm -------------------------------------------------------
+
+@pytest.mark.parametrize("B,H,weighted", [(1, 4096, False), (3, 4096, True), (5, 264, True), (64, 512, False)])
+def test_rmsnorm(B, H, weighted):
+    """moe_rmsnorm against the oracle's weighted RMS norm: every output is the
+    oracle's bf16 value or its neighbour (the fp32 product may land on the
+    other side of a rounding boundary), and almost all are identical."""
+    rng = np.random.default_rng(B * 1000 + H)
+    r = (rng.normal(size=(B, H)) * rng.uniform(0.1, 30.0, size=(B, 1))).astype(np.float32)
+    wbits = None
+    if weighted:
+        wbits = (rng.normal(1.0, 0.3, size=H).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    rd = torch.from_numpy(r).cuda()
+    wd = torch.from_numpy(wbits.view(np.int16)).cuda() if weighted else None
+    xn = torch.empty((B, H), dtype=torch.bfloat16, device="cuda")
+    moeq.moe_rmsnorm(rd, wd, B, H, 1e-6, xn)
+    torch.cuda.synchronize()
+    got = hz.bf16_bits(xn).astype(np.int32)
+    same = 0
+    for b in range(B):
+        want = ref.rmsnorm_weighted_bf16(r[b].astype(np.float64), wbits, 1e-6).astype(np.int32)
+        sign_ok = ((got[b] ^ want) & 0x8000) == 0
+        assert (sign_ok | ((got[b] | want) & 0x7FFF == 0)).all()
+        assert (np.abs((got[b] & 0x7FFF) - (want & 0x7FFF)) <= 1).all(), b
+        same += int((got[b] == want).sum())
+    assert same >= 0.99 * B * H
