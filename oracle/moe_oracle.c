@@ -52,15 +52,17 @@ size_t moe_ref_expert_bytes(int H, int I, int bits, int group) {
 
 static int pack_args_ok(int rows, int cols, int bits, int group) {
   if (rows < 0 || cols <= 0) return 0;
-  if (bits != 2 && bits != 4) return 0;
+  if (bits < 2 || bits > 4) return 0;
   if (group <= 0 || cols % group != 0) return 0;
   if ((cols * bits) % 8 != 0) return 0;
   return 1;
 }
 
-/* Code q[r,c] goes to byte floor(c*bits/8) of row r's packed bytes, at bit
- * offset (c*bits) mod 8 (lowest bits first). The (scale, bias) of group g of
- * row r is the bf16 pair sb[2*(r*ng+g)], sb[2*(r*ng+g)+1]. */
+/* Code q[r,c] occupies bits c*bits .. c*bits + bits - 1 of row r's packed
+ * bytes, read as one little-endian bit string (bit k is bit k%8 of byte
+ * k/8), lowest code bit first; at 3 bits a code may straddle two bytes. The
+ * (scale, bias) of group g of row r is the bf16 pair sb[2*(r*ng+g)],
+ * sb[2*(r*ng+g)+1]. */
 int moe_ref_pack(const uint8_t* codes, const uint16_t* scale, const uint16_t* bias,
                  int rows, int cols, int bits, int group, uint8_t* packed, uint16_t* sb) {
   if (!codes || !scale || !bias || !packed || !sb) return 1;
@@ -69,11 +71,14 @@ int moe_ref_pack(const uint8_t* codes, const uint16_t* scale, const uint16_t* bi
   int ng = cols / group;
   memset(packed, 0, row_bytes * (size_t)rows);
   for (int r = 0; r < rows; ++r) {
+    uint8_t* row = packed + (size_t)r * row_bytes;
     for (int c = 0; c < cols; ++c) {
       unsigned q = codes[(size_t)r * cols + c];
       if (q >> bits) return 1;
-      size_t bitpos = (size_t)c * bits;
-      packed[(size_t)r * row_bytes + bitpos / 8] |= (uint8_t)(q << (bitpos % 8));
+      for (int i = 0; i < bits; ++i) {
+        size_t k = (size_t)c * bits + i;
+        if ((q >> i) & 1u) row[k / 8] |= (uint8_t)(1u << (k % 8));
+      }
     }
     for (int g = 0; g < ng; ++g) {
       size_t rg = (size_t)r * ng + g;
@@ -90,16 +95,74 @@ int moe_ref_unpack(const uint8_t* packed, const uint16_t* sb, int rows, int cols
   if (!pack_args_ok(rows, cols, bits, group)) return 1;
   size_t row_bytes = (size_t)cols * bits / 8;
   int ng = cols / group;
-  unsigned mask = (1u << bits) - 1u;
   for (int r = 0; r < rows; ++r) {
+    const uint8_t* row = packed + (size_t)r * row_bytes;
     for (int c = 0; c < cols; ++c) {
-      size_t bitpos = (size_t)c * bits;
-      codes[(size_t)r * cols + c] = (uint8_t)((packed[(size_t)r * row_bytes + bitpos / 8] >> (bitpos % 8)) & mask);
+      unsigned q = 0;
+      for (int i = 0; i < bits; ++i) {
+        size_t k = (size_t)c * bits + i;
+        q |= (unsigned)((row[k / 8] >> (k % 8)) & 1u) << i;
+      }
+      codes[(size_t)r * cols + c] = (uint8_t)q;
     }
     for (int g = 0; g < ng; ++g) {
       size_t rg = (size_t)r * ng + g;
       scale[rg] = sb[2 * rg];
       bias[rg] = sb[2 * rg + 1];
+    }
+  }
+  return 0;
+}
+
+/* ---- quantisation ------------------------------------------------------ */
+
+/* Min-max group-affine quantisation of fp32 weights into the pages' affine
+ * form w ~ q*scale + bias (Flash-MoE page, "Kernel dequant toi uu FMA"), at
+ * 2, 3 or 4 bits (3 bits: the size/quality point of the Autoresearch page,
+ * "Optimizaciones Efectivas"). Per (row, group of `group` inputs):
+ *   lo, hi = min and max of the group's weights;
+ *   scale  = bf16((hi - lo) / (2^bits - 1)),  bias = bf16(lo);
+ *   q      = clamp(rint((w - bias) / scale), 0, 2^bits - 1), or 0 when the
+ *            bf16 scale is 0.
+ * The codes are integers decided by floating point, so they are decided in
+ * the precision of the GPU kernel: binary32 with one rounding to nearest
+ * even per operation (hi - lo, the division, w - bias, the quotient) and
+ * rint ties to even; bf16 narrowing is to nearest even. Returns 0, or 1 on
+ * bad arguments or a non-finite weight. */
+int moe_ref_quantize(const float* w, int rows, int cols, int bits, int group,
+                     uint8_t* codes, uint16_t* scale, uint16_t* bias) {
+  if (!w || !codes || !scale || !bias) return 1;
+  if (!pack_args_ok(rows, cols, bits, group)) return 1;
+  int ng = cols / group;
+  float levels = (float)((1 << bits) - 1);
+  for (int r = 0; r < rows; ++r) {
+    for (int g = 0; g < ng; ++g) {
+      const float* wg = w + (size_t)r * cols + (size_t)g * group;
+      float lo = wg[0], hi = wg[0];
+      for (int j = 0; j < group; ++j) {
+        if (!isfinite(wg[j])) return 1;
+        if (wg[j] < lo) lo = wg[j];
+        if (wg[j] > hi) hi = wg[j];
+      }
+      float range = hi - lo;
+      float s32 = range / levels;
+      uint16_t sbits = moe_ref_f64_to_bf16((double)s32);
+      uint16_t bbits = moe_ref_f64_to_bf16((double)lo);
+      float sf = (float)moe_ref_bf16_to_f64(sbits);
+      float bf = (float)moe_ref_bf16_to_f64(bbits);
+      size_t rg = (size_t)r * ng + g;
+      scale[rg] = sbits;
+      bias[rg] = bbits;
+      for (int j = 0; j < group; ++j) {
+        int q = 0;
+        if (sf != 0.0f) {
+          float d = wg[j] - bf;
+          float t = d / sf;
+          float qr = rintf(t);
+          q = qr < 0.0f ? 0 : (qr > levels ? (int)levels : (int)qr);
+        }
+        codes[(size_t)r * cols + (size_t)g * group + j] = (uint8_t)q;
+      }
     }
   }
   return 0;

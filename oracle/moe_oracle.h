@@ -22,8 +22,12 @@
  *         storage (each expert's data kept contiguous).
  *
  * Readings taken where the pages are silent:
- *  - q is unsigned (0..2^b-1); w = q*scale + bias per group of G consecutive
- *    input elements; scale and bias are bf16.
+ *  - q is unsigned (0..2^b-1), b in {2, 3, 4}; w = q*scale + bias per group
+ *    of G consecutive input elements; scale and bias are bf16.
+ *  - quantisation (weights -> codes) is min-max per group: bias = the
+ *    group's minimum, scale = its range / (2^b - 1), codes rounded to
+ *    nearest; 3 bits as the Autoresearch page's size/quality point
+ *    ("Autoresearch impulsa ... 20.34 tok/s", "Optimizaciones Efectivas").
  *  - packing is row-major, low bits first; the (scale, bias) pair of each
  *    (row, group) is stored interleaved, scale first.
  *  - an expert record is gate [I,H], up [I,H], down [H,I] packed codes, then
@@ -58,12 +62,19 @@ uint16_t moe_ref_f64_to_bf16(double v);
 /* bytes of one packed expert record (gate, up, down codes + their tables) */
 size_t moe_ref_expert_bytes(int H, int I, int bits, int group);
 
-/* packing of one [rows, cols] code matrix; returns 0, or 1 on bad arguments
- * or a code that does not fit in `bits` bits */
+/* packing of one [rows, cols] code matrix at bits in {2, 3, 4}; returns 0,
+ * or 1 on bad arguments or a code that does not fit in `bits` bits */
 int moe_ref_pack(const uint8_t* codes, const uint16_t* scale, const uint16_t* bias,
                  int rows, int cols, int bits, int group, uint8_t* packed, uint16_t* sb);
 int moe_ref_unpack(const uint8_t* packed, const uint16_t* sb, int rows, int cols, int bits,
                    int group, uint8_t* codes, uint16_t* scale, uint16_t* bias);
+
+/* min-max group-affine quantisation of fp32 weights [rows, cols] into codes
+ * u8 [rows, cols] and bf16 scale/bias [rows, cols/group]; the codes are
+ * decided in binary32 like the GPU kernel (see moe_oracle.c); 0, or 1 on bad
+ * arguments or a non-finite weight */
+int moe_ref_quantize(const float* w, int rows, int cols, int bits, int group,
+                     uint8_t* codes, uint16_t* scale, uint16_t* bias);
 
 /* y[r] = sum_c (q[r,c]*s[r,g(c)] + b[r,g(c)]) * x[c], three written-out forms */
 void moe_ref_dequant_gemv(const uint8_t* codes, const uint16_t* scale, const uint16_t* bias,

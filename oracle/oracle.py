@@ -56,6 +56,9 @@ def lib():
                                    ctypes.c_int, _u8p, _u16p]
         L.moe_ref_unpack.argtypes = [_u8p, _u16p, ctypes.c_int, ctypes.c_int, ctypes.c_int, ctypes.c_int,
                                      _u8p, _u16p, _u16p]
+        L.moe_ref_quantize.restype = ctypes.c_int
+        L.moe_ref_quantize.argtypes = [ctypes.POINTER(ctypes.c_float), ctypes.c_int, ctypes.c_int, ctypes.c_int,
+                                       ctypes.c_int, _u8p, _u16p, _u16p]
         for name in ("moe_ref_dequant_gemv", "moe_ref_dequant_gemv_fma", "moe_ref_dequant_gemv_grouped"):
             f = getattr(L, name)
             f.restype = None
@@ -142,6 +145,21 @@ def unpack(packed, sb, rows: int, cols: int, bits: int, group: int):
                               _p(codes, _u8p), _p(scale, _u16p), _p(bias, _u16p))
     if rc != 0:
         raise ValueError("moe_ref_unpack rejected its arguments")
+    return codes, scale, bias
+
+
+def quantize(w, bits: int, group: int):
+    """fp32 weights [rows, cols] -> (codes u8 [rows, cols], scale bf16 bits
+    [rows, cols/group], bias bf16 bits [rows, cols/group]), min-max per group."""
+    w = _c(w, np.float32)
+    rows, cols = w.shape
+    codes = np.zeros((rows, cols), dtype=np.uint8)
+    scale = np.zeros((rows, cols // group), dtype=np.uint16)
+    bias = np.zeros((rows, cols // group), dtype=np.uint16)
+    rc = lib().moe_ref_quantize(w.ctypes.data_as(ctypes.POINTER(ctypes.c_float)), rows, cols, bits, group,
+                                _p(codes, _u8p), _p(scale, _u16p), _p(bias, _u16p))
+    if rc != 0:
+        raise ValueError("moe_ref_quantize rejected its arguments")
     return codes, scale, bias
 
 

@@ -94,10 +94,10 @@ def test_pack_golden_bytes(ref):
         assert sb.shape == (1, ng, 2)
         assert (sb[..., 0] == 0x3F80).all() and (sb[..., 1] == 0xBF80).all()  # scale first
         n += 1
-    assert n >= 4
+    assert n >= 6
 
 
-@pytest.mark.parametrize("bits,group", [(4, 32), (4, 64), (2, 32), (2, 64), (4, 128)])
+@pytest.mark.parametrize("bits,group", [(4, 32), (4, 64), (2, 32), (2, 64), (4, 128), (3, 64), (3, 128)])
 def test_pack_is_little_endian_bitstring(ref, bits, group):
     """Independent reading of the layout: a packed row is the row's codes
     written as one little-endian integer, sum_c q_c * 2^(c*bits)."""
@@ -110,7 +110,7 @@ def test_pack_is_little_endian_bitstring(ref, bits, group):
         assert (sb[r, :, 0] == scale[r]).all() and (sb[r, :, 1] == bias[r]).all()
 
 
-@pytest.mark.parametrize("bits,group", [(4, 32), (2, 64)])
+@pytest.mark.parametrize("bits,group", [(4, 32), (2, 64), (3, 64)])
 def test_pack_roundtrip_and_range(ref, bits, group):
     rng = np.random.default_rng(7)
     codes, scale, bias = _rand_layer(rng, 5, 128, bits, group)
@@ -120,6 +120,85 @@ def test_pack_roundtrip_and_range(ref, bits, group):
     codes[2, 3] = 1 << bits
     with pytest.raises(ValueError):
         ref.pack(codes, scale, bias, bits, group)
+
+
+# ---- quantisation (weights -> codes, scale, bias) -----------------------------
+
+def _bf16_round(v):
+    """float value of the nearest bf16 (ties to even), via _rne_bf16_bits."""
+    return float(_f64(np.array([_rne_bf16_bits(float(v))], np.uint16))[0])
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_quantize_constant_groups(ref, bits):
+    """A constant group has range 0: scale 0, bias = bf16(the constant),
+    every code 0."""
+    w = np.array([[0.3] * 64 + [-2.5] * 64], np.float32)
+    codes, scale, bias = ref.quantize(w, bits, 64)
+    assert (codes == 0).all() and (scale == 0).all()
+    assert [int(b) for b in bias[0]] == [_rne_bf16_bits(float(np.float32(0.3))), _rne_bf16_bits(-2.5)]
+
+
+@pytest.mark.parametrize("bits,group", [(2, 64), (3, 64), (4, 64), (3, 128)])
+def test_quantize_ramp_recovers_its_levels(ref, bits, group):
+    """A group whose values are the 2^bits evenly spaced levels lo + j*d
+    (bf16-exact, arithmetic exact in fp32) gets scale d, bias lo and code j
+    for level j, so dequantisation returns every input exactly."""
+    n = 1 << bits
+    lo, d = -1.0, 0.25
+    j = np.arange(group) % n
+    w = (lo + j * d).astype(np.float32)[None, :]
+    codes, scale, bias = ref.quantize(w, bits, group)
+    assert (codes[0] == j).all()
+    assert _f64(scale)[0, 0] == d and _f64(bias)[0, 0] == lo
+    assert (codes[0] * d + lo == w[0]).all()
+
+
+@pytest.mark.parametrize("bits", [2, 3, 4])
+def test_quantize_picks_the_nearest_level(ref, bits):
+    """Brute force: each code is the nearest of the 2^bits levels bias + q*scale
+    of its group (exact fp64 distances; inputs within 1e-4 of a midpoint
+    between levels are left out, since the rounding of the kernel's binary32
+    quotient decides those), and the round-trip error stays within half a
+    scale step plus the bf16 rounding of scale and bias."""
+    rng = np.random.default_rng(bits)
+    G = 64
+    w = (rng.normal(size=(6, 256)) * rng.uniform(0.01, 3.0, size=(6, 1))).astype(np.float32)
+    # groups far from zero for their range: bf16(bias) misses the minimum by
+    # up to a quarter, so codes clamp at the top or the bottom
+    far = (rng.choice([-1.0, 1.0], size=(4, 1)) * rng.uniform(90.0, 120.0, size=(4, 1)) +
+           rng.uniform(0.0, 1.0, size=(4, 256))).astype(np.float32)
+    w = np.concatenate([w, far])
+    codes, scale, bias = ref.quantize(w, bits, G)
+    n = (1 << bits) - 1
+    checked = 0
+    for r in range(w.shape[0]):
+        for g in range(w.shape[1] // G):
+            wg = w[r, g * G:(g + 1) * G].astype(np.float64)
+            lo, hi = wg.min(), wg.max()
+            s_exact = (hi - lo) / n
+            sh = _f64(scale[r, g])
+            bh = _f64(bias[r, g])
+            assert sh == _bf16_round(np.float32(np.float32(hi - lo) / np.float32(n)))
+            assert bh == _bf16_round(lo)
+            levels = bh + sh * np.arange(n + 1)
+            for jj, v in enumerate(wg):
+                q = int(codes[r, g * G + jj])
+                t = (v - bh) / sh
+                if abs(t - np.floor(t) - 0.5) < 1e-4:
+                    continue
+                assert q == int(np.argmin(np.abs(levels - v))), (r, g, jj)
+                checked += 1
+            err = np.abs(wg - (codes[r, g * G:(g + 1) * G] * sh + bh)).max()
+            assert err <= sh / 2 + abs(bh - lo) + n * abs(sh - s_exact) + 1e-6 * max(abs(lo), abs(hi))
+    assert checked >= 0.99 * w.size
+
+
+def test_quantize_rejects_non_finite(ref):
+    w = np.zeros((1, 64), np.float32)
+    w[0, 5] = np.nan
+    with pytest.raises(ValueError):
+        ref.quantize(w, 4, 64)
 
 
 # ---- dequant mat-vec --------------------------------------------------------
