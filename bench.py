@@ -608,7 +608,8 @@ def run_ours(args, w, rank: int, world: int, local_rank: int):
                      "layers_per_launch": nlayers, "bytes_per_layer": step_bytes,
                      "bytes_per_launch": bytes_per_launch, "avg_launch_us": avg_launch_us,
                      "launches_timed": launches, "peak_source": peak_src,
-                     "launch_distribution_us": {k: v * 1e3 if k.endswith("_ms") else v for k, v in dd.items()}},
+                     "launch_distribution_us": {k.replace("_ms", "_us"): v * 1e3 if k.endswith("_ms") else v
+                                                for k, v in dd.items()}},
         "per_call": {"value": 1.0 / (pc["median_ms"] / 1e3), "unit": "layer-tokens/s",
                      "path": "moe_router_topk + moe_expert_ffn_q + moe_combine_residual, one graph per layer",
                      "timing": pc, "ffn_call_us": ffn_mean * 1e3,

@@ -75,7 +75,7 @@ typedef enum moe_status {
  * One MoE layer's resident weights (all pointers are device memory).
  *
  * Expert record (expert-major: each expert is one contiguous block, as in
- * LOOM's layout), for `bits` in {2, 4} and group size `group`; the
+ * LOOM's layout), for `bits` in {2, 3, 4} and group size `group`; the
  * dequantised weight is w = q*scale + bias with q unsigned and one bf16
  * (scale, bias) pair per row and group of `group` inputs. Every matrix is
  * stored as tiles of 16 rows laid out for the int8 tensor-core dot: a tile
@@ -85,7 +85,12 @@ typedef enum moe_status {
  *          g*group + 32j + 8t .. +7 of local rows r and r+8: at 4 bits two
  *          words, input 8t+i at nibble i; at 2 bits one word, input 8t+2i of
  *          row r at bits 8i, of row r+8 at 8i+2, input 8t+2i+1 of row r at
- *          8i+4, of row r+8 at 8i+6
+ *          8i+4, of row r+8 at 8i+6. At 3 bits (group 64 or 128) the low two
+ *          bits of every code form such a 2-bit plane (4 bytes per lane and
+ *          k-step), followed by a plane of the third bits (2 bytes per lane
+ *          and k-step, lane L at byte 128*(group/32) + 2*L*(group/32)): in
+ *          the word of k-steps 2p and 2p+1, bit 8i + 4*(j & 1) + s holds the
+ *          third bit of the code at bit 8i + 2s of k-step j's 2-bit word
  *   tables: 8 x [(scale, bias) of local row r][(scale, bias) of row r+8]
  * The record is I/8 gate/up tiles of H inputs (tile T: gate rows 8T..8T+7
  * as local rows 0..7, up rows 8T..8T+7 as 8..15), then H/16 down tiles of I
@@ -100,8 +105,8 @@ typedef struct moe_layer_q {
   int E;           /* routed experts */
   int K;           /* routed experts per token, 1..MOEQ_MAX_K, K <= E */
   int group;       /* 32, 64 or 128; divides H and I */
-  int bits_routed; /* 2 or 4 */
-  int bits_shared; /* 2 or 4 */
+  int bits_routed; /* 2, 3 or 4 (3: group 64 or 128) */
+  int bits_shared; /* 2, 3 or 4 */
   const void* experts;       /* E routed records, back to back */
   const void* shared;        /* 1 shared-expert record (bits_shared) */
   const void* router_w;      /* bf16 [E, H], row-major */
@@ -155,14 +160,38 @@ moe_status moe_workspace_debug(void* ws, size_t ws_bytes, unsigned wait_budget_u
  *   sb_out     bf16 [rows, cols/group, 2]  (scale, bias) pairs
  *   ws         optional workspace (NULL allowed): a code >= 2^bits sets
  *              MOE_ERR_RANGE there; its low `bits` bits are packed.
- * bits in {2,4}; group in {32,64,128}; cols % group == 0; cols*bits/8 a
- * multiple of 16. The layout is the affine form of the Flash-MoE page
+ * bits in {2,3,4} (a 3-bit code may straddle two bytes); group in
+ * {32,64,128}; cols % group == 0; cols*bits/8 a multiple of 16 (at 3 bits:
+ * cols % 128 == 0). The layout is the affine form of the Flash-MoE page
  * ("Kernel dequant toi uu FMA": (nibble*scale+bias)), 4- and 2-bit widths as
- * in its "Metal Compute Shaders" section.
+ * in its "Metal Compute Shaders" section, 3 bits as on the Autoresearch page
+ * ("Optimizaciones Efectivas").
  */
 moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* bias_bf16,
                       int rows, int cols, int bits, int group,
                       void* packed_out, void* sb_out, void* ws, void* stream);
+
+/*
+ * moe_quantize -- min-max group-affine quantisation of a weight matrix into
+ * the codes and (scale, bias) that moe_pack_q and moe_pack_expert take: the
+ * affine form w ~ q*scale + bias of the Flash-MoE page ("Kernel dequant toi
+ * uu FMA"), at 2, 3 or 4 bits (3 bits: the size/quality point of the
+ * Autoresearch page, "Optimizaciones Efectivas").
+ *   w          weights [rows, cols]: fp32 (in_bf16 = 0) or bf16 (in_bf16 = 1)
+ *   codes_out  u8 [rows, cols], one code per byte
+ *   scale_bf16_out, bias_bf16_out  bf16 [rows, cols/group]
+ *   ws         optional workspace (NULL allowed): a non-finite weight sets
+ *              MOE_ERR_RANGE there and its group is written as zeros
+ * Per (row, group of `group` inputs): lo, hi = the group's extreme weights;
+ * scale = bf16((hi - lo) / (2^bits - 1)), bias = bf16(lo) (nearest even);
+ * q = clamp(rint((w - bias) / scale), 0, 2^bits - 1), or 0 when the bf16
+ * scale is 0. Each step is one binary32 operation rounded to nearest even,
+ * so the codes are reproducible bit for bit. bits in {2,3,4}; group in
+ * {32,64,128} dividing cols (the record of 3-bit experts needs group 64 or
+ * 128). MOE_ERR_UNSUPPORTED / MOE_ERR_INVALID_ARG / MOE_ERR_ALIGN otherwise.
+ */
+moe_status moe_quantize(const void* w, int in_bf16, int rows, int cols, int bits, int group, uint8_t* codes_out,
+                        void* scale_bf16_out, void* bias_bf16_out, void* ws, void* stream);
 
 /*
  * moe_pack_expert -- pack the gate [I,H], up [I,H] and down [H,I] code

@@ -53,6 +53,7 @@ _SIGS = {
     "moe_rmsnorm": (_INT, [_VP, _VP, _INT, _INT, _FLT, _VP, _VP]),
     "moe_pack_q": (_INT, [_VP, _VP, _VP, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP]),
     "moe_pack_expert": (_INT, [_VP] * 9 + [_INT, _INT, _INT, _INT, _VP, _VP, _VP]),
+    "moe_quantize": (_INT, [_VP, _INT, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP, _VP]),
     "moe_router_topk": (_INT, [_VP, _VP, _INT, _INT, _INT, _INT, _INT, _VP, _VP, _VP, _VP, _VP, _SZ, _VP]),
     "moe_expert_ffn_q": (_INT, [_LP, _VP, _INT, _VP, _VP, _VP, _SZ, _VP]),
     "moe_combine_residual": (_INT, [_LP, _VP, _VP, _VP, _VP, _INT, _VP, _VP, _FLT, _VP]),
@@ -141,6 +142,12 @@ def moe_pack_q(codes, scale_bf16, bias_bf16, rows: int, cols: int, bits: int, gr
                ws=None, stream=None) -> None:
     _check(lib().moe_pack_q(_ptr(codes), _ptr(scale_bf16), _ptr(bias_bf16), rows, cols, bits, group,
                             _ptr(packed_out), _ptr(sb_out), _ptr(ws), _stream(stream)), "moe_pack_q")
+
+
+def moe_quantize(w, in_bf16: bool, rows: int, cols: int, bits: int, group: int, codes_out, scale_out, bias_out,
+                 ws=None, stream=None) -> None:
+    _check(lib().moe_quantize(_ptr(w), int(bool(in_bf16)), rows, cols, bits, group, _ptr(codes_out), _ptr(scale_out),
+                              _ptr(bias_out), _ptr(ws), _stream(stream)), "moe_quantize")
 
 
 def moe_pack_expert(gate, up, down, H: int, I: int, bits: int, group: int, record_out, ws=None, stream=None) -> None:

@@ -40,7 +40,9 @@ __device__ __forceinline__ uint16_t f32_to_bf16_bits(float f) {
 // Geometry of one expert record (bytes). Every matrix is stored as tiles of
 // 16 rows laid out for the int8 tensor-core dot (mma m16n8k32 fragments):
 // tile T holds, for each group of G inputs, one block of
-//   codes  32 lanes x (G/32 k-steps) x W bytes (W = 8 at 4 bits, 4 at 2 bits)
+//   codes  32 lanes x (G/32 k-steps) x W bytes (W = 8 at 4 bits, 4 at 2 bits;
+//          3 bits: a 2-bit plane of 4 bytes per lane and k-step, then a
+//          1-bit plane of 2 bytes per lane and k-step)
 //   table  8 x [(scale, bias) of local row g, (scale, bias) of local row g+8]
 // Gate/up tile T (at T*U, I/8 tiles of H inputs) holds gate rows 8T..8T+7 as
 // local rows 0..7 and up rows 8T..8T+7 as local rows 8..15; down tile T (at
@@ -53,7 +55,7 @@ struct RecGeom {
   unsigned long long down_off;
 };
 __host__ __device__ inline uint32_t tile_block_bytes(int bits, int group) {
-  return (uint32_t)(group * (bits == 4 ? 8 : 4) + 64);
+  return (uint32_t)(2 * group * bits + 64);  // 16 rows x group codes of `bits` bits, then the tables
 }
 __host__ __device__ inline RecGeom rec_geom(int H, int I, int bits, int group) {
   RecGeom g;

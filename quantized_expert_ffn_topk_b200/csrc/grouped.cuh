@@ -152,6 +152,27 @@ __global__ void __launch_bounds__(256) k_stage_batch(const void* src, int is_h, 
 
 // ---- the multi-token tile dot ---------------------------------------------
 
+// NB bytes of code words from global memory, streaming (read once).
+template <int NB>
+__device__ __forceinline__ void ld_stream_words(const unsigned char* p, uint32_t* w) {
+  if (NB >= 16) {
+#pragma unroll
+    for (int i = 0; i < NB / 16; ++i) {
+      const uint4 v = ld_stream16(p + 16 * i);
+      w[4 * i] = v.x;
+      w[4 * i + 1] = v.y;
+      w[4 * i + 2] = v.z;
+      w[4 * i + 3] = v.w;
+    }
+  } else if (NB == 8) {
+    const uint2 v = ld_stream8(p);
+    w[0] = v.x;
+    w[1] = v.y;
+  } else {
+    w[0] = ld_stream4(p);
+  }
+}
+
 // Blocks [0, nblk) of one tile in global memory against groups [g0, g0+nblk)
 // of up to four tokens' images (imgs[c], c < nt; the lanes of column pair c
 // read image c). Lane (gid, t) accumulates token t: acc0 for local row gid,
@@ -167,30 +188,15 @@ __device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int n
   const uint2* planes = reinterpret_cast<const uint2*>(imgs[gid >> 1]) + (gid & 1) * 4 + t;
   const float2* gs = reinterpret_cast<const float2*>(imgs[t] + gs_off);  // this lane's token
   for (int b0 = 0; b0 < nblk; b0 += P) {
-    uint32_t w[P][F::LB / 4];
+    uint32_t w[P][F::NW];
     uint2 sb[P], bf[P][KS];
     float2 ms[P];
 #pragma unroll
     for (int q = 0; q < P; ++q) {
       const int b = min(b0 + q, nblk - 1);
       const unsigned char* blk = blk0 + (size_t)b * F::BB;
-      const unsigned char* cp = blk + lane * F::LB;
-      if (F::LB >= 16) {
-#pragma unroll
-        for (int i = 0; i < F::LB / 16; ++i) {
-          const uint4 v = ld_stream16(cp + 16 * i);
-          w[q][4 * i] = v.x;
-          w[q][4 * i + 1] = v.y;
-          w[q][4 * i + 2] = v.z;
-          w[q][4 * i + 3] = v.w;
-        }
-      } else if (F::LB == 8) {
-        const uint2 v = ld_stream8(cp);
-        w[q][0] = v.x;
-        w[q][1] = v.y;
-      } else {
-        w[q][0] = ld_stream4(cp);
-      }
+      ld_stream_words<F::LB>(blk + lane * F::LB, w[q]);
+      if (BITS == 3) ld_stream_words<F::LH>(blk + 32 * F::LB + lane * F::LH, w[q] + F::LB / 4);
       sb[q] = ld_stream8(blk + F::CB + gid * 8);
       const int g = g0 + b;
 #pragma unroll
@@ -204,7 +210,7 @@ __device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int n
 #pragma unroll
       for (int ks = 0; ks < KS; ++ks) {
         uint32_t a[4];
-        extract_a<BITS>(w[q], ks, a);
+        extract_a<BITS, KS>(w[q], ks, a);
         mma_u8s8(d, a, bf[q][ks], ks > 0);
       }
       const float p0 = (float)(d[0] * 256 + d[1]) * ms[q].x;

@@ -19,7 +19,7 @@ namespace {
 
 inline bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
 
-inline bool bits_ok(int bits) { return bits == 2 || bits == 4; }
+inline bool bits_ok(int bits) { return bits >= 2 && bits <= 4; }
 inline bool group_ok(int g) { return g == 32 || g == 64 || g == 128; }
 
 // A row of `cols` codes must be whole 16-byte chunks and whole groups.
@@ -196,6 +196,7 @@ const char* moe_status_str(moe_status s) {
 
 size_t moe_expert_bytes(int H, int I, int bits, int group) {
   if (H <= 0 || I <= 0 || !bits_ok(bits) || !group_ok(group)) return 0;
+  if (bits == 3 && group < 64) return 0;  // a 3-bit block pairs k-steps: group 64 or 128
   if (!cols_ok(H, bits, group) || !cols_ok(I, bits, group)) return 0;
   if (H % kTileRows != 0 || I % 8 != 0) return 0;  // whole tiles of 16 rows
   const size_t hi = 3 * (size_t)H * I;
@@ -259,7 +260,7 @@ moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* 
     return MOE_ERR_ALIGN;
   if (rows == 0) return MOE_OK;
   cudaStream_t s = (cudaStream_t)stream;
-  const int64_t nchunks = (int64_t)rows * cols * bits / 128;
+  const int64_t nchunks = bits == 3 ? (int64_t)rows * cols / 128 : (int64_t)rows * cols * bits / 128;
   const int64_t nsb = (int64_t)rows * (cols / group);
   const unsigned maxg = (unsigned)num_sms() * 8;
   unsigned g1 = (unsigned)std::min<int64_t>((nchunks + 255) / 256, maxg);
@@ -271,10 +272,36 @@ moe_status moe_pack_q(const uint8_t* codes, const void* scale_bf16, const void* 
   const int cpr = (int)(rowb / 16);
   if (bits == 4)
     k_pack_codes<4><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
+  else if (bits == 3)
+    k_pack_codes3<<<g1, 256, 0, s>>>(codes, nchunks, cols / 128, pc, ctrl);
   else
     k_pack_codes<2><<<g1, 256, 0, s>>>(codes, nchunks, cpr, pc, ctrl);
   k_pack_sb<<<g2, 256, 0, s>>>(reinterpret_cast<const uint16_t*>(scale_bf16), reinterpret_cast<const uint16_t*>(bias_bf16),
                                nsb, cols / group, ps);
+  return launch_status();
+}
+
+moe_status moe_quantize(const void* w, int in_bf16, int rows, int cols, int bits, int group, uint8_t* codes_out,
+                        void* scale_bf16_out, void* bias_bf16_out, void* ws, void* stream) {
+  if (!w || !codes_out || !scale_bf16_out || !bias_bf16_out) return MOE_ERR_INVALID_ARG;
+  if (rows < 0 || cols <= 0 || (in_bf16 != 0 && in_bf16 != 1)) return MOE_ERR_INVALID_ARG;
+  if (!bits_ok(bits) || !group_ok(group) || cols % group != 0) return MOE_ERR_UNSUPPORTED;
+  if (!aligned16(w) || !aligned16(codes_out) || !aligned16(scale_bf16_out) || !aligned16(bias_bf16_out) ||
+      (ws && !aligned16(ws)))
+    return MOE_ERR_ALIGN;
+  if (rows == 0) return MOE_OK;
+  const int64_t ngroups = (int64_t)rows * (cols / group);
+  const unsigned grid = (unsigned)std::min<int64_t>((ngroups + 7) / 8, (int64_t)num_sms() * 16);
+  cudaStream_t s = (cudaStream_t)stream;
+  WsCtrl* ctrl = reinterpret_cast<WsCtrl*>(ws);
+  uint16_t* sc = reinterpret_cast<uint16_t*>(scale_bf16_out);
+  uint16_t* bi = reinterpret_cast<uint16_t*>(bias_bf16_out);
+  if (group == 32)
+    k_quantize<1><<<grid, 256, 0, s>>>(w, in_bf16, ngroups, cols / group, cols, bits, codes_out, sc, bi, ctrl);
+  else if (group == 64)
+    k_quantize<2><<<grid, 256, 0, s>>>(w, in_bf16, ngroups, cols / group, cols, bits, codes_out, sc, bi, ctrl);
+  else
+    k_quantize<4><<<grid, 256, 0, s>>>(w, in_bf16, ngroups, cols / group, cols, bits, codes_out, sc, bi, ctrl);
   return launch_status();
 }
 
@@ -297,12 +324,14 @@ moe_status moe_pack_expert(const uint8_t* codes_gate, const void* scale_gate_bf1
   const unsigned maxg = (unsigned)num_sms() * 8;
   auto u16 = [](const void* q) { return reinterpret_cast<const uint16_t*>(q); };
   auto launch = [&](const TileSrc& src, int ntiles, int C, unsigned char* dst, uint32_t tile_bytes) {
-    const int64_t ncode = (int64_t)ntiles * C;  // threads: (tile, group, lane, k-step)
+    const int64_t ncode = (int64_t)ntiles * C / (bits == 3 ? 2 : 1);  // threads: (tile, group, lane, k-step[s])
     const int64_t nsb = (int64_t)ntiles * (C / group) * 8;
     const unsigned g1 = (unsigned)std::min<int64_t>((ncode + 255) / 256, maxg);
     const unsigned g2 = (unsigned)std::min<int64_t>((nsb + 255) / 256, maxg);
     if (bits == 4)
       k_pack_tile_codes<4><<<g1, 256, 0, s>>>(src, ntiles, C, group, dst, tile_bytes, g.blk, ctrl);
+    else if (bits == 3)
+      k_pack_tile_codes3<<<g1, 256, 0, s>>>(src, ntiles, C, group, dst, tile_bytes, g.blk, ctrl);
     else
       k_pack_tile_codes<2><<<g1, 256, 0, s>>>(src, ntiles, C, group, dst, tile_bytes, g.blk, ctrl);
     k_pack_tile_sb<<<g2, 256, 0, s>>>(src, ntiles, C, group, dst, tile_bytes, g.blk, g.blk - 64);

@@ -156,17 +156,25 @@ __device__ __forceinline__ void mma_u8s8(int (&d)[4], const uint32_t (&a)[4], ui
   }
 }
 
-// Bytes of one lane's codes in one block, and of a block's codes.
+// Bytes of a block's code planes. 4 and 2 bits: one plane, LB bytes per lane
+// (lane L at L*LB). 3 bits: the low 2 bits of every code in the 2-bit layout
+// (4 bytes per lane and k-step, lane L at L*4*KS), then their third bits
+// (2 bytes per lane and k-step, lane L at 128*KS + L*2*KS); in the third-bit
+// word of k-steps 2p and 2p+1, bit 8i + 4*(ks & 1) + r is the third bit of
+// byte i of A register r.
 template <int BITS, int KS>
 struct TileFmt {
-  static constexpr int W = BITS == 4 ? 8 : 4;  // bytes per lane per k-step
-  static constexpr int LB = KS * W;            // bytes per lane per group
-  static constexpr int CB = 32 * LB;           // code bytes per block
-  static constexpr int BB = CB + 64;           // block bytes
+  static_assert(BITS != 3 || KS % 2 == 0, "3-bit blocks need an even number of k-steps (group >= 64)");
+  static constexpr int W = BITS == 4 ? 8 : 4;          // bytes per lane per k-step of the first plane
+  static constexpr int LB = KS * W;                     // first-plane bytes per lane
+  static constexpr int LH = BITS == 3 ? KS * 2 : 0;     // third-bit plane bytes per lane
+  static constexpr int NW = (LB + LH) / 4;              // code words per lane
+  static constexpr int CB = 32 * (LB + LH);             // code bytes per block
+  static constexpr int BB = CB + 64;                    // block bytes
 };
 
-// A fragments of k-step ks from the lane's words w.
-template <int BITS>
+// A fragments of k-step ks from the lane's words w (NW of them).
+template <int BITS, int KS>
 __device__ __forceinline__ void extract_a(const uint32_t* w, int ks, uint32_t (&a)[4]) {
   if (BITS == 4) {
     const uint32_t w0 = w[2 * ks], w1 = w[2 * ks + 1];
@@ -180,27 +188,42 @@ __device__ __forceinline__ void extract_a(const uint32_t* w, int ks, uint32_t (&
     a[1] = (w0 >> 2) & 0x03030303u;
     a[2] = (w0 >> 4) & 0x03030303u;
     a[3] = (w0 >> 6) & 0x03030303u;
+    if (BITS == 3) {
+      const uint32_t h = w[KS + (ks >> 1)] >> (4 * (ks & 1));
+      a[0] |= (h & 0x01010101u) << 2;
+      a[1] |= ((h >> 1) & 0x01010101u) << 2;
+      a[2] |= ((h >> 2) & 0x01010101u) << 2;
+      a[3] |= ((h >> 3) & 0x01010101u) << 2;
+    }
   }
 }
 
-template <int LB>
-__device__ __forceinline__ void load_lane_codes(const unsigned char* p, uint32_t (&w)[LB / 4]) {
-  if (LB >= 16) {
+template <int NB>
+__device__ __forceinline__ void load_words(const unsigned char* p, uint32_t* w) {
+  if (NB >= 16) {
 #pragma unroll
-    for (int i = 0; i < LB / 16; ++i) {
+    for (int i = 0; i < NB / 16; ++i) {
       const uint4 q = reinterpret_cast<const uint4*>(p)[i];
       w[4 * i] = q.x;
       w[4 * i + 1] = q.y;
       w[4 * i + 2] = q.z;
       w[4 * i + 3] = q.w;
     }
-  } else if (LB == 8) {
+  } else if (NB == 8) {
     const uint2 q = *reinterpret_cast<const uint2*>(p);
     w[0] = q.x;
     w[1] = q.y;
   } else {
     w[0] = *reinterpret_cast<const uint32_t*>(p);
   }
+}
+
+// The lane's code words of one block (shared or global memory, plain loads).
+template <int BITS, int KS>
+__device__ __forceinline__ void load_lane_codes(const unsigned char* blk, int lane, uint32_t (&w)[TileFmt<BITS, KS>::NW]) {
+  using F = TileFmt<BITS, KS>;
+  load_words<F::LB>(blk + lane * F::LB, w);
+  if (BITS == 3) load_words<F::LH>(blk + 32 * F::LB + lane * F::LH, w + F::LB / 4);
 }
 
 // One block (group g of a tile) from the lane's code words w and table pair
@@ -214,7 +237,7 @@ __device__ __forceinline__ void block_acc(const uint32_t* w, uint2 sb, int g, co
 #pragma unroll
   for (int ks = 0; ks < KS; ++ks) {
     uint32_t a[4];
-    extract_a<BITS>(w, ks, a);
+    extract_a<BITS, KS>(w, ks, a);
     mma_u8s8(d, a, planes[(size_t)(g * KS + ks) * 8], ks > 0);
   }
   const float2 ms = X.gs[g];
@@ -237,20 +260,24 @@ __device__ __forceinline__ void tile_dot(const unsigned char* blk0, int nblk, in
 #pragma unroll 2
   for (int b = 0; b < nblk; ++b) {
     const unsigned char* blk = blk0 + (size_t)b * F::BB;
-    uint32_t w[F::LB / 4];
-    load_lane_codes<F::LB>(blk + lane * F::LB, w);
+    uint32_t w[F::NW];
+    load_lane_codes<BITS, KS>(blk, lane, w);
     const uint2 sb = *reinterpret_cast<const uint2*>(blk + F::CB + (lane >> 2) * 8);
     block_acc<BITS, KS>(w, sb, g0 + b, X, acc0, acc1);
   }
 }
 
-// Dispatch on (bits, group) for callers with runtime values.
+// Dispatch on (bits, group) for callers with runtime values (3 bits: group
+// 64 or 128 only; the host rejects 3-bit group 32).
 template <typename Fn>
 __device__ __forceinline__ void with_fmt(int bits, int G, Fn fn) {
   if (bits == 4) {
     if (G == 32) fn.template operator()<4, 1>();
     else if (G == 64) fn.template operator()<4, 2>();
     else fn.template operator()<4, 4>();
+  } else if (bits == 3) {
+    if (G == 64) fn.template operator()<3, 2>();
+    else if (G == 128) fn.template operator()<3, 4>();
   } else {
     if (G == 32) fn.template operator()<2, 1>();
     else if (G == 64) fn.template operator()<2, 2>();

@@ -16,6 +16,7 @@ Workload recipes (all seed 0):
 ``tiny``      H=256, E=8, I=128, top-2 + 1 shared, 4-bit, group 32
 ``layer4``    H=4096, E=512, I=1024, top-4 + 1 shared, 4-bit, group 64
 ``layer2``    as ``layer4`` with 2-bit routed experts (shared stays 4-bit)
+``layer3``    as ``layer4`` with 3-bit routed experts (shared stays 4-bit)
 ``stack24``   24 ``layer4`` layers, 256 sequential tokens, forced routing
               with 27 % per-layer overlap between consecutive tokens
 ``batch32``   ``layer4`` with 32 tokens per step, forced Zipf(1.1) routing
@@ -145,6 +146,7 @@ WORKLOADS = {
     "tiny": Workload("tiny", H=256, E=8, I=128, K=2, group=32),
     "layer4": Workload("layer4", H=4096, E=512, I=1024, K=4, group=64),
     "layer2": Workload("layer2", H=4096, E=512, I=1024, K=4, group=64, bits_routed=2),
+    "layer3": Workload("layer3", H=4096, E=512, I=1024, K=4, group=64, bits_routed=3),
     "stack24": Workload("stack24", H=4096, E=512, I=1024, K=4, group=64, layers=24, tokens=256,
                         routing="overlap"),
     "batch32": Workload("batch32", H=4096, E=512, I=1024, K=4, group=64, B=32, routing="zipf"),

@@ -53,7 +53,10 @@ def test_record_sizes_agree_with_oracle(moeq, ref):
     # 16-row tiles; one block per group: 32 lanes x 2 k-steps x 8 bytes + 8 x 8 bytes of tables
     assert lay == [64 * 576, 128 * 64 * 576, 16 * 576, 16, 576, 128]
     assert lay[1] + (4096 // 16) * lay[2] == 7077888
-    assert moeq.moe_expert_bytes(4096, 1024, 3, 64) == 0
+    assert moeq.moe_expert_bytes(4096, 1024, 3, 64) == ref.expert_bytes(4096, 1024, 3, 64) == 5505024
+    assert moeq.moe_expert_bytes(4096, 1024, 3, 32) == 0  # a 3-bit block pairs k-steps: group >= 64
+    assert moeq.moe_expert_layout(4096, 1024, 3, 64)[4] == 32 * 12 + 64
+    assert moeq.moe_expert_bytes(4096, 1024, 5, 64) == 0
     assert moeq.moe_expert_bytes(4096, 1000, 4, 64) == 0
     assert moeq.moe_expert_bytes(384, 128, 2, 128) == ref.expert_bytes(384, 128, 2, 128)  # odd H/group is fine
 
@@ -74,14 +77,16 @@ def test_pack_expert_rejects_bad_arguments(moeq):
     good = [A] * 9
     assert L.moe_pack_expert(*([None] + good[1:]), 4096, 1024, 4, 64, A, None, None) == moeq.MOE_ERR_INVALID_ARG
     assert L.moe_pack_expert(*good, 4096, 1024, 4, 64, None, None, None) == moeq.MOE_ERR_INVALID_ARG
-    assert L.moe_pack_expert(*good, 4096, 1024, 3, 64, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_pack_expert(*good, 4096, 1024, 5, 64, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_pack_expert(*good, 4096, 1024, 3, 32, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
     assert L.moe_pack_expert(*(good[:4] + [M] + good[5:]), 4096, 1024, 4, 64, A, None, None) == moeq.MOE_ERR_ALIGN
 
 
 def test_pack_rejects_bad_arguments(moeq):
     L = moeq.lib()
     assert L.moe_pack_q(None, A, A, 4, 64, 4, 32, A, A, None, None) == moeq.MOE_ERR_INVALID_ARG
-    assert L.moe_pack_q(A, A, A, 4, 64, 3, 32, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_pack_q(A, A, A, 4, 64, 5, 32, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_pack_q(A, A, A, 4, 64, 3, 32, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED  # 24-byte rows
     assert L.moe_pack_q(A, A, A, 4, 64, 4, 48, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
     assert L.moe_pack_q(A, A, A, 4, 48, 4, 16, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
     assert L.moe_pack_q(A, A, A, 4, 96, 2, 32, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED  # 24-byte rows
@@ -119,7 +124,8 @@ def test_ffn_and_combine_reject_bad_layers(moeq):
     def ffn(**kw):
         s = moeq.moe_layer_q(**dict(good, **kw))
         return L.moe_expert_ffn_q(ctypes.byref(s), A, 1, A, A, A, n, None)
-    assert ffn(bits_routed=3) == moeq.MOE_ERR_UNSUPPORTED
+    assert ffn(bits_routed=5) == moeq.MOE_ERR_UNSUPPORTED
+    assert ffn(bits_routed=3, group=32) == moeq.MOE_ERR_UNSUPPORTED
     assert ffn(group=16) == moeq.MOE_ERR_UNSUPPORTED
     assert ffn(I=1000) == moeq.MOE_ERR_UNSUPPORTED
     assert ffn(K=0) == moeq.MOE_ERR_INVALID_ARG
@@ -175,3 +181,15 @@ def test_static_call_checks_arguments_before_its_size(moeq):
     # a batch too large for the scratch, with a bad pointer: the pointer is reported
     assert L.moe_expert_ffn_q_static(ctypes.byref(s), M, 64, A, A, None, None) == moeq.MOE_ERR_ALIGN
     assert L.moe_expert_ffn_q_static(ctypes.byref(s), A, 64, A, A, None, None) == moeq.MOE_ERR_WORKSPACE
+
+
+def test_quantize_rejects_bad_arguments(moeq):
+    L = moeq.lib()
+    assert L.moe_quantize(None, 0, 4, 64, 4, 64, A, A, A, None, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize(A, 2, 4, 64, 4, 64, A, A, A, None, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize(A, 0, -1, 64, 4, 64, A, A, A, None, None) == moeq.MOE_ERR_INVALID_ARG
+    assert L.moe_quantize(A, 0, 4, 64, 5, 64, A, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_quantize(A, 0, 4, 96, 4, 64, A, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_quantize(A, 0, 4, 64, 4, 48, A, A, A, None, None) == moeq.MOE_ERR_UNSUPPORTED
+    assert L.moe_quantize(M, 0, 4, 64, 4, 64, A, A, A, None, None) == moeq.MOE_ERR_ALIGN
+    assert L.moe_quantize(A, 0, 0, 64, 4, 64, A, A, A, None, None) == moeq.MOE_OK  # nothing to do

@@ -66,7 +66,7 @@ def oracle_chain(w, n, x_bits, forced=None):
     return res
 
 
-@pytest.mark.parametrize("name", ["tiny", "layer4", "layer2"])
+@pytest.mark.parametrize("name", ["tiny", "layer4", "layer2", "layer3"])
 def test_one_layer_matches_oracle(name):
     w, Ls = layers_for(name, 1)
     toks, skipped = hz.decided_tokens(w, 0, 1, 321, ref.router_logits)

@@ -78,7 +78,9 @@ def test_device_generator_matches_host():
 # ---- A0 pack: byte-exact -----------------------------------------------------
 
 @pytest.mark.parametrize("rows,cols,bits,group", [(1, 32, 4, 32), (5, 64, 2, 32), (37, 320, 4, 64), (129, 256, 2, 64),
-                                                  (3, 512, 4, 128), (1024, 4096, 4, 64), (4096, 1024, 2, 64)])
+                                                  (3, 512, 4, 128), (1024, 4096, 4, 64), (4096, 1024, 2, 64),
+                                                  (5, 128, 3, 64), (3, 384, 3, 128), (7, 256, 3, 32),
+                                                  (1024, 4096, 3, 64)])
 def test_pack_byte_exact(rows, cols, bits, group):
     rng = np.random.default_rng(rows * 7 + cols + bits)
     codes = rng.integers(0, 1 << bits, size=(rows, cols), dtype=np.uint8)
@@ -119,7 +121,7 @@ def decode_tiles(region, ntiles, C, bits, group):
     holds inputs 32j + 8t .. 32j + 8t + 7 of the group for local rows g and
     g + 8."""
     ks, ng = group // 32, C // group
-    wb = 8 if bits == 4 else 4
+    wb = {4: 8, 3: 6, 2: 4}[bits]
     cb = 32 * ks * wb
     blk = region[:ntiles * ng * (cb + 64)].reshape(ntiles, ng, cb + 64)
     words = np.ascontiguousarray(blk[:, :, :cb]).view("<u4")
@@ -128,6 +130,17 @@ def decode_tiles(region, ntiles, C, bits, group):
         w = words.reshape(ntiles, ng, 8, 4, ks, 2)
         v = (w[..., None] >> (4 * np.arange(8, dtype=np.uint32))) & 0xF      # [T, g, gid, t, j, h, i]
         v = v.transpose(0, 5, 2, 1, 4, 3, 6)                                   # [T, h, gid, g, j, t, i]
+    elif bits == 3:
+        # a 2-bit plane (bits 8i + 2s, s = 2*odd + h, of k-step j's word), then
+        # the third bits (bit 8i + 4*(j & 1) + s of word j // 2)
+        lo = words[:, :, :32 * ks].reshape(ntiles, ng, 8, 4, ks)
+        hw = words[:, :, 32 * ks:].reshape(ntiles, ng, 8, 4, ks // 2)
+        hj = np.repeat(hw, 2, axis=-1) >> (4 * (np.arange(ks, dtype=np.uint32) % 2))  # [T, g, gid, t, j]
+        sh = 2 * np.arange(16, dtype=np.uint32)                                         # 8i + 2s for the 16 (i, s)
+        lo2 = (lo[..., None] >> sh) & 0x3
+        hi1 = (hj[..., None] >> (sh // 2 + 4 * (sh // 8))) & 0x1  # 8i + s from 8i + 2s
+        v = (lo2 | (hi1 << 2)).reshape(ntiles, ng, 8, 4, ks, 4, 2, 2)                   # [T, g, gid, t, j, i, odd, h]
+        v = v.transpose(0, 7, 2, 1, 4, 3, 5, 6)
     else:
         # one word: bits 8i + 4*odd + 2h hold input 8t + 2i + odd of local row gid + 8h
         w = words.reshape(ntiles, ng, 8, 4, ks)
@@ -154,7 +167,9 @@ def record_rows(rec, lay, H, I, bits, group):
 
 
 @pytest.mark.parametrize("name,over", [("tiny", {}), ("tiny", dict(bits_routed=2, bits_shared=2, group=64)),
-                                       ("tiny", dict(bits_routed=2, bits_shared=4, group=128))])
+                                       ("tiny", dict(bits_routed=2, bits_shared=4, group=128)),
+                                       ("tiny", dict(bits_routed=3, bits_shared=3, group=64)),
+                                       ("tiny", dict(bits_routed=3, bits_shared=4, group=128))])
 def test_packed_arena_matches_generator(name, over):
     w = synth.WORKLOADS[name].with_(**over)
     L = hz.build_layer(w, 0)
@@ -225,7 +240,7 @@ def test_router_forced_and_bad_index():
 
 # ---- A3..A5 expert FFN ---------------------------------------------------------
 
-@pytest.mark.parametrize("name", ["tiny", "layer4", "layer2"])
+@pytest.mark.parametrize("name", ["tiny", "layer4", "layer2", "layer3"])
 def test_expert_ffn(name):
     w, L = get_layer(name)
     B = 2
@@ -344,7 +359,8 @@ def test_combine_residual(with_gate, with_resid):
 
 # ---- A1..A6 whole layer -----------------------------------------------------------
 
-@pytest.mark.parametrize("name,B", [("tiny", 1), ("tiny", 4), ("layer4", 1), ("layer2", 1), ("layer4", 3)])
+@pytest.mark.parametrize("name,B", [("tiny", 1), ("tiny", 4), ("layer4", 1), ("layer2", 1), ("layer4", 3),
+                                    ("layer3", 1), ("layer3", 4)])
 def test_layer_end_to_end(name, B):
     """The three per-token calls against the oracle layer: indices exact on
     tokens whose ranking is decided (near-tie tokens are skipped, reported),
@@ -385,7 +401,9 @@ def test_batched_zipf_routing_layer():
 
 @pytest.mark.parametrize("over", [dict(H=320, I=96, E=5, K=1, group=32), dict(H=512, I=192, E=9, K=8, group=64),
                                   dict(H=512, I=128, E=6, K=3, group=128, bits_routed=2),
-                                  dict(H=256, I=64, E=4, K=4, group=32, bits_routed=2, bits_shared=2)])
+                                  dict(H=256, I=64, E=4, K=4, group=32, bits_routed=2, bits_shared=2),
+                                  dict(H=384, I=128, E=5, K=2, group=64, bits_routed=3, bits_shared=3),
+                                  dict(H=640, I=256, E=7, K=3, group=128, bits_routed=3)])
 @pytest.mark.parametrize("B", [1, 3])
 def test_ragged_and_edge_shapes(over, B):
     w = synth.WORKLOADS["tiny"].with_(**over)
@@ -428,3 +446,93 @@ def test_rmsnorm(B, H, weighted):
         assert (np.abs((got[b] & 0x7FFF) - (want & 0x7FFF)) <= 1).all(), b
         same += int((got[b] == want).sum())
     assert same >= 0.99 * B * H
+
+
+# ---- quantisation (weights -> codes, scale, bias) -------------------------------
+
+def _weights(rng, rows, cols, group):
+    """fp32 weights with groups of every kind the quantiser meets: spread
+    normal rows, groups far from zero for their range (the bias rounds away
+    from the minimum, so codes clamp), and constant groups (scale 0)."""
+    w = rng.normal(size=(rows, cols)) * rng.uniform(0.005, 3.0, size=(rows, 1))
+    far = rng.choice([-1.0, 1.0], size=(rows, 1)) * rng.uniform(60.0, 130.0, size=(rows, 1))
+    w[1::3] = far[1::3] + rng.uniform(0.0, 1.0, size=w[1::3].shape)
+    w[2::5, :group] = 0.375
+    return w.astype(np.float32)
+
+
+@pytest.mark.parametrize("rows,cols,bits,group", [(37, 256, 4, 32), (64, 512, 3, 64), (5, 1024, 2, 128),
+                                                  (1024, 4096, 4, 64), (4096, 1024, 3, 64), (3, 384, 3, 128)])
+@pytest.mark.parametrize("in_bf16", [False, True])
+def test_quantize_bit_exact(rows, cols, bits, group, in_bf16):
+    """moe_quantize against the oracle: codes, scale and bias identical bit
+    for bit (both decide the codes in binary32)."""
+    rng = np.random.default_rng(rows + cols + bits)
+    w = _weights(rng, rows, cols, group)
+    if in_bf16:
+        bits16 = (w.view(np.uint32) >> 16).astype(np.uint16)  # truncate to bf16, then both sides read that
+        w = (bits16.astype(np.uint32) << 16).view(np.float32)
+        wd = torch.from_numpy(bits16.view(np.int16)).cuda()
+    else:
+        wd = torch.from_numpy(w).cuda()
+    codes = torch.full((rows, cols), 0xEE, dtype=torch.uint8, device="cuda")
+    sc = torch.empty((rows, cols // group), dtype=torch.int16, device="cuda")
+    bi = torch.empty_like(sc)
+    ws = moeq.Workspace(1, 1, 32, 32, 1)
+    moeq.moe_quantize(wd, in_bf16, rows, cols, bits, group, codes, sc, bi, ws.buf)
+    torch.cuda.synchronize()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    rc, rs, rb = ref.quantize(w, bits, group)
+    assert (codes.cpu().numpy() == rc).all()
+    assert (sc.cpu().numpy().view(np.uint16) == rs).all()
+    assert (bi.cpu().numpy().view(np.uint16) == rb).all()
+
+
+def test_quantize_flags_non_finite_group():
+    w = np.ones((2, 128), np.float32)
+    w[1, 70] = np.inf
+    codes = torch.full((2, 128), 9, dtype=torch.uint8, device="cuda")
+    sc = torch.full((2, 2), 1, dtype=torch.int16, device="cuda")
+    bi = torch.full((2, 2), 1, dtype=torch.int16, device="cuda")
+    ws = moeq.Workspace(1, 1, 32, 32, 1)
+    moeq.moe_quantize(torch.from_numpy(w).cuda(), False, 2, 128, 4, 64, codes, sc, bi, ws.buf)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_ERR_RANGE
+    c = codes.cpu().numpy()
+    assert (c[1, 64:] == 0).all() and int(sc[1, 1]) == 0 and int(bi[1, 1]) == 0
+    assert int(bi[0, 0]) == 0x3F80 and int(sc[1, 0]) == 0  # the other groups as usual (constant 1.0)
+
+
+@pytest.mark.parametrize("bits,group", [(3, 64), (4, 64), (2, 128), (3, 128)])
+def test_quantize_pack_and_run_expert(bits, group):
+    """fp32 weights through the whole set-up path on the GPU (moe_quantize,
+    then moe_pack_expert) and one token through the resulting 3-matrix
+    expert, against the oracle's quantiser and expert FFN on the same
+    weights."""
+    H, I, E, K = 512, 256, 2, 1
+    rng = np.random.default_rng(bits * 100 + group)
+    mats = [(rng.normal(size=(I, H)) * 0.05).astype(np.float32), (rng.normal(size=(I, H)) * 0.05).astype(np.float32),
+            (rng.normal(size=(H, I)) * 0.05).astype(np.float32)]
+    L = moeq.QuantLayer(H, I, E, K, group, bits, bits)
+    ws = moeq.Workspace(1, K, H, I, E)
+    dev = []
+    for m in mats:
+        r, c = m.shape
+        codes = torch.empty((r, c), dtype=torch.uint8, device="cuda")
+        sc = torch.empty((r, c // group), dtype=torch.int16, device="cuda")
+        bi = torch.empty_like(sc)
+        moeq.moe_quantize(torch.from_numpy(m).cuda(), False, r, c, bits, group, codes, sc, bi, ws.buf)
+        dev.append((codes, sc, bi))
+    for e in range(E + 1):
+        L.pack_expert(e, *dev, ws=ws.buf)
+    L.router_w.zero_()
+    x_bits = (rng.normal(size=H).astype(np.float32).view(np.uint32) >> 16).astype(np.uint16)
+    x = torch.from_numpy(x_bits.view(np.int16)).cuda().view(torch.bfloat16)[None, :]
+    idx = torch.tensor([[1]], dtype=torch.int32, device="cuda")
+    y = torch.empty((1, K + 1, H), dtype=torch.float32, device="cuda")
+    moeq.moe_expert_ffn_q(L.struct, x, 1, idx, y, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    q = [ref.quantize(m, bits, group) for m in mats]
+    yr = ref.expert_ffn(H, I, group, q[0], q[1], q[2], hz.bf16_to_f64(x_bits))
+    for k in range(K + 1):
+        assert hz.max_rel_err(y[0, k].cpu().numpy(), yr) <= FFN_TOL, k
