@@ -21,7 +21,7 @@ LIB_PATH = _build.LIB
 MOE_OK, MOE_ERR_INVALID_ARG, MOE_ERR_ALIGN, MOE_ERR_UNSUPPORTED, MOE_ERR_CUDA = 0, 1, 2, 3, 4
 MOE_ERR_INDEX, MOE_ERR_TIMEOUT, MOE_ERR_WORKSPACE, MOE_ERR_RANGE = 5, 6, 7, 8
 MOEQ_MAX_K = 8
-MOEQ_MAX_B = 64
+MOEQ_MAX_B = 128
 MOEQ_STATIC_SCRATCH_BYTES = 2 << 20
 
 

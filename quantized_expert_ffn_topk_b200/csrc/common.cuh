@@ -14,10 +14,10 @@ struct WsCtrl {
   int error;                // first device-side moe_status (0 = none)
   unsigned router_ticket[16]; // last-CTA tickets of the router kernel, one per 8-token tile (0 between calls)
   unsigned exit_count;      // CTAs that left the fused decode kernel (0 between calls)
-  unsigned sync[4];         // arrival counters of the fused decode kernel (0 between calls)
+  unsigned sync[8];         // arrival counters of the fused decode kernel (0 between calls)
   unsigned wait_us;         // budget of every bounded wait in microseconds (0: about one second)
   int withhold_cta;         // c + 1: CTA c of the fused kernel withholds its first logits arrival (0: none)
-  unsigned pad[40];
+  unsigned pad[36];
 };
 static_assert(sizeof(WsCtrl) == 256, "control block is 256 bytes");
 

@@ -35,6 +35,11 @@ struct FfnParams {
   // shared-memory plans of the one-token kernels (byte offsets)
   int gu_nbuf, gu_gs, gu_part, gu_tiles, gu_stride;
   int dn_nbuf, dn_img_stride, dn_img_gs, dn_part, dn_tiles, dn_stride;
+  int dn_ctas;  // CTAs of the down kernel (its shares are prefetched into L2 by the gate/up kernel)
+  // 1: the dots run on the CUDA cores in fp32 (tile_dot_fma) on fp32 copies
+  // of the inputs at gu_xf / (image) + dn_img_xf, for comparison with the
+  // tensor-core dot (0, the default)
+  int dot_fma, gu_xf, dn_img_xf;
 };
 
 // Groups [lo, hi) of piece q of a tile with ng groups.
@@ -129,8 +134,34 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
       if (r0 == t_lo) ffn_issue(tiles, p.gu_stride, bar, r0, nt, src, is_routed);
       else ffn_issue(tiles, p.gu_stride, bar, r0, nt, src, any);
     }
+#ifndef MOEQ_NO_DOWN_PREFETCH
+    if (r0 == t_lo && warp == 1 && blockIdx.x < p.dn_ctas) {
+      // the down kernel's share for this CTA index, pulled into L2 now so
+      // that its bytes stream while the gate/up tiles are worked (the down
+      // kernel cannot start on this SM before this kernel leaves it)
+      const int tpd = p.H / kTileRows, dtot = (p.K + 1) * tpd;
+      const int d_lo = (int)((long long)dtot * blockIdx.x / p.dn_ctas);
+      const int d_hi = (int)((long long)dtot * (blockIdx.x + 1) / p.dn_ctas);
+      for (int u = d_lo + lane; u < d_hi; u += 32) {
+        const int k = u / tpd, T = u % tpd;
+        const uint8_t* rec = ffn_slot_rec(p, k);
+        if (!rec) continue;
+        const RecGeom& g = k < p.K ? p.geo_r : p.geo_s;
+        prefetch_l2(rec + g.down_off + (size_t)T * g.D, g.D);
+      }
+    }
+#endif
     if (r0 == t_lo) {  // the input image, while the first round's tiles are in flight
-      qstage_vector([&](int j0, float (&v)[16]) { load_bf16_16(p.x + j0, v); }, p.H, p.G, X, tid, blockDim.x);
+      float* xf = reinterpret_cast<float*>(smem + p.gu_xf);
+      qstage_vector(
+          [&](int j0, float (&v)[16]) {
+            load_bf16_16(p.x + j0, v);
+            if (p.dot_fma)
+#pragma unroll
+              for (int q = 0; q < 4; ++q)
+                reinterpret_cast<float4*>(xf + j0)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+          },
+          p.H, p.G, X, tid, blockDim.x);
       __syncthreads();
     }
     for (int pc = warp; pc < nt * kFfnPieces; pc += kFfnWarps) {
@@ -141,8 +172,11 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
         const int g0 = piece_lo(q, (int)g.ng_h), g1 = piece_lo(q + 1, (int)g.ng_h);
         const unsigned char* blk = tiles + (size_t)j * p.gu_stride + (size_t)g0 * g.blk;
-        with_fmt(routed ? p.bits_r : p.bits_s, p.G,
-                 [&]<int BITS, int KS>() { tile_dot<BITS, KS>(blk, g1 - g0, g0, X, acc0, acc1); });
+        const float* xf = reinterpret_cast<const float*>(smem + p.gu_xf);
+        with_fmt(routed ? p.bits_r : p.bits_s, p.G, [&]<int BITS, int KS>() {
+          if (p.dot_fma) tile_dot_fma<BITS, KS>(blk, g1 - g0, g0, xf, X.gs, acc0, acc1);
+          else tile_dot<BITS, KS>(blk, g1 - g0, g0, X, acc0, acc1);
+        });
       }
       if ((lane & 3) == 0) {
         float* pp = part + ((size_t)j * kFfnPieces + q) * kTileRows;
@@ -217,8 +251,16 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
     if (r0 == t_lo) {  // images of the slots this CTA's jobs touch
       for (int k = t_lo / tpd; k <= (t_hi - 1) / tpd; ++k) {
         const float* hk = p.h + (size_t)k * p.I;
-        qstage_vector([&](int j0, float (&v)[16]) { load_f32_16_cg(hk + j0, v); }, p.I, p.G, img(k), tid,
-                      blockDim.x);
+        float* hf = reinterpret_cast<float*>(smem + (size_t)k * p.dn_img_stride + p.dn_img_xf);
+        qstage_vector(
+            [&](int j0, float (&v)[16]) {
+              load_f32_16_cg(hk + j0, v);
+              if (p.dot_fma)
+#pragma unroll
+                for (int q = 0; q < 4; ++q)
+                  reinterpret_cast<float4*>(hf + j0)[q] = make_float4(v[4 * q], v[4 * q + 1], v[4 * q + 2], v[4 * q + 3]);
+            },
+            p.I, p.G, img(k), tid, blockDim.x);
       }
       __syncthreads();
     }
@@ -231,8 +273,11 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
         const int g0 = piece_lo(q, (int)g.ng_i), g1 = piece_lo(q + 1, (int)g.ng_i);
         const unsigned char* blk = tiles + (size_t)j * p.dn_stride + (size_t)g0 * g.blk;
         const QImg Hk = img(k);
-        with_fmt(routed ? p.bits_r : p.bits_s, p.G,
-                 [&]<int BITS, int KS>() { tile_dot<BITS, KS>(blk, g1 - g0, g0, Hk, acc0, acc1); });
+        const float* hf = reinterpret_cast<const float*>(smem + (size_t)k * p.dn_img_stride + p.dn_img_xf);
+        with_fmt(routed ? p.bits_r : p.bits_s, p.G, [&]<int BITS, int KS>() {
+          if (p.dot_fma) tile_dot_fma<BITS, KS>(blk, g1 - g0, g0, hf, Hk.gs, acc0, acc1);
+          else tile_dot<BITS, KS>(blk, g1 - g0, g0, Hk, acc0, acc1);
+        });
       }
       if ((lane & 3) == 0) {
         float* pp = part + ((size_t)j * kFfnPieces + q) * kTileRows;

@@ -3,6 +3,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <cstdlib>
 #include <cstring>
 #include <mutex>
 
@@ -96,7 +97,8 @@ moe_status ensure_smem(K kern, size_t bytes) {
 }
 
 // Workspace layout: [control 256 B][logits B*E fp32][h B*(K+1)*I fp32]
-//                   [r B*H fp32][ss kStackMaxLayers fp32]
+//                   [r B*H fp32][ss kStackMaxCtas fp32: partial sums of squares]
+//                   [token grouping][input images]
 struct WsLayout {
   size_t logits, h, r, ss;
   size_t cnt, off, list, act, nact;  // token grouping (batches)
@@ -114,7 +116,7 @@ inline WsLayout ws_layout(int B, int K, int H, int I, int E) {
   l.r = o;
   o += align_up((size_t)B * H * sizeof(float));
   l.ss = o;
-  o += align_up((size_t)kStackMaxLayers * sizeof(float));
+  o += align_up((size_t)kStackMaxCtas * sizeof(float));
   l.cnt = o;
   o += align_up((size_t)E * 4);
   l.off = o;
@@ -152,6 +154,27 @@ moe_status check_layer(const moe_layer_q* L) {
 }
 
 bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes);  // below
+
+// The one-token FFN kernels' dot: the tensor-core dot, or with
+// MOEQ_BATCH1_DOT=fma in the environment the fp32 CUDA-core dot (a switch
+// for comparing the two on the same kernels; read once).
+int batch1_dot_fma() {
+  static int v = -1;
+  if (v < 0) {
+    const char* e = getenv("MOEQ_BATCH1_DOT");
+    v = (e && strcmp(e, "fma") == 0) ? 1 : 0;
+  }
+  return v;
+}
+
+// Ring of the grouped kernels: as many slots of one tile as fit (at least 2).
+bool grp_plan(size_t tile_bytes, int& slot_bytes, int& nslot, size_t& smem) {
+  const size_t budget = 227 * 1024 - 4 * 1024;  // the static barriers and flags are well under 4 KB
+  slot_bytes = (int)align_up(tile_bytes, 128);
+  nslot = (int)std::min<size_t>(kGrpMaxSlots, budget / (size_t)slot_bytes);
+  smem = (size_t)nslot * slot_bytes;
+  return nslot >= 2;
+}
 
 __global__ void k_ws_debug(WsCtrl* c, unsigned wait_us, int withhold_cta) {
   c->wait_us = wait_us;
@@ -417,7 +440,14 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
                  reinterpret_cast<int*>((char*)ws + wl.list), reinterpret_cast<int*>((char*)ws + wl.act),
                  reinterpret_cast<int*>((char*)ws + wl.nact)};
     const int max_act = std::min(p.E, B * p.K) + kGrpExtraChunks;  // work items at most
-    const int ctas = kGrpCtasPerSm * num_sms();
+    const int ctas = num_sms();  // one CTA per SM: a ring of tile slots fills its shared memory
+    size_t gu_smem = 0, dn_smem = 0;
+    int gu_slot = 0, gu_nslot = 0, dn_slot = 0, dn_nslot = 0;
+    if (!grp_plan((size_t)std::max(p.geo_r.U, p.geo_s.U), gu_slot, gu_nslot, gu_smem) ||
+        !grp_plan((size_t)std::max(p.geo_r.D, p.geo_s.D), dn_slot, dn_nslot, dn_smem))
+      return MOE_ERR_UNSUPPORTED;
+    if (ensure_smem(k_ffn_grp<false>, gu_smem) != MOE_OK || ensure_smem(k_ffn_grp<true>, dn_smem) != MOE_OK)
+      return MOE_ERR_UNSUPPORTED;
     st = launch_pdl(k_group, dim3(1), dim3(256), (size_t)(p.E + 1) * 4, s, idx, B, p.K, p.E, p.H, gp.g, y_out,
                     p.ctrl);
     if (st != MOE_OK) return st;
@@ -431,7 +461,9 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     gp.img_gs_off = wl.ximg_gs;
     gp.tps = p.I / 8;
     gp.max_units = (1 + max_act) * gp.tps;
-    st = launch_pdl(k_ffn_grp<false>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
+    gp.slot_bytes = gu_slot;
+    gp.nslot = gu_nslot;
+    st = launch_pdl(k_ffn_grp<false>, dim3(ctas), dim3(kGrpThreads), gu_smem, s, gp);
     if (st != MOE_OK) return st;
     st = launch_pdl(k_stage_batch, dim3(B, p.K + 1), dim3(256), 0, s, (const void*)p.h, 1, p.I, p.G, himg,
                     wl.himg_stride, wl.himg_gs);
@@ -441,17 +473,21 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     gp.img_gs_off = wl.himg_gs;
     gp.tps = p.H / kTileRows;
     gp.max_units = (1 + max_act) * gp.tps;
-    return launch_pdl(k_ffn_grp<true>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
+    gp.slot_bytes = dn_slot;
+    gp.nslot = dn_nslot;
+    return launch_pdl(k_ffn_grp<true>, dim3(ctas), dim3(kGrpThreads), dn_smem, s, gp);
   }
 
   // one token: every CTA bulk-copies its share of whole tiles into shared memory
+  p.dot_fma = batch1_dot_fma();
   size_t gu_bytes = 0, dn_bytes = 0;
   if (!ffn_plan(p, num_sms(), gu_bytes, dn_bytes)) return MOE_ERR_UNSUPPORTED;
   if (ensure_smem(k_gate_up, gu_bytes) != MOE_OK || ensure_smem(k_down, dn_bytes) != MOE_OK) return MOE_ERR_UNSUPPORTED;
   const int gu_tiles = (p.K + 1) * (p.I / 8), dn_jobs = (p.K + 1) * (p.H / kTileRows);
+  p.dn_ctas = std::min(num_sms(), dn_jobs);
   st = launch_pdl(k_gate_up, dim3(std::min(num_sms(), gu_tiles)), dim3(kFfnWarps * 32), gu_bytes, s, p);
   if (st != MOE_OK) return st;
-  return launch_pdl(k_down, dim3(std::min(num_sms(), dn_jobs)), dim3(kFfnWarps * 32), dn_bytes, s, p);
+  return launch_pdl(k_down, dim3(p.dn_ctas), dim3(kFfnWarps * 32), dn_bytes, s, p);
 }
 
 moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const float* w, const void* x_bf16,
@@ -512,6 +548,8 @@ bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes) {
   size_t o = align_up(qimg_plane_bytes(p.H), 128);
   p.gu_gs = (int)o;
   o += align_up(qimg_gs_bytes(p.H, p.G), 128);
+  p.gu_xf = (int)o;
+  if (p.dot_fma) o += align_up((size_t)p.H * 4, 128);
   const int gu_want = std::min(kFfnMaxBuf, cdiv(gu_total, std::min(G, gu_total)));
   p.gu_part = (int)o;
   o += align_up((size_t)gu_want * kFfnPieces * kTileRows * 4, 128);
@@ -522,7 +560,8 @@ bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes) {
   gu_bytes = o + (size_t)p.gu_nbuf * p.gu_stride;
   // down
   p.dn_img_gs = (int)align_up(qimg_plane_bytes(p.I), 128);
-  p.dn_img_stride = p.dn_img_gs + (int)align_up(qimg_gs_bytes(p.I, p.G), 128);
+  p.dn_img_xf = p.dn_img_gs + (int)align_up(qimg_gs_bytes(p.I, p.G), 128);
+  p.dn_img_stride = p.dn_img_xf + (p.dot_fma ? (int)align_up((size_t)p.I * 4, 128) : 0);
   o = (size_t)p.dn_img_stride * (p.K + 1);
   const int dn_want = std::min(kFfnMaxBuf, cdiv(dn_total, std::min(G, dn_total)));
   p.dn_part = (int)o;
@@ -533,6 +572,18 @@ bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes) {
   p.dn_nbuf = (int)std::min<size_t>(dn_want, (budget - o) / p.dn_stride);
   dn_bytes = o + (size_t)p.dn_nbuf * p.dn_stride;
   return true;
+}
+
+// Static shared memory of the fused decode kernel (bytes), read once.
+size_t stack_static_smem() {
+  static size_t bytes = 0;
+  if (bytes == 0) {
+    cudaFuncAttributes fa{};
+    if (cudaFuncGetAttributes(&fa, k_decode_layers) == cudaSuccess) bytes = fa.sharedSizeBytes;
+    else (void)cudaGetLastError();
+    if (bytes == 0) bytes = 16 * 1024;  // unknown: leave a generous margin
+  }
+  return bytes;
 }
 
 // Shared-memory plan of the fused decode kernel; false when it does not fit.
@@ -552,7 +603,9 @@ bool stack_plan(StackParams& p, int G) {
   p.hgs_stride = (int)align_up(qimg_gs_bytes(I, p.G), 128);
   p.sm_hplanes = take((size_t)p.hplanes_stride * (K + 1));
   p.sm_hgs = take((size_t)p.hgs_stride * (K + 1));
-  const int ntiles_max = cdiv(I / 8, G) + cdiv(K * (I / 8), G) + 1;
+  const int nw = std::min(kMaxWaves, K);
+  int ntiles_max = cdiv(I / 8, G) + 1;
+  for (int w = 0; w < nw; ++w) ntiles_max += cdiv(((w + 1) * K / nw - w * K / nw) * (I / 8), G);
   const int nd_max = cdiv(H / kTileRows, G);
   if (ntiles_max > kMaxTiles || nd_max > kMaxDnTiles) return false;
   p.sm_gpart = take((size_t)ntiles_max * kGuPieces * kTileRows * 4);
@@ -564,7 +617,7 @@ bool stack_plan(StackParams& p, int G) {
                            std::max(p.geo_r.blk, p.geo_s.blk);
   const size_t down_item = (size_t)nd_max * std::max(p.geo_r.D, p.geo_s.D);
   p.slot_bytes = (int)align_up(std::max(std::max((size_t)2 * H * 2, half_tile), down_item), 128);
-  const size_t budget = 227 * 1024 - 6 * 1024;  // leave room for the static shared memory
+  const size_t budget = 227 * 1024 - align_up(stack_static_smem(), 1024);  // room for the static shared memory
   if (o + (size_t)p.slot_bytes * 2 > budget) return false;
   p.nslot = (int)std::min<size_t>(kMaxSlots, (budget - o) / p.slot_bytes);
   p.sm_ring = take((size_t)p.slot_bytes * p.nslot);
@@ -599,10 +652,14 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   if (ws_bytes < moe_workspace_bytes(1, L0.K, L0.H, L0.I, L0.E)) return MOE_ERR_WORKSPACE;
   const int G = num_sms();
   auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
-  if (L0.E > 1024 || cdiv(L0.E, G) > kMaxRouterRowsPerCta) return MOE_ERR_UNSUPPORTED;
+  if (L0.E > kStackMaxE || cdiv(L0.E, G) > kMaxRouterRowsPerCta || G > kStackMaxCtas) return MOE_ERR_UNSUPPORTED;
   const int tps = L0.I / 8;
-  if (cdiv(cdiv(L0.E, G), 2) + 2 * (cdiv(tps, G) + cdiv(L0.K * tps, G) + 1) + L0.K + 1 > kMaxItems)
-    return MOE_ERR_UNSUPPORTED;
+  {
+    const int nw = std::min(kMaxWaves, L0.K);
+    int gu = cdiv(tps, G);
+    for (int w = 0; w < nw; ++w) gu += cdiv(((w + 1) * L0.K / nw - w * L0.K / nw) * tps, G);
+    if (cdiv(cdiv(L0.E, G), 2) + 2 * gu + L0.K + 1 > kMaxItems) return MOE_ERR_UNSUPPORTED;
+  }
   if (L0.H % 32 != 0 || L0.H / 16 > kCThreads) return MOE_ERR_UNSUPPORTED;
 
   StackParams p{};
@@ -638,6 +695,14 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   p.h = reinterpret_cast<float*>((char*)ws + wl.h);
   p.r = reinterpret_cast<float*>((char*)ws + wl.r);
   p.sync = reinterpret_cast<WsCtrl*>(ws)->sync;
+  p.ss_part = reinterpret_cast<float*>((char*)ws + wl.ss);
+#ifdef MOEQ_STACK_TRACE
+  // timeline builds: the phase stamps go right after the workspace proper
+  const size_t trace_bytes = (size_t)n_layers * kTracePhases * G * sizeof(unsigned long long);
+  p.trace = ws_bytes >= wl.total + trace_bytes ? reinterpret_cast<unsigned long long*>((char*)ws + wl.total) : nullptr;
+#else
+  p.trace = nullptr;
+#endif
   if (!stack_plan(p, G)) return MOE_ERR_UNSUPPORTED;
   const size_t smem = stack_smem_bytes(p);
   if (ensure_smem(k_decode_layers, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;

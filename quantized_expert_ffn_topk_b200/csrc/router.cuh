@@ -6,7 +6,10 @@
 
 namespace moeq {
 
-constexpr int kRouterWarps = 8;     // warps per CTA, one expert row per warp at a time
+#ifndef MOEQ_ROUTER_WARPS
+#define MOEQ_ROUTER_WARPS 8
+#endif
+constexpr int kRouterWarps = MOEQ_ROUTER_WARPS;  // warps per CTA, one expert row per warp at a time
 constexpr int kRouterTokTile = 8;   // tokens of one CTA (its x staged in shared memory)
 constexpr int kRouterUnroll = 8;    // 16-byte loads of one row in flight per lane (the rows were prefetched to L2)
 constexpr int kRouterMaxE = 1024;   // experts the selection holds: 32 keys per lane

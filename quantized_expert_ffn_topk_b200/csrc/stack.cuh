@@ -52,7 +52,19 @@ constexpr int kItemPieces = kDnPieces * kMaxDnTiles;  // pieces of the largest i
 constexpr int kMaxItems = 32;
 constexpr int kMaxPieces = kMaxItems * kItemPieces;
 constexpr int kMaxTiles = 16;                    // gate/up tiles per CTA per layer
-enum { kSyncLogits = 0, kSyncSharedH = 1, kSyncRoutedH = 2, kSyncResid = 3 };  // counters in the workspace
+constexpr int kStackMaxCtas = 1024;              // CTAs of the grid at most (partial sums in the workspace)
+constexpr int kStackMaxE = 1024;                 // experts at most (two logits per compute thread)
+// The routed experts' h is exchanged in waves of slots: a CTA works the
+// gate/up tiles of wave 0, publishes them, works wave 1 while wave 0's
+// exchange completes, and only then waits for wave 0's h to run its down
+// tiles, so the exchange of one wave overlaps the work of the next.
+#ifndef MOEQ_ROUTED_WAVES
+#define MOEQ_ROUTED_WAVES 2
+#endif
+constexpr int kMaxWaves = MOEQ_ROUTED_WAVES;
+// counters in the workspace: logits, shared h, routed h per wave, r
+enum { kSyncLogits = 0, kSyncSharedH = 1, kSyncRoutedH = 2, kSyncResid = kSyncRoutedH + kMaxWaves, kNumSync };
+static_assert(kNumSync <= 8, "arrival counters of the control block");
 
 enum { kItemRouter = 0, kItemGateUp = 1, kItemDown = 2 };
 
@@ -83,11 +95,32 @@ struct StackParams {
   float* h;                 // [K+1, I]
   float* r;                 // [H] residual stream
   unsigned* sync;           // [4] arrival counters (kSync*)
+  float* ss_part;           // [G] each CTA's sum of squares of its rows of r
+  unsigned long long* trace;  // per-phase timestamps (builds with MOEQ_STACK_TRACE only), or null
   // shared-memory plan (byte offsets into the dynamic buffer)
   int sm_xs, sm_xplanes, sm_xgs;
   int sm_hplanes, hplanes_stride, sm_hgs, hgs_stride;
   int sm_gpart, sm_dpart, sm_ring, slot_bytes, nslot;
 };
+
+// Optional phase timeline (compiled in with -DMOEQ_STACK_TRACE only): one
+// thread per CTA stamps %globaltimer at phase ends into
+// trace[(layer * kTracePhases + phase) * G + cta]. Off in the library build.
+constexpr int kTracePhases = 14;
+#ifdef MOEQ_STACK_TRACE
+#define STACK_MARK(cond, l, ph)                                                                    \
+  do {                                                                                             \
+    if ((cond) && p.trace) {                                                                       \
+      unsigned long long t_;                                                                       \
+      asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_));                                       \
+      p.trace[((size_t)(l) * kTracePhases + (ph)) * gridDim.x + blockIdx.x] = t_;                  \
+    }                                                                                              \
+  } while (0)
+#else
+#define STACK_MARK(cond, l, ph) \
+  do {                          \
+  } while (0)
+#endif
 
 // CTA c's share [lo, hi) of n items split evenly over G CTAs.
 __host__ __device__ inline int share_lo(int c, int G, int n) { return (int)((long long)n * c / G); }
@@ -99,7 +132,11 @@ struct ItemPlan {
   int n_items, n_router_items, n_sgu_items, n_pre_items, n_rgu_items;  // item ranges, in ring order:
   // [0, n_router_items) router, [.., n_sgu_items) shared gate/up, [.., n_pre_items)
   // shared down (all three issued during the previous layer), [.., n_rgu_items)
-  // routed gate/up, [.., n_items) routed down
+  // routed gate/up (wave by wave: wave w ends at gu_end[w]), [.., n_items) routed
+  // down (wave w ends at dn_end[w])
+  int nwaves;
+  int wave_k0[kMaxWaves + 1];              // wave w holds slots [wave_k0[w], wave_k0[w+1])
+  int gu_end[kMaxWaves], dn_end[kMaxWaves];
   int n_pieces, n_router_pieces, n_pre_pieces;
   int kind[kMaxItems];
   int k[kMaxItems];                        // slot (K: shared)
@@ -164,10 +201,19 @@ __device__ void make_plan(const StackParams& p, ItemPlan& P) {
   if (P.nd > 0) add_down(p.K);
   P.n_pre_items = n;
   P.n_pre_pieces = pc;
-  for (int u = share_lo(c, G, p.K * tps); u < share_lo(c + 1, G, p.K * tps); ++u) add_tile(u / tps, u % tps);
+  P.nwaves = min(kMaxWaves, p.K);
+  for (int w = 0; w <= P.nwaves; ++w) P.wave_k0[w] = w * p.K / P.nwaves;
+  for (int w = 0; w < P.nwaves; ++w) {
+    const int k0 = P.wave_k0[w], nwt = (P.wave_k0[w + 1] - k0) * tps;
+    for (int u = share_lo(c, G, nwt); u < share_lo(c + 1, G, nwt); ++u) add_tile(k0 + u / tps, u % tps);
+    P.gu_end[w] = n;
+  }
   P.n_rgu_items = n;
-  if (P.nd > 0)
-    for (int k = 0; k < p.K; ++k) add_down(k);
+  for (int w = 0; w < P.nwaves; ++w) {
+    if (P.nd > 0)
+      for (int k = P.wave_k0[w]; k < P.wave_k0[w + 1]; ++k) add_down(k);
+    P.dn_end[w] = n;
+  }
   P.n_items = n;
   P.n_pieces = pc;
   P.ntiles = tl;
@@ -254,7 +300,8 @@ struct TopkScratch {
   float m[kCWarps], z[kCWarps];       // each warp's max logit and sum of exp(v - max)
 };
 
-// Softmax and top-K of layer l's logits (router gating as the Flash-MoE page
+// Softmax and top-K of layer l's logits `lg` (in shared memory, relayed there
+// by the copy warp) (router gating as the Flash-MoE page
 // gives it in "Metal Compute Shaders": softmax over all experts, the K
 // largest, weights renormalised on request), run by all compute warps of the
 // CTA. Thread t holds logits t and t + kCThreads; a warp takes its K best by
@@ -265,17 +312,18 @@ struct TopkScratch {
 // The normaliser is summed per warp around the warp's own maximum and
 // rescaled to the global one. Warp 0 writes the picks and weights to
 // s_idx/s_w and then raises *ready to l + 1 for the producer warp.
-__device__ void block_topk(const StackParams& p, int l, TopkScratch& S, int* s_idx, float* s_w, volatile int* ready) {
+__device__ void block_topk(const StackParams& p, int l, const float* lg, TopkScratch& S, int* s_idx, float* s_w,
+                           volatile int* ready) {
   const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
   const int E = p.E, K = p.K;
   const int t1 = tid + kCThreads;
   float v0 = -INFINITY, v1 = -INFINITY;
   if (tid < E) {
-    const float x = __ldcg(p.logits + tid);
+    const float x = lg[tid];
     v0 = x == x ? x : -INFINITY;
   }
   if (t1 < E) {
-    const float x = __ldcg(p.logits + t1);
+    const float x = lg[t1];
     v1 = x == x ? x : -INFINITY;
   }
   uint32_t k0 = tid < E ? logit_key(v0) : 0u, k1 = t1 < E ? logit_key(v1) : 0u;
@@ -328,7 +376,7 @@ __device__ void block_topk(const StackParams& p, int l, TopkScratch& S, int* s_i
       const int bi = forced[lane];
       const bool okf = bi >= 0 && bi < E;
       pick_e = okf ? bi : -1;
-      pick_l = okf ? __ldcg(p.logits + bi) : -INFINITY;
+      pick_l = okf ? lg[bi] : -INFINITY;
     }
   } else {
     // candidate c = lane + 32 j of the warps' kCWarps * K
@@ -421,6 +469,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
   __shared__ TopkScratch s_topk;
   __shared__ volatile int s_abort;
   __shared__ volatile int s_topk_ready;
+  __shared__ volatile int s_logits_ready;  // layer + 1 once s_logits holds that layer's logits
+  __shared__ __align__(16) float s_logits[kStackMaxE];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
   const int G = gridDim.x;
@@ -441,6 +491,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     for (int t = 0; t < kMaxTiles; ++t) s_gcnt[t] = 0;
     s_abort = 0;
     s_topk_ready = 0;
+    s_logits_ready = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -456,10 +507,22 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     Ring R{full_bar, empty_bar, s_last, sm + p.sm_ring, p.slot_bytes, p.nslot};
     if (!issue_items(p, P, R, 0, 0, P.n_pre_items, 0u, s_idx, &s_abort, budget) && lane == 0) fail();
     for (int l = 0; l < p.n_layers; ++l) {
+      // relay: once every CTA has published layer l's logits, copy them into
+      // shared memory for the compute warps' top-K (the poll and the L2 read
+      // overlap the compute warps' shared-expert work)
+      if (lane == 0 && !s_abort && !counter_wait(p.sync + kSyncLogits, (unsigned)(l + 1) * (unsigned)G, &s_abort, budget) &&
+          !s_abort)
+        fail();
+      __syncwarp();
+      for (int e = lane; e < p.E; e += 32) s_logits[e] = __ldcg(p.logits + e);
+      __syncwarp();
+      __threadfence_block();
+      if (lane == 0) s_logits_ready = l + 1;
       // routing: the compute warps publish layer l's picks in s_idx/s_w
       if (lane == 0 && !s_abort && !flag_wait(&s_topk_ready, l + 1, &s_abort, budget) && !s_abort) fail();
       __syncwarp();
       __threadfence_block();
+      STACK_MARK(lane == 0, l, 13);
       // routed gate/up items (they gate the h exchange), the routed down
       // items (needed only after it), then the next layer's router, shared
       // gate/up and shared down items
@@ -611,6 +674,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
 
     const unsigned G1 = (unsigned)G;
     for (int l = 0; l < p.n_layers; ++l) {
+      STACK_MARK(tid == 0, l, 0);
       // ---- stage x_l ----
       {
         const uint16_t* gw = p.L[l].gate_w;
@@ -619,19 +683,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         const bool active = tid < nseg;
         if (l > 0) {
           if (tid == 0 && !counter_wait(p.sync + kSyncResid, (unsigned)l * G1, &s_abort, budget) && !s_abort) fail();
+          STACK_MARK(tid == 0, l, 1);
           named_sync(1, kCThreads);
-          float ss = 0.f;
-          if (active) {
-            load_f32_16_cg(p.r + (size_t)tid * 16, v);
-#pragma unroll
-            for (int j = 0; j < 16; ++j) ss += v[j] * v[j];
-          }
-          ss = warp_sum(ss);
-          if (lane == 0) s_red[0][warp] = ss;
-          named_sync(1, kCThreads);
-          float tot = 0.f;
-          for (int w = 0; w < kCWarps; ++w) tot += s_red[0][w];
-          const float inv_norm = rsqrtf(tot / (float)H + p.eps);
+          // the RMS norm's sum of squares from the CTAs' published partial
+          // sums, in one fixed order (every warp of every CTA gets the same
+          // value), read in the same round trip as r
+          float part = 0.f;
+          for (int c = lane; c < G; c += 32) part += __ldcg(p.ss_part + c);
+          if (active) load_f32_16_cg(p.r + (size_t)tid * 16, v);
+          const float inv_norm = rsqrtf(warp_sum(part) / (float)H + p.eps);
           if (active) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = bf16_bits_to_f32(f32_to_bf16_bits(v[j] * inv_norm));
@@ -664,6 +724,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         if (lane == 0) s_red[1][warp] = gdot;
         named_sync(1, kCThreads);
       }
+      STACK_MARK(tid == 0, l, 2);
       float gamma = 1.f;
       if (p.L[l].gate_w) {
         float d = 0.f;
@@ -684,30 +745,43 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         __syncwarp();
         if (lane == 0 && !(withhold && l == 0)) arrive_release_gpu(p.sync + kSyncLogits);
       }
+      STACK_MARK(tid == 0, l, 3);
       run_items(l, P.n_router_items, P.n_sgu_items);
       named_sync(1, kCThreads);
       if (tid == 0) arrive_release_gpu(p.sync + kSyncSharedH);
+      STACK_MARK(tid == 0, l, 4);
 
       // ---- softmax / top-K over every CTA's logits (the producer waits for it) ----
-      if (tid == 0 && !counter_wait(p.sync + kSyncLogits, (unsigned)(l + 1) * G1, &s_abort, budget) && !s_abort) fail();
-      named_sync(1, kCThreads);
-      block_topk(p, l, s_topk, s_idx, s_w, &s_topk_ready);
+      if (lane == 0 && !flag_wait(&s_logits_ready, l + 1, &s_abort, budget) && !s_abort) fail();
+      __syncwarp();
+      STACK_MARK(tid == 0, l, 5);
+      block_topk(p, l, s_logits, s_topk, s_idx, s_w, &s_topk_ready);
+      STACK_MARK(tid == 0, l, 6);
 
       // ---- the shared expert's down tiles, once every CTA's shared h is out ----
       stage_h(K, K + 1, kSyncSharedH, (unsigned)(l + 1) * G1);
       named_sync(1, kCThreads);
+      STACK_MARK(tid == 0, l, 7);
       run_items(l, P.n_sgu_items, P.n_pre_items);
+      STACK_MARK(tid == 0, l, 8);
 
-      // ---- routed gate/up pieces ----
-      run_items(l, P.n_pre_items, P.n_rgu_items);
-      named_sync(1, kCThreads);
-      if (tid == 0) arrive_release_gpu(p.sync + kSyncRoutedH);
+      // ---- routed gate/up pieces, wave by wave, each wave's h published ----
+      for (int w = 0; w < P.nwaves; ++w) {
+        run_items(l, w == 0 ? P.n_pre_items : P.gu_end[w - 1], P.gu_end[w]);
+        named_sync(1, kCThreads);
+        if (tid == 0) arrive_release_gpu(p.sync + kSyncRoutedH + w);
+      }
+      STACK_MARK(tid == 0, l, 9);
 
-      // ---- routed down tiles ----
-      stage_h(0, K, kSyncRoutedH, (unsigned)(l + 1) * G1);
+      // ---- routed down tiles, wave by wave once the wave's h is out ----
+      for (int w = 0; w < P.nwaves; ++w) {
+        stage_h(P.wave_k0[w], P.wave_k0[w + 1], kSyncRoutedH + w, (unsigned)(l + 1) * G1);
+        named_sync(1, kCThreads);
+        if (w == 0) STACK_MARK(tid == 0, l, 10);
+        run_items(l, w == 0 ? P.n_rgu_items : P.dn_end[w - 1], P.dn_end[w]);
+      }
       named_sync(1, kCThreads);
-      run_items(l, P.n_rgu_items, n_items);
-      named_sync(1, kCThreads);
+      STACK_MARK(tid == 0, l, 11);
 
       // ---- combine: r_{l+1} = r_l + sum_k w_k y_k + gamma y_shared ----
       if (my_row >= 0) {
@@ -725,8 +799,18 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         if (l + 1 < p.n_layers || p.xnorm_out) __stcg(p.r + my_row, my_r);
         if (l + 1 == p.n_layers) p.resid_out[my_row] = my_r;
       }
+      {  // this CTA's partial sum of squares of r_{l+1}, published with its rows
+        const float sq = warp_sum(my_row >= 0 ? my_r * my_r : 0.f);
+        if (lane == 0) s_red[0][warp] = sq;
+      }
       named_sync(1, kCThreads);
-      if (tid == 0) arrive_release_gpu(p.sync + kSyncResid);
+      if (tid == 0) {
+        float t = 0.f;
+        for (int w = 0; w < kCWarps; ++w) t += s_red[0][w];
+        __stcg(p.ss_part + blockIdx.x, t);
+        arrive_release_gpu(p.sync + kSyncResid);
+      }
+      STACK_MARK(tid == 0, l, 12);
     }
 
     // ---- optional RMSNorm'd bf16 output of the last layer ----
@@ -735,18 +819,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       float ss = 0.f;
       if (tid == 0 && !counter_wait(p.sync + kSyncResid, (unsigned)p.n_layers * G1, &s_abort, budget) && !s_abort) fail();
       named_sync(1, kCThreads);
-      if (tid < nseg) {
-        float v[16];
-        load_f32_16_cg(p.r + (size_t)tid * 16, v);
-#pragma unroll
-        for (int j = 0; j < 16; ++j) ss += v[j] * v[j];
-      }
-      ss = warp_sum(ss);
-      if (lane == 0) s_red[0][warp] = ss;
-      named_sync(1, kCThreads);
-      float tot = 0.f;
-      for (int w = 0; w < kCWarps; ++w) tot += s_red[0][w];
-      const float inv = rsqrtf(tot / (float)H + p.eps);
+      (void)nseg;
+      for (int c = lane; c < G; c += 32) ss += __ldcg(p.ss_part + c);
+      const float inv = rsqrtf(warp_sum(ss) / (float)H + p.eps);
       if (my_row >= 0) p.xnorm_out[my_row] = f32_to_bf16_bits(my_r * inv);
     }
   }
@@ -757,7 +832,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     __threadfence();
     const unsigned t = atomicAdd(&p.ctrl->exit_count, 1u);
     if (t == (unsigned)G - 1) {
-      for (int c = 0; c < 4; ++c) atomicExch(p.sync + c, 0u);
+      for (int c = 0; c < kNumSync; ++c) atomicExch(p.sync + c, 0u);
       __threadfence();
       atomicExch(&p.ctrl->exit_count, 0u);
     }

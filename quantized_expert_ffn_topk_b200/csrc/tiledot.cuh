@@ -267,6 +267,64 @@ __device__ __forceinline__ void tile_dot(const unsigned char* blk0, int nblk, in
   }
 }
 
+// ---- the same tile dot on the CUDA cores (for comparison) -------------------
+//
+// The group-hoisted affine dot of the Flash-MoE page ("Kernel dequant toi uu
+// FMA") in fp32 on the CUDA cores, over the same record blocks: each lane
+// turns its codes into floats (one byte permute and one subtraction each:
+// 2^23 + q as a binary32 pattern, minus 2^23), forms sum(q * x) over its
+// eight inputs per k-step for its two rows with FFMA, scales by the group's
+// scale and adds bias * sum(x) once per row; the four lanes of a row quad
+// are summed at the end. x is the fp32 input vector in shared memory; gs[g].y
+// is the group's exact sum of inputs. No rounding of x beyond fp32.
+__device__ __forceinline__ float code_f(uint32_t a, int i) {
+  return __uint_as_float(__byte_perm(a, 0x4B000000u, 0x7540u | (uint32_t)i)) - 8388608.f;
+}
+
+template <int BITS, int KS>
+__device__ __forceinline__ void tile_dot_fma(const unsigned char* blk0, int nblk, int g0, const float* xf,
+                                             const float2* gs, float& acc0, float& acc1) {
+  using F = TileFmt<BITS, KS>;
+  const int lane = threadIdx.x & 31, t = lane & 3;
+  float s0 = 0.f, s1 = 0.f;
+#pragma unroll 2
+  for (int b = 0; b < nblk; ++b) {
+    const unsigned char* blk = blk0 + (size_t)b * F::BB;
+    uint32_t w[F::NW];
+    load_lane_codes<BITS, KS>(blk, lane, w);
+    const uint2 sb = *reinterpret_cast<const uint2*>(blk + F::CB + (lane >> 2) * 8);
+    const int g = g0 + b;
+    float p0 = 0.f, p1 = 0.f;
+#pragma unroll
+    for (int ks = 0; ks < KS; ++ks) {
+      uint32_t a[4];
+      extract_a<BITS, KS>(w, ks, a);
+      const float4* xv = reinterpret_cast<const float4*>(xf + ((size_t)g * KS + ks) * 32 + 8 * t);
+      const float4 x0 = xv[0], x1 = xv[1];
+      const float xe[4] = {x0.x, x0.z, x1.x, x1.z};  // inputs 8t + 2i
+      const float xo[4] = {x0.y, x0.w, x1.y, x1.w};  // inputs 8t + 2i + 1
+#pragma unroll
+      for (int i = 0; i < 4; ++i) {
+        p0 = fmaf(code_f(a[0], i), xe[i], p0);
+        p0 = fmaf(code_f(a[2], i), xo[i], p0);
+        p1 = fmaf(code_f(a[1], i), xe[i], p1);
+        p1 = fmaf(code_f(a[3], i), xo[i], p1);
+      }
+    }
+    const float sx = t == 0 ? gs[g].y : 0.f;
+    s0 = fmaf(__uint_as_float(sb.x << 16), p0, s0);
+    s0 = fmaf(__uint_as_float(sb.x & 0xFFFF0000u), sx, s0);
+    s1 = fmaf(__uint_as_float(sb.y << 16), p1, s1);
+    s1 = fmaf(__uint_as_float(sb.y & 0xFFFF0000u), sx, s1);
+  }
+  s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 1);
+  s0 += __shfl_xor_sync(0xFFFFFFFFu, s0, 2);
+  s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 1);
+  s1 += __shfl_xor_sync(0xFFFFFFFFu, s1, 2);
+  acc0 += s0;
+  acc1 += s1;
+}
+
 // Dispatch on (bits, group) for callers with runtime values (3 bits: group
 // 64 or 128 only; the host rejects 3-bit group 32).
 template <typename Fn>

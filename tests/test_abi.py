@@ -108,7 +108,7 @@ def test_router_rejects_bad_arguments(moeq):
     assert call(K=9) == moeq.MOE_ERR_INVALID_ARG
     assert call(K=5, E=4) == moeq.MOE_ERR_INVALID_ARG
     assert call(B=0) == moeq.MOE_ERR_INVALID_ARG
-    assert call(B=65) == moeq.MOE_ERR_INVALID_ARG
+    assert call(B=129) == moeq.MOE_ERR_INVALID_ARG
     assert call(ws=None) == moeq.MOE_ERR_WORKSPACE
     assert call(n=100) == moeq.MOE_ERR_WORKSPACE
     assert call(x=M) == moeq.MOE_ERR_ALIGN
@@ -181,6 +181,7 @@ def test_static_call_checks_arguments_before_its_size(moeq):
     # a batch too large for the scratch, with a bad pointer: the pointer is reported
     assert L.moe_expert_ffn_q_static(ctypes.byref(s), M, 64, A, A, None, None) == moeq.MOE_ERR_ALIGN
     assert L.moe_expert_ffn_q_static(ctypes.byref(s), A, 64, A, A, None, None) == moeq.MOE_ERR_WORKSPACE
+    assert L.moe_expert_ffn_q_static(ctypes.byref(s), A, 35, A, A, None, None) == moeq.MOE_ERR_WORKSPACE
 
 
 def test_quantize_rejects_bad_arguments(moeq):

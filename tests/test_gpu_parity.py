@@ -380,6 +380,33 @@ def test_layer_end_to_end(name, B):
     print("near-tie tokens skipped:", skipped)
 
 
+@pytest.mark.parametrize("B", [64, 128])
+def test_batched_zipf_larger_batches(B):
+    """Batches of 64 and 128 tokens on the layer4 arena (Zipf(1.1) picks, so
+    popular experts carry many tokens and the shared expert carries all of
+    them): every token's weights, every expert slot and every residual row
+    against the oracle (the oracle runs the tokens on a thread pool)."""
+    from concurrent.futures import ThreadPoolExecutor
+    import os
+    w, L = get_layer("batch32")
+    routing = synth.zipf_routing(w.E, w.K, B, 1, w.zipf_s, 17 + B)[0]
+    x = hz.x_device(w, 3000 + B, B)
+    out = run_layer(w, L, x, forced=routing)
+    xb = synth.x_host(w, 3000 + B, B)
+    yg = out["y"].cpu().numpy()
+    wg = out["w"].cpu().numpy()
+    rg = out["resid"].cpu().numpy()
+    def one(b):
+        return b, oracle_token(w, 0, xb[b], forced=routing[b])
+
+    with ThreadPoolExecutor(max_workers=min(16, os.cpu_count() or 1)) as pool:
+        for b, ro in pool.map(one, range(B)):
+            assert np.abs(wg[b] - ro["w"]).max() <= W_TOL, b
+            for k in range(w.K + 1):
+                assert hz.max_rel_err(yg[b, k], ro["y"][k]) <= FFN_TOL, (b, k)
+            assert hz.max_rel_err(rg[b], ro["out"]) <= FFN_TOL, b
+
+
 def test_batched_zipf_routing_layer():
     """The batched workload (32 tokens, forced Zipf(1.1) picks, grouped per
     expert): every token's weights, every expert slot of y and every
@@ -536,3 +563,49 @@ def test_quantize_pack_and_run_expert(bits, group):
     yr = ref.expert_ffn(H, I, group, q[0], q[1], q[2], hz.bf16_to_f64(x_bits))
     for k in range(K + 1):
         assert hz.max_rel_err(y[0, k].cpu().numpy(), yr) <= FFN_TOL, k
+
+
+# ---- the CUDA-core comparison dot of the one-token kernels ---------------------
+
+_FMA_CHECK = r'''
+import sys
+import numpy as np
+import torch
+sys.path.insert(0, ".")
+from synth import synth
+from tests import harness as hz
+from oracle import oracle as ref
+import quantized_expert_ffn_topk_b200 as moeq
+for name in ("layer4", "layer3", "tiny"):
+    w = synth.WORKLOADS[name]
+    L = hz.build_layer(w, 0)
+    x = hz.x_device(w, 31, 1)
+    idx_np = np.random.default_rng(3).choice(w.E, size=(1, w.K), replace=False).astype(np.int32)
+    ws = moeq.Workspace(1, w.K, w.H, w.I, w.E)
+    y = torch.empty((1, w.K + 1, w.H), dtype=torch.float32, device="cuda")
+    moeq.moe_expert_ffn_q(L.struct, x, 1, torch.from_numpy(idx_np).cuda(), y, ws.buf, ws.nbytes)
+    torch.cuda.synchronize()
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    experts = hz.oracle_experts(w, 0)
+    xd = hz.bf16_to_f64(synth.x_host(w, 31, 1)[0])
+    for k, e in enumerate(list(idx_np[0]) + [w.E]):
+        g, u, d = experts(int(e))
+        err = hz.max_rel_err(y[0, k].cpu().numpy(), ref.expert_ffn(w.H, w.I, w.group, g, u, d, xd))
+        assert err <= 2e-3, (name, k, err)
+    del L
+    torch.cuda.empty_cache()
+print("fma dot ok")
+'''
+
+
+def test_expert_ffn_cuda_core_dot():
+    """The one-token expert FFN with its dots on the CUDA cores in fp32
+    (MOEQ_BATCH1_DOT=fma, read once per process, hence a child process): the
+    same parity bar as the tensor-core dot."""
+    import os
+    import subprocess
+    import sys
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    r = subprocess.run([sys.executable, "-c", _FMA_CHECK], cwd=root, capture_output=True, text=True, timeout=900,
+                       env=dict(os.environ, MOEQ_BATCH1_DOT="fma"))
+    assert r.returncode == 0 and "fma dot ok" in r.stdout, r.stdout[-2000:] + r.stderr[-4000:]

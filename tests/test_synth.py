@@ -23,8 +23,10 @@ def test_codes_cover_their_range(syn):
     assert c4.max() == 15 and c4.min() == 0
     c2 = syn.codes_host(w.with_(bits_routed=2), 0, 0, syn.DOWN)
     assert c2.max() == 3 and c2.min() == 0
+    c3 = syn.codes_host(w.with_(bits_routed=3), 0, 0, syn.DOWN)
+    assert c3.max() == 7 and c3.min() == 0
     # low bits of the same draws
-    assert ((c4 & 3) == c2).all()
+    assert ((c4 & 3) == c2).all() and ((c4 & 7) == c3).all()
     counts = np.bincount(c4.ravel(), minlength=16) / c4.size
     assert np.abs(counts - 1 / 16).max() < 0.01
 
