@@ -282,8 +282,9 @@ moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const floa
  *   resid_out   fp32 [H]: r_n
  *   xnorm_bf16_out  bf16 [H] or NULL: bf16(RMSNorm(r_n))
  * Needs one CTA per SM for the whole launch (co-resident; cooperative
- * launch), E <= 1024, H/16 <= 512, and a shared-memory plan that fits
- * one SM (MOE_ERR_UNSUPPORTED otherwise; use the per-call path). A wait that
+ * launch), E <= 1024, H/16 <= 512, a shared-memory plan that fits one SM,
+ * and a shared expert at 4 bits or at the routed width (MOE_ERR_UNSUPPORTED
+ * otherwise; use the per-call path). A wait that
  * exceeds about one second ends the kernel with MOE_ERR_TIMEOUT in the
  * workspace, which must then be re-initialised with moe_workspace_init.
  */

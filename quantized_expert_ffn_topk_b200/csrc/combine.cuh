@@ -4,12 +4,14 @@
 // sections "Metal Compute Shaders" and "Deferred GPU Expert Compute").
 #pragma once
 
+#include <cooperative_groups.h>
+
 #include "common.cuh"
 
 namespace moeq {
 
 constexpr int kCombineThreads = 512;
-constexpr int kCombineU = 8;  // elements per thread per pass (one pass covers H <= 4096)
+constexpr int kCombineCluster = 8;  // CTAs per token (a thread block cluster)
 
 struct CombineParams {
   const float* y;          // [B, K+1, H]
@@ -23,12 +25,19 @@ struct CombineParams {
   float eps;
 };
 
-// grid: B CTAs, one token each. A thread keeps the outputs of its first pass
-// in registers for the RMSNorm'd copy; only when H > kCombineThreads *
-// kCombineU does it read later ones back (each thread only what it wrote).
-__global__ void __launch_bounds__(kCombineThreads) k_combine(CombineParams p) {
+// grid: B clusters of kCombineCluster CTAs, one cluster per token; CTA rank
+// q of a cluster owns elements [q*per, (q+1)*per) of its token (per =
+// ceil(H / kCombineCluster)), one or a few per thread. The RMSNorm'd copy
+// needs the token's whole sum of squares: each CTA reduces its part in
+// shared memory and reads its cluster peers' parts through distributed
+// shared memory (two cluster barriers; every CTA reaches both).
+__global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombineThreads)
+    k_combine(CombineParams p) {
   __shared__ float red[32];
-  const int b = blockIdx.x;
+  __shared__ float s_part;
+  namespace cg = cooperative_groups;
+  cg::cluster_group cluster = cg::this_cluster();
+  const int b = blockIdx.x / kCombineCluster, q = (int)cluster.block_rank();
   pdl_trigger();
   pdl_wait();
   const uint16_t* xb = p.x + (size_t)b * p.H;
@@ -46,46 +55,32 @@ __global__ void __launch_bounds__(kCombineThreads) k_combine(CombineParams p) {
   for (int k = 0; k <= MOEQ_MAX_K; ++k) wk[k] = k < p.K ? p.w[(size_t)b * p.K + k] : (k == p.K ? gamma : 0.f);
   const float* yb = p.y + (size_t)b * (p.K + 1) * p.H;
   float* rb = p.resid_out + (size_t)b * p.H;
-  float ss = 0.f, keep[kCombineU];
-  const int stride = blockDim.x * kCombineU;
-  for (int j0 = threadIdx.x; j0 < p.H; j0 += stride) {
-    float acc[kCombineU];
+  const int per = (p.H + kCombineCluster - 1) / kCombineCluster;
+  const int j0 = q * per, j1 = min(p.H, j0 + per);
+  float ss = 0.f, keep = 0.f;
+  for (int j = j0 + (int)threadIdx.x; j < j1; j += blockDim.x) {
+    float acc = p.resid_in ? p.resid_in[(size_t)b * p.H + j] : bf16_bits_to_f32(xb[j]);
 #pragma unroll
-    for (int u = 0; u < kCombineU; ++u) {
-      const int j = j0 + u * blockDim.x;
-      acc[u] = j < p.H ? (p.resid_in ? p.resid_in[(size_t)b * p.H + j] : bf16_bits_to_f32(xb[j])) : 0.f;
-    }
-#pragma unroll
-    for (int k = 0; k <= MOEQ_MAX_K; ++k) {
-      if (k <= p.K) {
-#pragma unroll
-        for (int u = 0; u < kCombineU; ++u) {
-          const int j = j0 + u * blockDim.x;
-          if (j < p.H) acc[u] += wk[k] * yb[(size_t)k * p.H + j];
-        }
-      }
-    }
-#pragma unroll
-    for (int u = 0; u < kCombineU; ++u) {
-      const int j = j0 + u * blockDim.x;
-      if (j0 == (int)threadIdx.x) keep[u] = acc[u];
-      if (j < p.H) {
-        rb[j] = acc[u];
-        ss += acc[u] * acc[u];
-      }
-    }
+    for (int k = 0; k <= MOEQ_MAX_K; ++k)
+      if (k <= p.K) acc += wk[k] * yb[(size_t)k * p.H + j];
+    if (j == j0 + (int)threadIdx.x) keep = acc;
+    rb[j] = acc;
+    ss += acc * acc;
   }
   if (p.xnorm) {
     ss = block_sum(ss, red);
-    const float inv = rsqrtf(ss / (float)p.H + p.eps);
-    uint16_t* xn = p.xnorm + (size_t)b * p.H;
-#pragma unroll
-    for (int u = 0; u < kCombineU; ++u) {
-      const int j = threadIdx.x + u * blockDim.x;
-      if (j < p.H) xn[j] = f32_to_bf16_bits(keep[u] * inv);
-    }
-    for (int j = threadIdx.x + stride; j < p.H; j += blockDim.x) xn[j] = f32_to_bf16_bits(rb[j] * inv);
+    if (threadIdx.x == 0) s_part = ss;
   }
+  cluster.sync();  // every CTA's part is in its shared memory
+  if (p.xnorm) {
+    float tot = 0.f;
+    for (int r = 0; r < kCombineCluster; ++r) tot += *cluster.map_shared_rank(&s_part, r);
+    const float inv = rsqrtf(tot / (float)p.H + p.eps);
+    uint16_t* xn = p.xnorm + (size_t)b * p.H;
+    for (int j = j0 + (int)threadIdx.x; j < j1; j += blockDim.x)
+      xn[j] = f32_to_bf16_bits((j == j0 + (int)threadIdx.x ? keep : rb[j]) * inv);
+  }
+  cluster.sync();  // peers' reads of this CTA's shared memory are done before it leaves
 }
 
 // moe_rmsnorm: grid B, one token per CTA. xn = bf16(r * rsqrt(mean(r^2) +

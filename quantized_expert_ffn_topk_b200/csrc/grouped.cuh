@@ -4,23 +4,18 @@
 // one token at a time).
 //
 //   k_group           stable counting sort of the (token, slot) picks by
-//                     expert id: cnt, off, list, and the work items (an
-//                     expert's entries in chunks of at most kGrpMaxTok)
+//                     expert id: cnt, off, list, and the active experts
 //   k_stage_batch     the input image of every token (x, or h per slot) in
 //                     the workspace, so that a tile can be applied to
 //                     several tokens without restaging
-//   k_ffn_grp<DOWN>   unit = (work item, tile). One CTA per SM: a copy warp
-//                     streams the CTA's units' tiles with bulk copies into a
-//                     ring of shared-memory slots; each compute warp takes a
-//                     piece = (unit, four of its tokens) and runs the whole
-//                     tile against those four tokens' images (four tokens
-//                     share each mma: columns 2t, 2t+1 carry token t's hi and
-//                     lo planes), so a lane ends with finished outputs and no
-//                     partial sums cross warps. gate/up: h per (token, slot);
-//                     down: y per (token, slot).
+//   k_gate_up_grp     unit = (expert, gate/up tile): the tile is read once;
+//                     four tokens share each mma (columns 2t, 2t+1 carry
+//                     token t's hi and lo planes); h per (token, slot)
+//   k_down_grp        unit = (expert, down tile): y per (token, slot)
 //
-// The work items of a step are [shared expert (every token, slot K),
-// routed chunks by expert id].
+// The work items of a step are [the shared expert's token chunks, the
+// active routed experts' chunks in increasing id]; the shared expert serves
+// every token (slot K).
 #pragma once
 
 #include "common.cuh"
@@ -29,16 +24,16 @@
 
 namespace moeq {
 
-constexpr int kGrpWarps = 15;                         // compute warps (one more copies tiles: 16 warps, 128 registers)
-constexpr int kGrpThreads = (kGrpWarps + 1) * 32;
-constexpr int kGrpMaxTok = 128;                       // entries of one work item at most
-constexpr int kGrpMaxPieces = kGrpMaxTok / 4;         // pieces of one unit at most
-constexpr int kGrpMaxSlots = 16;                      // ring slots
-static_assert(MOEQ_MAX_B <= kGrpMaxTok, "the shared expert's tokens are one work item");
+constexpr int kGrpWarps = 8;
+constexpr int kGrpCtasPerSm = 4;                   // resident CTAs per SM (64 registers a thread)
+constexpr int kGrpUnits = kGrpWarps / kFfnPieces;  // units per round (four warps each)
+constexpr int kGrpMaxTok = 64;                      // tokens of one work item at most
+constexpr int kGrpSharedItems = (MOEQ_MAX_B + kGrpMaxTok - 1) / kGrpMaxTok;  // the shared expert's work items at most
 
-// A routed expert with more than kGrpMaxTok entries (forced picks may repeat
-// an expert within a token) is split into several chunks; a chunk is one
-// work item.
+// A routed expert with more than kGrpMaxTok entries (popular experts of a
+// large batch, or forced picks that repeat an expert within a token) is split
+// into several chunks; a chunk is one work item. The shared expert serves
+// every token: ceil(B / kGrpMaxTok) work items of consecutive tokens.
 constexpr int kGrpExtraChunks = (MOEQ_MAX_B * MOEQ_MAX_K) / kGrpMaxTok;
 struct GrpWs {
   int* cnt;   // [E]
@@ -55,8 +50,8 @@ struct GrpParams {
   int img_stride;       // bytes between consecutive images
   int img_gs_off;       // byte offset of the gs array within an image
   int tps;              // tiles per expert (I/8 gate/up, H/16 down)
-  int max_units;        // (1 + most work items) * tps
-  int slot_bytes, nslot;  // ring of tile slots in dynamic shared memory
+  int max_units;        // (shared work items + most routed work items) * tps
+  int nsh;              // the shared expert's work items: ceil(B / kGrpMaxTok)
 };
 
 // ---- grouping -------------------------------------------------------------
@@ -182,218 +177,151 @@ __device__ __forceinline__ void ld_stream_words(const unsigned char* p, uint32_t
   }
 }
 
-// One whole tile in shared memory (nblk blocks) against four tokens' images
-// in global memory (imgs[c]; the lanes of column pair c read image c). Lane
-// (gid, t) accumulates token t: acc0 for local row gid, acc1 for row gid+8.
-// The images' fragments of the next P groups are loaded ahead (they come
-// from L2).
+// Blocks [0, nblk) of one tile in global memory against groups [g0, g0+nblk)
+// of up to four tokens' images (imgs[c], c < nt; the lanes of column pair c
+// read image c). Lane (gid, t) accumulates token t: acc0 for local row gid,
+// acc1 for row gid+8.
 template <int BITS, int KS>
-__device__ __forceinline__ void tile_dot_tokens(const unsigned char* tile, int nblk,
+__device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int nblk, int g0,
                                                 const unsigned char* const (&imgs)[4], int gs_off, float& acc0,
                                                 float& acc1) {
   using F = TileFmt<BITS, KS>;
-  constexpr int P = KS >= 4 ? 4 : 8;  // groups in flight (about 16 KB of fragments per warp)
+  constexpr int P = 2;  // blocks in flight per warp (four CTAs per SM keep the bytes in flight)
   const int lane = threadIdx.x & 31, gid = lane >> 2, t = lane & 3;
   // B fragments of column gid: token gid/2, plane hi (gid even) or lo
   const uint2* planes = reinterpret_cast<const uint2*>(imgs[gid >> 1]) + (gid & 1) * 4 + t;
   const float2* gs = reinterpret_cast<const float2*>(imgs[t] + gs_off);  // this lane's token
-  uint2 bf[P][KS];
-  float2 ms[P];
-#pragma unroll
-  for (int q = 0; q < P; ++q) {
-    const int g = min(q, nblk - 1);
-#pragma unroll
-    for (int ks = 0; ks < KS; ++ks) bf[q][ks] = __ldg(planes + (size_t)(g * KS + ks) * 8);
-    ms[q] = __ldg(gs + g);
-  }
   for (int b0 = 0; b0 < nblk; b0 += P) {
+    uint32_t w[P][F::NW];
+    uint2 sb[P], bf[P][KS];
+    float2 ms[P];
 #pragma unroll
     for (int q = 0; q < P; ++q) {
-      const int b = b0 + q;
-      if (b < nblk) {
-        const unsigned char* blk = tile + (size_t)b * F::BB;
-        uint32_t w[F::NW];
-        load_lane_codes<BITS, KS>(blk, lane, w);
-        const uint2 sb = *reinterpret_cast<const uint2*>(blk + F::CB + gid * 8);
-        int d[4];
+      const int b = min(b0 + q, nblk - 1);
+      const unsigned char* blk = blk0 + (size_t)b * F::BB;
+      ld_stream_words<F::LB>(blk + lane * F::LB, w[q]);
+      if (BITS == 3) ld_stream_words<F::LH>(blk + 32 * F::LB + lane * F::LH, w[q] + F::LB / 4);
+      sb[q] = ld_stream8(blk + F::CB + gid * 8);
+      const int g = g0 + b;
 #pragma unroll
-        for (int ks = 0; ks < KS; ++ks) {
-          uint32_t a[4];
-          extract_a<BITS, KS>(w, ks, a);
-          mma_u8s8(d, a, bf[q][ks], ks > 0);
-        }
-        const float p0 = (float)(d[0] * 256 + d[1]) * ms[q].x;
-        const float p1 = (float)(d[2] * 256 + d[3]) * ms[q].x;
-        acc0 = fmaf(__uint_as_float(sb.x << 16), p0, acc0);
-        acc0 = fmaf(__uint_as_float(sb.x & 0xFFFF0000u), ms[q].y, acc0);
-        acc1 = fmaf(__uint_as_float(sb.y << 16), p1, acc1);
-        acc1 = fmaf(__uint_as_float(sb.y & 0xFFFF0000u), ms[q].y, acc1);
-        const int nb = b + P;
-        if (nb < nblk) {
+      for (int ks = 0; ks < KS; ++ks) bf[q][ks] = __ldcg(planes + (size_t)(g * KS + ks) * 8);
+      ms[q] = __ldcg(gs + g);
+    }
 #pragma unroll
-          for (int ks = 0; ks < KS; ++ks) bf[q][ks] = __ldg(planes + (size_t)(nb * KS + ks) * 8);
-          ms[q] = __ldg(gs + nb);
-        }
+    for (int q = 0; q < P; ++q) {
+      if (b0 + q >= nblk) continue;
+      int d[4];
+#pragma unroll
+      for (int ks = 0; ks < KS; ++ks) {
+        uint32_t a[4];
+        extract_a<BITS, KS>(w[q], ks, a);
+        mma_u8s8(d, a, bf[q][ks], ks > 0);
       }
+      const float p0 = (float)(d[0] * 256 + d[1]) * ms[q].x;
+      const float p1 = (float)(d[2] * 256 + d[3]) * ms[q].x;
+      acc0 = fmaf(__uint_as_float(sb[q].x << 16), p0, acc0);
+      acc0 = fmaf(__uint_as_float(sb[q].x & 0xFFFF0000u), ms[q].y, acc0);
+      acc1 = fmaf(__uint_as_float(sb[q].y << 16), p1, acc1);
+      acc1 = fmaf(__uint_as_float(sb[q].y & 0xFFFF0000u), ms[q].y, acc1);
     }
   }
 }
 
-// A work item's tokens: (batch index, output slot) of its i-th entry. Work
-// item 0 is the shared expert (every token, slot K); work item a >= 1 is
-// chunk a-1 of a routed expert, whose entries b*K + k sit in list from
-// `start` on.
-struct GrpItem {
-  int a, ntok, start;
-};
-__device__ __forceinline__ GrpItem grp_item(const GrpParams& p, int a) {
-  if (a == 0) return GrpItem{0, p.f.B, 0};
-  const int* c = p.g.act + 3 * (a - 1);
-  return GrpItem{a, c[2], c[1]};
-}
-__device__ __forceinline__ int2 item_token(const GrpParams& p, const GrpItem& it, int i) {
-  if (it.a == 0) return make_int2(i, p.f.K);
-  const int ent = __ldg(p.g.list + it.start + i);
-  return make_int2(ent / p.f.K, ent % p.f.K);
+// Token i of work item a: its (batch index, output slot). a < nsh is the
+// shared expert (tokens a*kGrpMaxTok.., slot K); a >= nsh is chunk a-nsh of a
+// routed expert, whose entries b*K + k sit in list from act[1] on.
+__device__ __forceinline__ void unit_token(const GrpParams& p, int a, int i, int& b, int& k) {
+  if (a < p.nsh) {
+    b = a * kGrpMaxTok + i;
+    k = p.f.K;
+  } else {
+    const int ent = p.g.list[p.g.act[3 * (a - p.nsh) + 1] + i];
+    b = ent / p.f.K;
+    k = ent % p.f.K;
+  }
 }
 
 // ---- grouped gate/up and down -----------------------------------------------
 
 // DOWN == false: gate/up tiles against x images, h per (token, slot).
 // DOWN == true: down tiles against h images, y per (token, slot).
-// CTA c takes a contiguous share of the step's units; its copy warp fills the
-// ring in unit order and its compute warps take the units' pieces in turn
-// (piece j of the CTA's sequence goes to warp j % kGrpWarps). A slot is free
-// once every piece of its unit has arrived on its empty barrier (the first
-// piece arrives for the pieces the unit does not have). Every wait is
-// bounded: on a timeout the CTA records MOE_ERR_TIMEOUT, skips the rest of
-// its work and waits (bounded) for its copies in flight before it leaves.
 template <bool DOWN>
-__global__ void __launch_bounds__(kGrpThreads, 1) k_ffn_grp(const __grid_constant__ GrpParams p) {
-  extern __shared__ __align__(128) unsigned char ring[];
-  __shared__ __align__(8) uint64_t full_bar[kGrpMaxSlots], empty_bar[kGrpMaxSlots];
-  __shared__ int s_last[kGrpMaxSlots];
-  __shared__ volatile int s_abort;
+__global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpParams p) {
+  __shared__ float part[kGrpUnits][kFfnPieces][kGrpMaxTok][kTileRows];
+  __shared__ int s_tok[kGrpUnits][kGrpMaxTok][2];
   const FfnParams& f = p.f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  if (threadIdx.x == 0) {
-    for (int i = 0; i < p.nslot; ++i) {
-      mbar_init(&full_bar[i], 1);
-      mbar_init(&empty_bar[i], kGrpMaxPieces);
-      s_last[i] = -1;
-    }
-    s_abort = 0;
-    fence_mbar_init();
-  }
-  __syncthreads();
   pdl_wait();
-  const long long budget = wait_budget(f.ctrl);
-  const int nunits = min(p.max_units, (1 + p.g.nact[0]) * p.tps);
-  const int u_lo = (int)((long long)nunits * blockIdx.x / gridDim.x);
-  const int u_hi = (int)((long long)nunits * (blockIdx.x + 1) / gridDim.x);
-  auto unit_rec = [&](int a, const RecGeom*& g) -> const uint8_t* {
-    g = a == 0 ? &f.geo_s : &f.geo_r;
-    return a == 0 ? f.shared : f.experts + (size_t)p.g.act[3 * (a - 1)] * f.rec_r;
-  };
-
-  if (warp == kGrpWarps) {
-    // ---- copy warp: one tile per unit into the ring, in unit order ----
-    for (int u = u_lo; u < u_hi && !s_abort; ++u) {
-      const int seq = u - u_lo, slot = seq % p.nslot, fill = seq / p.nslot;
-      bool ok = true;
-      if (lane == 0) {
-        if (fill > 0) ok = mbar_wait(&empty_bar[slot], (uint32_t)((fill - 1) & 1), &s_abort, budget);
-        if (ok) {
-          const int a = u / p.tps, T = u % p.tps;
-          const RecGeom* g;
-          const uint8_t* rec = unit_rec(a, g);
-          const uint8_t* src = rec + (DOWN ? g->down_off + (size_t)T * g->D : (size_t)T * g->U);
-          const uint32_t bytes = DOWN ? g->D : g->U;
-          *reinterpret_cast<volatile int*>(&s_last[slot]) = seq;
-          mbar_arrive_expect_tx(&full_bar[slot], bytes);
-          bulk_g2s(ring + (size_t)slot * p.slot_bytes, src, bytes, &full_bar[slot]);
-        } else if (!s_abort) {
-          set_error(f.ctrl, MOE_ERR_TIMEOUT);
-          s_abort = 1;
-        }
-      }
-      __syncwarp();
-    }
-    // every copy issued must land before the CTA leaves (bounded)
-    if (lane < p.nslot) {
-      const int j = s_last[lane];
-      if (j >= 0) {
-        const long long t0 = clock64();
-        while (!mbar_try_wait(&full_bar[lane], (uint32_t)((j / p.nslot) & 1)) && clock64() - t0 < budget) {
-        }
+  const int nunits = min(p.max_units, (p.nsh + p.g.nact[0]) * p.tps);
+  const int u_end = nunits;
+  // rounds of kGrpUnits consecutive units, dealt to the CTAs in turn
+  for (int u0 = blockIdx.x * kGrpUnits; u0 < nunits; u0 += gridDim.x * kGrpUnits) {
+    // the units of this round and their token lists
+    int ntok[kGrpUnits];
+#pragma unroll
+    for (int r = 0; r < kGrpUnits; ++r) {
+      const int u = u0 + r;
+      ntok[r] = 0;
+      if (u < u_end) {
+        const int a = u / p.tps;
+        ntok[r] = a < p.nsh ? min(kGrpMaxTok, f.B - a * kGrpMaxTok) : p.g.act[3 * (a - p.nsh) + 2];
+        for (int i = threadIdx.x; i < ntok[r]; i += blockDim.x) unit_token(p, a, i, s_tok[r][i][0], s_tok[r][i][1]);
       }
     }
-  } else {
-    // ---- compute warps: pieces (unit, four tokens) in turn ----
-    int pc = 0;  // pieces of the CTA's units before unit u
-    GrpItem it{-1, 0, 0};
-    for (int u = u_lo; u < u_hi; ++u) {
+    __syncthreads();
+    const int r = warp / kFfnPieces, q = warp % kFfnPieces, u = u0 + r;
+    if (u < u_end) {
       const int a = u / p.tps, T = u % p.tps;
-      if (a != it.a) it = grp_item(p, a);  // a work item spans tps consecutive units
-      const int np = (it.ntok + 3) / 4;
-      const int first = (warp - pc % kGrpWarps + kGrpWarps) % kGrpWarps;  // this warp's first piece of the unit
-      const int seq = u - u_lo, slot = seq % p.nslot;
-      for (int c = first; c < np; c += kGrpWarps) {
-        // the four tokens' (batch index, slot): one L2 round trip, issued
-        // before the wait for the tile
-        int2 tok[4];
+      const bool routed = a >= p.nsh;
+      const RecGeom& g = routed ? f.geo_r : f.geo_s;
+      const uint8_t* rec = routed ? f.experts + (size_t)p.g.act[3 * (a - p.nsh)] * f.rec_r : f.shared;
+      const int ng = DOWN ? (int)g.ng_i : (int)g.ng_h;
+      const int g0 = piece_lo(q, ng), g1 = piece_lo(q + 1, ng);
+      const unsigned char* blk =
+          rec + (DOWN ? g.down_off + (size_t)T * g.D : (size_t)T * g.U) + (size_t)g0 * g.blk;
+      for (int c0 = 0; c0 < ntok[r]; c0 += 4) {
+        const unsigned char* imgs[4];
 #pragma unroll
-        for (int cc = 0; cc < 4; ++cc) tok[cc] = item_token(p, it, min(4 * c + cc, it.ntok - 1));
-        // wait until the copy warp has issued this fill, then for its bytes
-        bool ok = true;
-        if (lane == 0) {
-          const volatile int* last = s_last;
-          const long long t0 = clock64();
-          while (last[slot] != seq) {
-            if (s_abort || clock64() - t0 > budget) {
-              ok = false;
-              break;
-            }
-            __nanosleep(64);
-          }
-          ok = ok && mbar_wait(&full_bar[slot], (uint32_t)((seq / p.nslot) & 1), &s_abort, budget);
-          if (!ok && !s_abort) {
-            set_error(f.ctrl, MOE_ERR_TIMEOUT);
-            s_abort = 1;
-          }
+        for (int c = 0; c < 4; ++c) {
+          const int i = min(c0 + c, ntok[r] - 1);
+          const int src = DOWN ? s_tok[r][i][0] * (f.K + 1) + s_tok[r][i][1] : s_tok[r][i][0];
+          imgs[c] = p.img + (size_t)src * p.img_stride;
         }
-        ok = __shfl_sync(0xFFFFFFFFu, ok ? 1 : 0, 0) != 0;
-        if (ok) {
-          const unsigned char* imgs[4];
-#pragma unroll
-          for (int cc = 0; cc < 4; ++cc)
-            imgs[cc] = p.img + (size_t)(DOWN ? tok[cc].x * (f.K + 1) + tok[cc].y : tok[cc].x) * p.img_stride;
-          const RecGeom* g;
-          unit_rec(a, g);
-          const bool routed = a != 0;
-          const int nblk = DOWN ? (int)g->ng_i : (int)g->ng_h;
-          float acc0 = 0.f, acc1 = 0.f;
-          with_fmt(routed ? f.bits_r : f.bits_s, f.G, [&]<int BITS, int KS>() {
-            tile_dot_tokens<BITS, KS>(ring + (size_t)slot * p.slot_bytes, nblk, imgs, p.img_gs_off, acc0, acc1);
-          });
-          const int cc = lane & 3;
-          if (4 * c + cc < it.ntok) {
-            const int2 tk = cc == 0 ? tok[0] : (cc == 1 ? tok[1] : (cc == 2 ? tok[2] : tok[3]));
-            const int b = tk.x, k = tk.y, gid = lane >> 2;
-            if (DOWN) {
-              float* y = f.y + ((size_t)b * (f.K + 1) + k) * f.H + (size_t)T * kTileRows;
-              y[gid] = acc0;
-              y[gid + 8] = acc1;
-            } else {
-              f.h[((size_t)b * (f.K + 1) + k) * f.I + 8 * T + gid] = silu_f(acc0) * acc1;
-            }
-          }
+        float acc0 = 0.f, acc1 = 0.f;
+        with_fmt(routed ? f.bits_r : f.bits_s, f.G, [&]<int BITS, int KS>() {
+          tile_dot_tokens<BITS, KS>(blk, g1 - g0, g0, imgs, p.img_gs_off, acc0, acc1);
+        });
+        const int i = c0 + (lane & 3);
+        if (i < ntok[r]) {
+          part[r][q][i][lane >> 2] = acc0;
+          part[r][q][i][(lane >> 2) + 8] = acc1;
         }
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cnt(&empty_bar[slot], c == 0 ? (uint32_t)(kGrpMaxPieces - np + 1) : 1u);
       }
-      pc += np;
     }
+    __syncthreads();
+    // finish: gate/up -> h = silu(gate) * up for 8 units; down -> y rows
+#pragma unroll
+    for (int rr = 0; rr < kGrpUnits; ++rr) {
+      const int uu = u0 + rr;
+      if (uu >= u_end) continue;
+      const int T = uu % p.tps;
+      const int per = DOWN ? kTileRows : 8;
+      for (int j = threadIdx.x; j < ntok[rr] * per; j += blockDim.x) {
+        const int i = j / per, row = j % per;
+        const int b = s_tok[rr][i][0], k = s_tok[rr][i][1];
+        float s0 = 0.f, s1 = 0.f;
+#pragma unroll
+        for (int qq = 0; qq < kFfnPieces; ++qq) {
+          s0 += part[rr][qq][i][row];
+          if (!DOWN) s1 += part[rr][qq][i][row + 8];
+        }
+        if (DOWN)
+          f.y[((size_t)b * (f.K + 1) + k) * f.H + (size_t)T * kTileRows + row] = s0;
+        else
+          f.h[((size_t)b * (f.K + 1) + k) * f.I + 8 * T + row] = silu_f(s0) * s1;
+      }
+    }
+    __syncthreads();
   }
   pdl_trigger();
 }

@@ -167,15 +167,6 @@ int batch1_dot_fma() {
   return v;
 }
 
-// Ring of the grouped kernels: as many slots of one tile as fit (at least 2).
-bool grp_plan(size_t tile_bytes, int& slot_bytes, int& nslot, size_t& smem) {
-  const size_t budget = 227 * 1024 - 4 * 1024;  // the static barriers and flags are well under 4 KB
-  slot_bytes = (int)align_up(tile_bytes, 128);
-  nslot = (int)std::min<size_t>(kGrpMaxSlots, budget / (size_t)slot_bytes);
-  smem = (size_t)nslot * slot_bytes;
-  return nslot >= 2;
-}
-
 __global__ void k_ws_debug(WsCtrl* c, unsigned wait_us, int withhold_cta) {
   c->wait_us = wait_us;
   c->withhold_cta = withhold_cta;
@@ -439,15 +430,9 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     gp.g = GrpWs{reinterpret_cast<int*>((char*)ws + wl.cnt), reinterpret_cast<int*>((char*)ws + wl.off),
                  reinterpret_cast<int*>((char*)ws + wl.list), reinterpret_cast<int*>((char*)ws + wl.act),
                  reinterpret_cast<int*>((char*)ws + wl.nact)};
-    const int max_act = std::min(p.E, B * p.K) + kGrpExtraChunks;  // work items at most
-    const int ctas = num_sms();  // one CTA per SM: a ring of tile slots fills its shared memory
-    size_t gu_smem = 0, dn_smem = 0;
-    int gu_slot = 0, gu_nslot = 0, dn_slot = 0, dn_nslot = 0;
-    if (!grp_plan((size_t)std::max(p.geo_r.U, p.geo_s.U), gu_slot, gu_nslot, gu_smem) ||
-        !grp_plan((size_t)std::max(p.geo_r.D, p.geo_s.D), dn_slot, dn_nslot, dn_smem))
-      return MOE_ERR_UNSUPPORTED;
-    if (ensure_smem(k_ffn_grp<false>, gu_smem) != MOE_OK || ensure_smem(k_ffn_grp<true>, dn_smem) != MOE_OK)
-      return MOE_ERR_UNSUPPORTED;
+    const int max_act = std::min(p.E, B * p.K) + kGrpExtraChunks;  // routed work items at most
+    const int ctas = kGrpCtasPerSm * num_sms();
+    gp.nsh = (B + kGrpMaxTok - 1) / kGrpMaxTok;
     st = launch_pdl(k_group, dim3(1), dim3(256), (size_t)(p.E + 1) * 4, s, idx, B, p.K, p.E, p.H, gp.g, y_out,
                     p.ctrl);
     if (st != MOE_OK) return st;
@@ -460,10 +445,8 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     gp.img_stride = wl.ximg_stride;
     gp.img_gs_off = wl.ximg_gs;
     gp.tps = p.I / 8;
-    gp.max_units = (1 + max_act) * gp.tps;
-    gp.slot_bytes = gu_slot;
-    gp.nslot = gu_nslot;
-    st = launch_pdl(k_ffn_grp<false>, dim3(ctas), dim3(kGrpThreads), gu_smem, s, gp);
+    gp.max_units = (gp.nsh + max_act) * gp.tps;
+    st = launch_pdl(k_ffn_grp<false>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
     if (st != MOE_OK) return st;
     st = launch_pdl(k_stage_batch, dim3(B, p.K + 1), dim3(256), 0, s, (const void*)p.h, 1, p.I, p.G, himg,
                     wl.himg_stride, wl.himg_gs);
@@ -472,10 +455,8 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     gp.img_stride = wl.himg_stride;
     gp.img_gs_off = wl.himg_gs;
     gp.tps = p.H / kTileRows;
-    gp.max_units = (1 + max_act) * gp.tps;
-    gp.slot_bytes = dn_slot;
-    gp.nslot = dn_nslot;
-    return launch_pdl(k_ffn_grp<true>, dim3(ctas), dim3(kGrpThreads), dn_smem, s, gp);
+    gp.max_units = (gp.nsh + max_act) * gp.tps;
+    return launch_pdl(k_ffn_grp<true>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
   }
 
   // one token: every CTA bulk-copies its share of whole tiles into shared memory
@@ -511,7 +492,7 @@ moe_status moe_combine_residual(const moe_layer_q* L, const float* y, const floa
   p.H = L->H;
   p.K = L->K;
   p.eps = eps;
-  return launch_pdl(k_combine, dim3(B), dim3(kCombineThreads), 0, (cudaStream_t)stream, p);
+  return launch_pdl(k_combine, dim3(B * kCombineCluster), dim3(kCombineThreads), 0, (cudaStream_t)stream, p);
 }
 
 moe_status moe_get_device_error(void* ws, void* stream) {
@@ -574,20 +555,39 @@ bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes) {
   return true;
 }
 
-// Static shared memory of the fused decode kernel (bytes), read once.
-size_t stack_static_smem() {
-  static size_t bytes = 0;
-  if (bytes == 0) {
-    cudaFuncAttributes fa{};
-    if (cudaFuncGetAttributes(&fa, k_decode_layers) == cudaSuccess) bytes = fa.sharedSizeBytes;
-    else (void)cudaGetLastError();
-    if (bytes == 0) bytes = 16 * 1024;  // unknown: leave a generous margin
-  }
-  return bytes;
+// The fused kernel's instance for (routed bits, shared bits, group):
+// shared experts at 4 bits or at the routed width. Null when there is none.
+using StackKernel = void (*)(StackParams);
+StackKernel stack_kernel(int br, int bs, int G) {
+#define MOEQ_STACK_CASE(R, S, Gp, KS) \
+  if (br == R && bs == S && G == Gp) return k_decode_layers<R, S, KS>;
+#define MOEQ_STACK_GROUPS(R, S)  \
+  MOEQ_STACK_CASE(R, S, 64, 2)   \
+  MOEQ_STACK_CASE(R, S, 128, 4)
+  MOEQ_STACK_GROUPS(4, 4)
+  MOEQ_STACK_GROUPS(2, 4)
+  MOEQ_STACK_GROUPS(3, 4)
+  MOEQ_STACK_GROUPS(2, 2)
+  MOEQ_STACK_GROUPS(3, 3)
+  MOEQ_STACK_CASE(4, 4, 32, 1)
+  MOEQ_STACK_CASE(2, 4, 32, 1)
+  MOEQ_STACK_CASE(2, 2, 32, 1)
+#undef MOEQ_STACK_GROUPS
+#undef MOEQ_STACK_CASE
+  return nullptr;
+}
+
+// Static shared memory of a fused-kernel instance (bytes).
+size_t stack_static_smem(StackKernel kern) {
+  cudaFuncAttributes fa{};
+  size_t bytes = 0;
+  if (cudaFuncGetAttributes(&fa, kern) == cudaSuccess) bytes = fa.sharedSizeBytes;
+  else (void)cudaGetLastError();
+  return bytes ? bytes : 16 * 1024;  // unknown: leave a generous margin
 }
 
 // Shared-memory plan of the fused decode kernel; false when it does not fit.
-bool stack_plan(StackParams& p, int G) {
+bool stack_plan(StackParams& p, int G, size_t static_smem) {
   const int H = p.H, I = p.I, K = p.K;
   size_t o = 0;
   auto take = [&](size_t bytes) {
@@ -603,9 +603,7 @@ bool stack_plan(StackParams& p, int G) {
   p.hgs_stride = (int)align_up(qimg_gs_bytes(I, p.G), 128);
   p.sm_hplanes = take((size_t)p.hplanes_stride * (K + 1));
   p.sm_hgs = take((size_t)p.hgs_stride * (K + 1));
-  const int nw = std::min(kMaxWaves, K);
-  int ntiles_max = cdiv(I / 8, G) + 1;
-  for (int w = 0; w < nw; ++w) ntiles_max += cdiv(((w + 1) * K / nw - w * K / nw) * (I / 8), G);
+  const int ntiles_max = cdiv(I / 8, G) + cdiv(K * (I / 8), G) + 1;
   const int nd_max = cdiv(H / kTileRows, G);
   if (ntiles_max > kMaxTiles || nd_max > kMaxDnTiles) return false;
   p.sm_gpart = take((size_t)ntiles_max * kGuPieces * kTileRows * 4);
@@ -617,7 +615,7 @@ bool stack_plan(StackParams& p, int G) {
                            std::max(p.geo_r.blk, p.geo_s.blk);
   const size_t down_item = (size_t)nd_max * std::max(p.geo_r.D, p.geo_s.D);
   p.slot_bytes = (int)align_up(std::max(std::max((size_t)2 * H * 2, half_tile), down_item), 128);
-  const size_t budget = 227 * 1024 - align_up(stack_static_smem(), 1024);  // room for the static shared memory
+  const size_t budget = 227 * 1024 - align_up(static_smem, 1024);  // room for the static shared memory
   if (o + (size_t)p.slot_bytes * 2 > budget) return false;
   p.nslot = (int)std::min<size_t>(kMaxSlots, (budget - o) / p.slot_bytes);
   p.sm_ring = take((size_t)p.slot_bytes * p.nslot);
@@ -654,12 +652,8 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   auto cdiv = [](int a, int b) { return (a + b - 1) / b; };
   if (L0.E > kStackMaxE || cdiv(L0.E, G) > kMaxRouterRowsPerCta || G > kStackMaxCtas) return MOE_ERR_UNSUPPORTED;
   const int tps = L0.I / 8;
-  {
-    const int nw = std::min(kMaxWaves, L0.K);
-    int gu = cdiv(tps, G);
-    for (int w = 0; w < nw; ++w) gu += cdiv(((w + 1) * L0.K / nw - w * L0.K / nw) * tps, G);
-    if (cdiv(cdiv(L0.E, G), 2) + 2 * gu + L0.K + 1 > kMaxItems) return MOE_ERR_UNSUPPORTED;
-  }
+  if (cdiv(cdiv(L0.E, G), 2) + 2 * (cdiv(tps, G) + cdiv(L0.K * tps, G) + 1) + L0.K + 1 > kMaxItems)
+    return MOE_ERR_UNSUPPORTED;
   if (L0.H % 32 != 0 || L0.H / 16 > kCThreads) return MOE_ERR_UNSUPPORTED;
 
   StackParams p{};
@@ -703,9 +697,24 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
 #else
   p.trace = nullptr;
 #endif
-  if (!stack_plan(p, G)) return MOE_ERR_UNSUPPORTED;
+  const StackKernel kern = stack_kernel(p.bits_r, p.bits_s, p.G);
+  if (!kern) return MOE_ERR_UNSUPPORTED;
+  static std::mutex mu;
+  static size_t static_smem[64] = {};  // per instance, read once (the instances' addresses are fixed)
+  static StackKernel seen[64] = {};
+  size_t ss = 0;
+  std::unique_lock<std::mutex> lock(mu);
+  for (int i = 0; i < 64 && !ss; ++i) {
+    if (seen[i] == kern) ss = static_smem[i];
+    else if (!seen[i]) {
+      seen[i] = kern;
+      ss = static_smem[i] = stack_static_smem(kern);
+    }
+  }
+  lock.unlock();
+  if (!stack_plan(p, G, ss ? ss : 16 * 1024)) return MOE_ERR_UNSUPPORTED;
   const size_t smem = stack_smem_bytes(p);
-  if (ensure_smem(k_decode_layers, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;
+  if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;
 
   cudaLaunchConfig_t cfg = {};
   cfg.gridDim = dim3(G);
@@ -717,7 +726,7 @@ extern "C" moe_status moe_decode_layers(const moe_layer_q* layers, int n_layers,
   attr[0].val.cooperative = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 1;
-  if (cudaLaunchKernelEx(&cfg, k_decode_layers, p) != cudaSuccess) {
+  if (cudaLaunchKernelEx(&cfg, kern, p) != cudaSuccess) {
     (void)cudaGetLastError();
     return MOE_ERR_CUDA;
   }

@@ -54,16 +54,8 @@ constexpr int kMaxPieces = kMaxItems * kItemPieces;
 constexpr int kMaxTiles = 16;                    // gate/up tiles per CTA per layer
 constexpr int kStackMaxCtas = 1024;              // CTAs of the grid at most (partial sums in the workspace)
 constexpr int kStackMaxE = 1024;                 // experts at most (two logits per compute thread)
-// The routed experts' h is exchanged in waves of slots: a CTA works the
-// gate/up tiles of wave 0, publishes them, works wave 1 while wave 0's
-// exchange completes, and only then waits for wave 0's h to run its down
-// tiles, so the exchange of one wave overlaps the work of the next.
-#ifndef MOEQ_ROUTED_WAVES
-#define MOEQ_ROUTED_WAVES 2
-#endif
-constexpr int kMaxWaves = MOEQ_ROUTED_WAVES;
-// counters in the workspace: logits, shared h, routed h per wave, r
-enum { kSyncLogits = 0, kSyncSharedH = 1, kSyncRoutedH = 2, kSyncResid = kSyncRoutedH + kMaxWaves, kNumSync };
+// counters in the workspace: logits, shared h, routed h, r
+enum { kSyncLogits = 0, kSyncSharedH = 1, kSyncRoutedH = 2, kSyncResid = 3, kNumSync };
 static_assert(kNumSync <= 8, "arrival counters of the control block");
 
 enum { kItemRouter = 0, kItemGateUp = 1, kItemDown = 2 };
@@ -106,7 +98,7 @@ struct StackParams {
 // Optional phase timeline (compiled in with -DMOEQ_STACK_TRACE only): one
 // thread per CTA stamps %globaltimer at phase ends into
 // trace[(layer * kTracePhases + phase) * G + cta]. Off in the library build.
-constexpr int kTracePhases = 14;
+constexpr int kTracePhases = 17;  // 14, 15: first/last routed gate/up item landed; 16: longest such piece (ns)
 #ifdef MOEQ_STACK_TRACE
 #define STACK_MARK(cond, l, ph)                                                                    \
   do {                                                                                             \
@@ -132,11 +124,7 @@ struct ItemPlan {
   int n_items, n_router_items, n_sgu_items, n_pre_items, n_rgu_items;  // item ranges, in ring order:
   // [0, n_router_items) router, [.., n_sgu_items) shared gate/up, [.., n_pre_items)
   // shared down (all three issued during the previous layer), [.., n_rgu_items)
-  // routed gate/up (wave by wave: wave w ends at gu_end[w]), [.., n_items) routed
-  // down (wave w ends at dn_end[w])
-  int nwaves;
-  int wave_k0[kMaxWaves + 1];              // wave w holds slots [wave_k0[w], wave_k0[w+1])
-  int gu_end[kMaxWaves], dn_end[kMaxWaves];
+  // routed gate/up, [.., n_items) routed down
   int n_pieces, n_router_pieces, n_pre_pieces;
   int kind[kMaxItems];
   int k[kMaxItems];                        // slot (K: shared)
@@ -201,19 +189,10 @@ __device__ void make_plan(const StackParams& p, ItemPlan& P) {
   if (P.nd > 0) add_down(p.K);
   P.n_pre_items = n;
   P.n_pre_pieces = pc;
-  P.nwaves = min(kMaxWaves, p.K);
-  for (int w = 0; w <= P.nwaves; ++w) P.wave_k0[w] = w * p.K / P.nwaves;
-  for (int w = 0; w < P.nwaves; ++w) {
-    const int k0 = P.wave_k0[w], nwt = (P.wave_k0[w + 1] - k0) * tps;
-    for (int u = share_lo(c, G, nwt); u < share_lo(c + 1, G, nwt); ++u) add_tile(k0 + u / tps, u % tps);
-    P.gu_end[w] = n;
-  }
+  for (int u = share_lo(c, G, p.K * tps); u < share_lo(c + 1, G, p.K * tps); ++u) add_tile(u / tps, u % tps);
   P.n_rgu_items = n;
-  for (int w = 0; w < P.nwaves; ++w) {
-    if (P.nd > 0)
-      for (int k = P.wave_k0[w]; k < P.wave_k0[w + 1]; ++k) add_down(k);
-    P.dn_end[w] = n;
-  }
+  if (P.nd > 0)
+    for (int k = 0; k < p.K; ++k) add_down(k);
   P.n_items = n;
   P.n_pieces = pc;
   P.ntiles = tl;
@@ -433,6 +412,22 @@ __device__ __forceinline__ bool flag_wait(const volatile int* f, int target, con
   return true;
 }
 
+// The sum of the G CTAs' published partial sums of squares, in one fixed
+// order (lane j adds entries j, j+32, ... then a butterfly over the lanes), so
+// every warp of every CTA gets the same value. The loads are all issued
+// before the first add (one L2 round trip for G <= 256).
+__device__ __forceinline__ float sum_partials(const float* part, int G) {
+  const int lane = threadIdx.x & 31;
+  float v[8];
+#pragma unroll
+  for (int j = 0; j < 8; ++j) v[j] = lane + 32 * j < G ? __ldcg(part + lane + 32 * j) : 0.f;
+  float s = 0.f;
+#pragma unroll
+  for (int j = 0; j < 8; ++j) s += v[j];
+  for (int c = lane + 256; c < G; c += 32) s += __ldcg(part + c);
+  return warp_sum(s);
+}
+
 // ---- compute pieces ------------------------------------------------------------
 
 // Bounded wait until the producer has issued ring sequence number seq into
@@ -455,6 +450,9 @@ __device__ __forceinline__ QImg stack_himg(unsigned char* sm, const StackParams&
               reinterpret_cast<float2*>(sm + p.sm_hgs + (size_t)k * p.hgs_stride)};
 }
 
+// One kernel per format (BR bits routed, BS bits shared, KS k-steps per
+// group): the host picks the instance for the layers' widths and group.
+template <int BR, int BS, int KS>
 __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid_constant__ StackParams p) {
   extern __shared__ __align__(128) unsigned char sm[];
   __shared__ __align__(8) uint64_t full_bar[kMaxSlots], empty_bar[kMaxSlots];
@@ -470,6 +468,14 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
   __shared__ volatile int s_abort;
   __shared__ volatile int s_topk_ready;
   __shared__ volatile int s_logits_ready;  // layer + 1 once s_logits holds that layer's logits
+#ifdef MOEQ_STACK_TRACE
+  __shared__ unsigned long long s_tr[3];
+  if (threadIdx.x == 0) {
+    s_tr[0] = ~0ull;
+    s_tr[1] = 0ull;
+    s_tr[2] = 0ull;
+  }
+#endif
   __shared__ __align__(16) float s_logits[kStackMaxE];
 
   const int tid = threadIdx.x, warp = tid >> 5, lane = tid & 31;
@@ -568,6 +574,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       bool ok = slot_issued(s_last, slot, (int)seq, &s_abort, budget);
       ok = ok && mbar_wait(&full_bar[slot], (seq / p.nslot) & 1, &s_abort, budget);
       if (!ok && lane == 0 && !s_abort) fail();
+#ifdef MOEQ_STACK_TRACE
+      unsigned long long t_landed = 0;
+      const bool traced = it >= P.n_pre_items && it < P.n_rgu_items;
+      if (traced && lane == 0) {
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_landed));
+        atomicMin(&s_tr[0], t_landed);
+        atomicMax(&s_tr[1], t_landed);
+      }
+#endif
       const unsigned char* sl = ring + (size_t)slot * p.slot_bytes;
       if (P.kind[it] == kItemRouter) {
         const int row = pos / kRouterPieces, qr = pos % kRouterPieces;
@@ -588,8 +603,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         if (ok && (!routed || s_idx[k] >= 0)) {
           const unsigned char* blk = sl + (size_t)j * g.D + (size_t)g0 * g.blk;
           const QImg Hk = stack_himg(sm, p, k);
-          with_fmt(routed ? p.bits_r : p.bits_s, p.G,
-                   [&]<int BITS, int KS>() { tile_dot<BITS, KS>(blk, g1 - g0, g0, Hk, acc0, acc1); });
+          with_fixed_fmt<BR, BS, KS>(
+              routed, [&]<int BITS, int KS_>() { tile_dot<BITS, KS_>(blk, g1 - g0, g0, Hk, acc0, acc1); });
         }
         if ((lane & 3) == 0) {
           float* dp = dpart + (((size_t)j * (K + 1) + k) * kDnPieces + q) * kTileRows;
@@ -606,8 +621,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         float acc0 = 0.f, acc1 = 0.f;
         if (valid) {
           const unsigned char* blk = sl + (size_t)(g0 - ga) * g.blk;
-          with_fmt(routed ? p.bits_r : p.bits_s, p.G,
-                   [&]<int BITS, int KS>() { tile_dot<BITS, KS>(blk, g1 - g0, g0, X, acc0, acc1); });
+          with_fixed_fmt<BR, BS, KS>(
+              routed, [&]<int BITS, int KS_>() { tile_dot<BITS, KS_>(blk, g1 - g0, g0, X, acc0, acc1); });
         }
         float* gp = gpart + ((size_t)tl * kGuPieces + q) * kTileRows;
         if ((lane & 3) == 0) {
@@ -636,6 +651,13 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         }
       }
       __syncwarp();
+#ifdef MOEQ_STACK_TRACE
+      if (traced && lane == 0) {
+        unsigned long long t_done;
+        asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_done));
+        atomicMax(&s_tr[2], t_done - t_landed);
+      }
+#endif
       if (lane == 0) {
         const uint32_t cnt = (pos == 0) ? (uint32_t)(kItemPieces - P.npieces[it] + 1) : 1u;
         mbar_arrive_cnt(&empty_bar[slot], cnt);
@@ -688,10 +710,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
           // the RMS norm's sum of squares from the CTAs' published partial
           // sums, in one fixed order (every warp of every CTA gets the same
           // value), read in the same round trip as r
-          float part = 0.f;
-          for (int c = lane; c < G; c += 32) part += __ldcg(p.ss_part + c);
           if (active) load_f32_16_cg(p.r + (size_t)tid * 16, v);
-          const float inv_norm = rsqrtf(warp_sum(part) / (float)H + p.eps);
+          const float inv_norm = rsqrtf(sum_partials(p.ss_part, G) / (float)H + p.eps);
           if (active) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = bf16_bits_to_f32(f32_to_bf16_bits(v[j] * inv_norm));
@@ -765,21 +785,28 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       run_items(l, P.n_sgu_items, P.n_pre_items);
       STACK_MARK(tid == 0, l, 8);
 
-      // ---- routed gate/up pieces, wave by wave, each wave's h published ----
-      for (int w = 0; w < P.nwaves; ++w) {
-        run_items(l, w == 0 ? P.n_pre_items : P.gu_end[w - 1], P.gu_end[w]);
-        named_sync(1, kCThreads);
-        if (tid == 0) arrive_release_gpu(p.sync + kSyncRoutedH + w);
-      }
+      // ---- routed gate/up pieces ----
+      run_items(l, P.n_pre_items, P.n_rgu_items);
+      named_sync(1, kCThreads);
+      if (tid == 0) arrive_release_gpu(p.sync + kSyncRoutedH);
       STACK_MARK(tid == 0, l, 9);
-
-      // ---- routed down tiles, wave by wave once the wave's h is out ----
-      for (int w = 0; w < P.nwaves; ++w) {
-        stage_h(P.wave_k0[w], P.wave_k0[w + 1], kSyncRoutedH + w, (unsigned)(l + 1) * G1);
-        named_sync(1, kCThreads);
-        if (w == 0) STACK_MARK(tid == 0, l, 10);
-        run_items(l, w == 0 ? P.n_rgu_items : P.dn_end[w - 1], P.dn_end[w]);
+#ifdef MOEQ_STACK_TRACE
+      if (tid == 0 && p.trace) {
+        const size_t at = (size_t)l * kTracePhases * gridDim.x + blockIdx.x;
+        p.trace[at + (size_t)14 * gridDim.x] = s_tr[0];
+        p.trace[at + (size_t)15 * gridDim.x] = s_tr[1];
+        p.trace[at + (size_t)16 * gridDim.x] = s_tr[2];
+        s_tr[0] = ~0ull;
+        s_tr[1] = 0ull;
+        s_tr[2] = 0ull;
       }
+#endif
+
+      // ---- routed down tiles ----
+      stage_h(0, K, kSyncRoutedH, (unsigned)(l + 1) * G1);
+      named_sync(1, kCThreads);
+      STACK_MARK(tid == 0, l, 10);
+      run_items(l, P.n_rgu_items, n_items);
       named_sync(1, kCThreads);
       STACK_MARK(tid == 0, l, 11);
 
@@ -820,8 +847,8 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       if (tid == 0 && !counter_wait(p.sync + kSyncResid, (unsigned)p.n_layers * G1, &s_abort, budget) && !s_abort) fail();
       named_sync(1, kCThreads);
       (void)nseg;
-      for (int c = lane; c < G; c += 32) ss += __ldcg(p.ss_part + c);
-      const float inv = rsqrtf(warp_sum(ss) / (float)H + p.eps);
+      (void)ss;
+      const float inv = rsqrtf(sum_partials(p.ss_part, G) / (float)H + p.eps);
       if (my_row >= 0) p.xnorm_out[my_row] = f32_to_bf16_bits(my_r * inv);
     }
   }

@@ -249,6 +249,12 @@ __device__ __forceinline__ void block_acc(const uint32_t* w, uint2 sb, int g, co
   acc1 = fmaf(__uint_as_float(sb.y & 0xFFFF0000u), ms.y, acc1);
 }
 
+// Groups of a tile dot whose loads and mma chains the compiler interleaves.
+#ifndef MOEQ_TILE_UNROLL
+#define MOEQ_TILE_UNROLL 2
+#endif
+constexpr int kTileUnroll = MOEQ_TILE_UNROLL;
+
 // Blocks [0, nblk) of one tile in shared memory (at blk0, consecutive)
 // against groups [g0, g0+nblk) of image X. Every lane of a row quad ends with
 // the same values.
@@ -257,7 +263,7 @@ __device__ __forceinline__ void tile_dot(const unsigned char* blk0, int nblk, in
                                          float& acc1) {
   using F = TileFmt<BITS, KS>;
   const int lane = threadIdx.x & 31;
-#pragma unroll 2
+#pragma unroll kTileUnroll
   for (int b = 0; b < nblk; ++b) {
     const unsigned char* blk = blk0 + (size_t)b * F::BB;
     uint32_t w[F::NW];
@@ -341,6 +347,15 @@ __device__ __forceinline__ void with_fmt(int bits, int G, Fn fn) {
     else if (G == 64) fn.template operator()<2, 2>();
     else fn.template operator()<2, 4>();
   }
+}
+
+// The same dispatch with the widths fixed at compile time (a kernel built
+// for routed experts at BR bits, the shared expert at BS bits, KS k-steps
+// per group): only the two formats in use are compiled into it.
+template <int BR, int BS, int KS, typename Fn>
+__device__ __forceinline__ void with_fixed_fmt(bool routed, Fn fn) {
+  if (routed) fn.template operator()<BR, KS>();
+  else fn.template operator()<BS, KS>();
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
