@@ -25,7 +25,14 @@
 namespace moeq {
 
 constexpr int kGrpWarps = 8;
-constexpr int kGrpCtasPerSm = 4;                   // resident CTAs per SM (64 registers a thread)
+#ifndef MOEQ_GRP_CTAS
+#define MOEQ_GRP_CTAS 4
+#endif
+#ifndef MOEQ_GRP_INFLIGHT
+#define MOEQ_GRP_INFLIGHT 2
+#endif
+constexpr int kGrpCtasPerSm = MOEQ_GRP_CTAS;        // resident CTAs per SM (64 registers a thread at 4)
+constexpr int kGrpInFlight = MOEQ_GRP_INFLIGHT;     // blocks whose loads a warp keeps in flight
 constexpr int kGrpUnits = kGrpWarps / kFfnPieces;  // units per round (four warps each)
 constexpr int kGrpMaxTok = 64;                      // tokens of one work item at most
 constexpr int kGrpSharedItems = (MOEQ_MAX_B + kGrpMaxTok - 1) / kGrpMaxTok;  // the shared expert's work items at most
@@ -186,7 +193,7 @@ __device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int n
                                                 const unsigned char* const (&imgs)[4], int gs_off, float& acc0,
                                                 float& acc1) {
   using F = TileFmt<BITS, KS>;
-  constexpr int P = 2;  // blocks in flight per warp (four CTAs per SM keep the bytes in flight)
+  constexpr int P = kGrpInFlight;
   const int lane = threadIdx.x & 31, gid = lane >> 2, t = lane & 3;
   // B fragments of column gid: token gid/2, plane hi (gid even) or lo
   const uint2* planes = reinterpret_cast<const uint2*>(imgs[gid >> 1]) + (gid & 1) * 4 + t;

@@ -258,9 +258,14 @@ constexpr int kTileUnroll = MOEQ_TILE_UNROLL;
 // Blocks [0, nblk) of one tile in shared memory (at blk0, consecutive)
 // against groups [g0, g0+nblk) of image X. Every lane of a row quad ends with
 // the same values.
+#ifdef MOEQ_TILE_NOINLINE
+#define MOEQ_TILE_INLINE __noinline__
+#else
+#define MOEQ_TILE_INLINE __forceinline__
+#endif
 template <int BITS, int KS>
-__device__ __forceinline__ void tile_dot(const unsigned char* blk0, int nblk, int g0, const QImg& X, float& acc0,
-                                         float& acc1) {
+__device__ MOEQ_TILE_INLINE void tile_dot(const unsigned char* blk0, int nblk, int g0, const QImg& X, float& acc0,
+                                          float& acc1) {
   using F = TileFmt<BITS, KS>;
   const int lane = threadIdx.x & 31;
 #pragma unroll kTileUnroll
@@ -354,8 +359,12 @@ __device__ __forceinline__ void with_fmt(int bits, int G, Fn fn) {
 // per group): only the two formats in use are compiled into it.
 template <int BR, int BS, int KS, typename Fn>
 __device__ __forceinline__ void with_fixed_fmt(bool routed, Fn fn) {
-  if (routed) fn.template operator()<BR, KS>();
-  else fn.template operator()<BS, KS>();
+  if (BR == BS) {
+    fn.template operator()<BR, KS>();  // one copy of the code when both widths agree
+  } else {
+    if (routed) fn.template operator()<BR, KS>();
+    else fn.template operator()<BS, KS>();
+  }
 }
 
 __device__ __forceinline__ float silu_f(float z) { return z / (1.0f + __expf(-z)); }
