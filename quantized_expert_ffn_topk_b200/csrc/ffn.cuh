@@ -35,7 +35,7 @@ struct FfnParams {
   // shared-memory plans of the one-token kernels (byte offsets)
   int gu_nbuf, gu_gs, gu_part, gu_tiles, gu_stride;
   int dn_nbuf, dn_img_stride, dn_img_gs, dn_part, dn_tiles, dn_stride;
-  int dn_ctas;  // CTAs of the down kernel (its shares are prefetched into L2 by the gate/up kernel)
+  int dn_ctas;  // CTAs of the down kernel
   // 1: the dots run on the CUDA cores in fp32 (tile_dot_fma) on fp32 copies
   // of the inputs at gu_xf / (image) + dn_img_xf, for comparison with the
   // tensor-core dot (0, the default)
@@ -134,23 +134,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
       if (r0 == t_lo) ffn_issue(tiles, p.gu_stride, bar, r0, nt, src, is_routed);
       else ffn_issue(tiles, p.gu_stride, bar, r0, nt, src, any);
     }
-#ifndef MOEQ_NO_DOWN_PREFETCH
-    if (r0 == t_lo && warp == 1 && blockIdx.x < p.dn_ctas) {
-      // the down kernel's share for this CTA index, pulled into L2 now so
-      // that its bytes stream while the gate/up tiles are worked (the down
-      // kernel cannot start on this SM before this kernel leaves it)
-      const int tpd = p.H / kTileRows, dtot = (p.K + 1) * tpd;
-      const int d_lo = (int)((long long)dtot * blockIdx.x / p.dn_ctas);
-      const int d_hi = (int)((long long)dtot * (blockIdx.x + 1) / p.dn_ctas);
-      for (int u = d_lo + lane; u < d_hi; u += 32) {
-        const int k = u / tpd, T = u % tpd;
-        const uint8_t* rec = ffn_slot_rec(p, k);
-        if (!rec) continue;
-        const RecGeom& g = k < p.K ? p.geo_r : p.geo_s;
-        prefetch_l2(rec + g.down_off + (size_t)T * g.D, g.D);
-      }
-    }
-#endif
+
     if (r0 == t_lo) {  // the input image, while the first round's tiles are in flight
       float* xf = reinterpret_cast<float*>(smem + p.gu_xf);
       qstage_vector(

@@ -67,7 +67,7 @@ struct GrpParams {
 // group, and get a zero output slot here.
 __global__ void __launch_bounds__(256) k_group(const int32_t* idx, int B, int K, int E, int H, GrpWs g, float* y,
                                                WsCtrl* ctrl) {
-  extern __shared__ int s_cnt[];  // [E + 1]
+  extern __shared__ int s_cnt[];  // [max(E + 1, B*K)]: counts, then the picks
   pdl_wait();
   const int n = B * K;
   for (int e = threadIdx.x; e <= E; e += blockDim.x) s_cnt[e] = 0;
@@ -134,11 +134,17 @@ __global__ void __launch_bounds__(256) k_group(const int32_t* idx, int B, int K,
     g.nact[0] = tk;
   }
   __syncthreads();
+  // each entry's rank among the earlier entries of its expert (a stable
+  // order), from a copy of the picks in the shared memory the counts used
+  // (sized for max(E + 1, B*K) ints by the host)
+  int* s_idx = s_cnt;
+  for (int i = threadIdx.x; i < n; i += blockDim.x) s_idx[i] = idx[i];
+  __syncthreads();
   for (int i = threadIdx.x; i < n; i += blockDim.x) {
-    const int e = idx[i];
+    const int e = s_idx[i];
     if (e < 0 || e >= E) continue;
     int r = 0;
-    for (int j = 0; j < i; ++j) r += idx[j] == e;
+    for (int j = 0; j < i; ++j) r += s_idx[j] == e;
     g.list[g.off[e] + r] = i;
   }
   pdl_trigger();

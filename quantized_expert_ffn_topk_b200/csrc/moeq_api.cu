@@ -433,7 +433,8 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     const int max_act = std::min(p.E, B * p.K) + kGrpExtraChunks;  // routed work items at most
     const int ctas = kGrpCtasPerSm * num_sms();
     gp.nsh = (B + kGrpMaxTok - 1) / kGrpMaxTok;
-    st = launch_pdl(k_group, dim3(1), dim3(256), (size_t)(p.E + 1) * 4, s, idx, B, p.K, p.E, p.H, gp.g, y_out,
+    st = launch_pdl(k_group, dim3(1), dim3(256), (size_t)std::max(p.E + 1, B * p.K) * 4, s, idx, B, p.K, p.E, p.H, gp.g,
+                    y_out,
                     p.ctrl);
     if (st != MOE_OK) return st;
     unsigned char* ximg = reinterpret_cast<unsigned char*>(ws) + wl.ximg;

@@ -125,18 +125,35 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterPara
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [tok_tile, H]
   __shared__ int s_last;
+  __shared__ __align__(8) uint64_t s_bar;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gwarp = blockIdx.x * kRouterWarps + warp, nwarps = gridDim.x * kRouterWarps;
   const int nvec = p.H / 8;  // 16-byte words per row
   const int b0 = blockIdx.y * kRouterTokTile, tb = min(kRouterTokTile, p.B - b0);
 
+  if (threadIdx.x == 0) {
+    mbar_init(&s_bar, 1);
+    fence_mbar_init();
+  }
   pdl_trigger();
   // the weight rows do not depend on the previous kernel: pull them into L2
   if (lane == 0 && blockIdx.y == 0)
     for (int e = gwarp; e < p.E; e += nwarps) prefetch_l2(p.wr + (size_t)e * p.H, (uint32_t)p.H * 2);
+  __syncthreads();
   pdl_wait();
-  for (int i = threadIdx.x; i < tb * nvec; i += blockDim.x)
-    reinterpret_cast<uint4*>(xs)[i] = reinterpret_cast<const uint4*>(p.x + (size_t)b0 * p.H)[i];
+  // the token tile's x rows (contiguous) in one bulk copy; bounded wait
+  if (threadIdx.x == 0) {
+    const uint32_t bytes = (uint32_t)tb * (uint32_t)p.H * 2u;
+    mbar_arrive_expect_tx(&s_bar, bytes);
+    bulk_g2s(xs, p.x + (size_t)b0 * p.H, bytes, &s_bar);
+  }
+  {
+    const long long budget = wait_budget(p.ctrl);
+    const long long t0 = clock64();
+    bool ok;
+    while (!(ok = mbar_try_wait(&s_bar, 0u)) && clock64() - t0 < budget) __nanosleep(32);
+    if (!ok && threadIdx.x == 0) set_error(p.ctrl, MOE_ERR_TIMEOUT);
+  }
   __syncthreads();
   for (int e = gwarp; e < p.E; e += nwarps) {
     const uint16_t* row = p.wr + (size_t)e * p.H;
@@ -177,7 +194,24 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterPara
   if (!s_last) return;
   __threadfence();
   float* lsm = reinterpret_cast<float*>(smem_raw);  // this tile's logits
-  for (int i = threadIdx.x; i < tb * p.E; i += blockDim.x) lsm[i] = __ldcg(p.logits + (size_t)b0 * p.E + i);
+  {
+    // every load of the tile in flight before the stores (the logits come from L2)
+    const float* src = p.logits + (size_t)b0 * p.E;
+    const int n = tb * p.E;
+    for (int i0 = 0; i0 < n; i0 += 8 * (int)blockDim.x) {
+      float v[8];
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + j * (int)blockDim.x + (int)threadIdx.x;
+        v[j] = i < n ? __ldcg(src + i) : 0.f;
+      }
+#pragma unroll
+      for (int j = 0; j < 8; ++j) {
+        const int i = i0 + j * (int)blockDim.x + (int)threadIdx.x;
+        if (i < n) lsm[i] = v[j];
+      }
+    }
+  }
   __syncthreads();
   for (int t = warp; t < tb; t += kRouterWarps) {
     const int b = b0 + t;
