@@ -98,7 +98,10 @@ struct StackParams {
 // Optional phase timeline (compiled in with -DMOEQ_STACK_TRACE only): one
 // thread per CTA stamps %globaltimer at phase ends into
 // trace[(layer * kTracePhases + phase) * G + cta]. Off in the library build.
-constexpr int kTracePhases = 17;  // 14, 15: first/last routed gate/up item landed; 16: longest such piece (ns)
+// 14, 15: first/last routed gate/up item landed; 16: longest such piece (ns);
+// 19, 20: x staging loads back / image written; 22, 23: the copy warp done
+// issuing layer l's routed items / the next layer's items
+constexpr int kTracePhases = 24;
 #ifdef MOEQ_STACK_TRACE
 #define STACK_MARK(cond, l, ph)                                                                    \
   do {                                                                                             \
@@ -115,7 +118,10 @@ constexpr int kTracePhases = 17;  // 14, 15: first/last routed gate/up item land
 #endif
 
 // CTA c's share [lo, hi) of n items split evenly over G CTAs.
-__host__ __device__ inline int share_lo(int c, int G, int n) { return (int)((long long)n * c / G); }
+// (n * c stays below 2^32: n is at most E, H/16 or K*I/8 of a plan that fits
+// the kernel's tables, c at most kStackMaxCtas; 32-bit division keeps the
+// plan's code short)
+__host__ __device__ inline int share_lo(int c, int G, int n) { return (int)((unsigned)n * (unsigned)c / (unsigned)G); }
 // Groups [lo, hi) of quarter q of a tile with ng groups.
 __host__ __device__ inline int quarter_lo(int q, int ng) { return q * ng / 4; }
 
@@ -143,6 +149,7 @@ __device__ void make_plan(const StackParams& p, ItemPlan& P) {
   int n = 0, pc = 0, tl = 0;
   P.r0 = share_lo(c, G, p.E);
   P.nr = share_lo(c + 1, G, p.E) - P.r0;
+#pragma unroll 1
   for (int r = 0; r < P.nr; r += 2) {
     P.kind[n] = kItemRouter;
     P.k[n] = 0;
@@ -157,6 +164,7 @@ __device__ void make_plan(const StackParams& p, ItemPlan& P) {
   P.n_router_pieces = pc;
   P.n_router_items = n;
   auto add_tile = [&](int k, int T) {
+#pragma unroll 1
     for (int h = 0; h < 2; ++h) {
       P.kind[n] = kItemGateUp;
       P.k[n] = k;
@@ -184,14 +192,17 @@ __device__ void make_plan(const StackParams& p, ItemPlan& P) {
     ++n;
   };
   const int tps = p.I / 8;  // gate/up tiles per slot
+#pragma unroll 1
   for (int T = share_lo(c, G, tps); T < share_lo(c + 1, G, tps); ++T) add_tile(p.K, T);
   P.n_sgu_items = n;
   if (P.nd > 0) add_down(p.K);
   P.n_pre_items = n;
   P.n_pre_pieces = pc;
+#pragma unroll 1
   for (int u = share_lo(c, G, p.K * tps); u < share_lo(c + 1, G, p.K * tps); ++u) add_tile(u / tps, u % tps);
   P.n_rgu_items = n;
   if (P.nd > 0)
+#pragma unroll 1
     for (int k = 0; k < p.K; ++k) add_down(k);
   P.n_items = n;
   P.n_pieces = pc;
@@ -316,6 +327,7 @@ __device__ void block_topk(const StackParams& p, int l, const float* lg, TopkScr
   if (!p.forced) {
     uint32_t ck = 0u;
     int ci = -1;
+#pragma unroll 1
     for (int kk = 0; kk < K; ++kk) {
       const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(k0, k1));
       const uint32_t cand = k0 == m ? (uint32_t)tid : (k1 == m ? (uint32_t)t1 : 0xFFFFFFFFu);
@@ -368,6 +380,7 @@ __device__ void block_topk(const StackParams& p, int l, const float* lg, TopkScr
       ck[j] = c < nc ? S.key[c] : 0u;
       ci[j] = c < nc ? S.idx[c] : 0xFFFFFFFFu;
     }
+#pragma unroll 1
     for (int kk = 0; kk < K; ++kk) {
       const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(max(ck[0], ck[1]), max(ck[2], ck[3])));
       uint32_t cand = 0xFFFFFFFFu;
@@ -487,7 +500,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
 
   if (tid == 0) {
     make_plan(p, P);
+#pragma unroll 1
     for (int it = 0; it < P.n_items; ++it)
+#pragma unroll 1
       for (int q = 0; q < P.npieces[it]; ++q) s_piece_item[P.piece0[it] + q] = (unsigned char)it;
     for (int i = 0; i < p.nslot; ++i) {
       mbar_init(&full_bar[i], 1);
@@ -534,8 +549,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       // gate/up and shared down items
       const uint32_t seq_l = (uint32_t)(l * n_items);
       bool ok = !s_abort && issue_items(p, P, R, l, P.n_pre_items, n_items, seq_l + P.n_pre_items, s_idx, &s_abort, budget);
+      STACK_MARK(lane == 0, l, 22);
       if (ok && l + 1 < p.n_layers)
         ok = issue_items(p, P, R, l + 1, 0, P.n_pre_items, (uint32_t)((l + 1) * n_items), s_idx, &s_abort, budget);
+      STACK_MARK(lane == 0, l, 23);
       if (!ok && lane == 0 && !s_abort) fail();
       __syncwarp();
     }
@@ -712,6 +729,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
           // value), read in the same round trip as r
           if (active) load_f32_16_cg(p.r + (size_t)tid * 16, v);
           const float inv_norm = rsqrtf(sum_partials(p.ss_part, G) / (float)H + p.eps);
+          STACK_MARK(tid == 0 && v[0] == v[0], l, 19);
           if (active) {
 #pragma unroll
             for (int j = 0; j < 16; ++j) v[j] = bf16_bits_to_f32(f32_to_bf16_bits(v[j] * inv_norm));
@@ -740,6 +758,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
           for (int j = 0; j < 16; ++j) v[j] = 0.f;
         }
         if (warp * 32 < nseg) qstage_seg(v, tid, p.G, X, active);
+        STACK_MARK(tid == 0, l, 20);
         gdot = warp_sum(gdot);
         if (lane == 0) s_red[1][warp] = gdot;
         named_sync(1, kCThreads);
