@@ -49,15 +49,15 @@ __device__ __forceinline__ float key_logit(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// Top-K of one token's logits (E <= 1024) by one warp, softmax weights at
+// Top-K of one token's logits (E <= 32 * NV) by one warp, softmax weights at
 // the picks (router gating of the Flash-MoE page, "Metal Compute Shaders").
 // Lane l keeps the keys of logits l + 32 j in registers; each of the K rounds
 // takes a warp-wide max over the keys and a warp-wide min over the indices
 // holding it (ties go to the lower index), and the owner lane clears its key.
-__device__ void topk_one_token(const float* lg, int E, int K, int renorm, const int32_t* forced, int32_t* idx_out,
-                               float* w_out, WsCtrl* ctrl) {
+template <int NV>
+__device__ void topk_one_token_nv(const float* lg, int E, int K, int renorm, const int32_t* forced, int32_t* idx_out,
+                                  float* w_out, WsCtrl* ctrl) {
   const int lane = threadIdx.x & 31;
-  constexpr int NV = kRouterMaxE / 32;
   uint32_t key[NV];
   uint32_t lk = 0u;
 #pragma unroll
@@ -116,6 +116,141 @@ __device__ void topk_one_token(const float* lg, int E, int K, int renorm, const 
       w_out[k] = (renorm && tot > 0.f) ? p[k] / tot : p[k];
     }
   }
+}
+
+// Softmax and top-K of one token's logits `lg` (shared memory) by NW warps
+// together (threads 0 .. 32*NW-1, each holding up to PT logits: E <= 32*NW*PT)
+// (router gating as the Flash-MoE page gives it in "Metal Compute Shaders":
+// softmax over all experts, the K largest, weights renormalised on request).
+// Thread t holds logits t + 32*NW*i as order-preserving keys; each warp takes
+// its K best by K rounds of a warp-wide max over the keys and a warp-wide min
+// over the indices holding it (ties go to the lower index), and warp 0 takes
+// the K best of the warps' candidates the same way: the top K of all logits
+// are among the warps' top K, so the picks are those of one global ranking.
+// The normaliser is summed per warp around the warp's own maximum and
+// rescaled to the global one. `sync` is the barrier of the NW warps. Warp 0's
+// lanes k < K end with sel[k] (the pick; -1 for none: no finite logit left or
+// an invalid forced index) and wsel[k] (its weight) written; the other warps
+// return after the barrier.
+template <int NW>
+struct SelScratch {
+  uint32_t key[NW * MOEQ_MAX_K];  // warp w's K best at w*K .. w*K+K-1, in rank order
+  uint32_t idx[NW * MOEQ_MAX_K];
+  float m[NW], z[NW];            // each warp's max logit and sum of exp(v - max)
+};
+
+template <int NW, int PT, typename Sync>
+__device__ void block_select(const float* lg, int E, int K, int renorm, const int32_t* forced, SelScratch<NW>& S,
+                             Sync sync, int* sel, float* wsel, WsCtrl* ctrl) {
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  constexpr int kT = NW * 32;
+  uint32_t key[PT];
+  uint32_t kmax = 0u;
+#pragma unroll
+  for (int i = 0; i < PT; ++i) {
+    const int e = tid + kT * i;
+    key[i] = e < E ? logit_key(lg[e]) : 0u;
+    kmax = max(kmax, key[i]);
+  }
+  const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, kmax);
+  const float mw = wm > kKeyNegInf ? key_logit(wm) : -INFINITY;
+  float zw = 0.f;
+  if (mw > -INFINITY) {  // warp-uniform
+#pragma unroll
+    for (int i = 0; i < PT; ++i) zw += key[i] > kKeyNegInf ? __expf(key_logit(key[i]) - mw) : 0.f;
+    zw = warp_sum(zw);
+  }
+  if (!forced) {
+    uint32_t ck = 0u;
+    int ci = -1;
+#pragma unroll 1
+    for (int kk = 0; kk < K; ++kk) {
+      uint32_t km = 0u;
+#pragma unroll
+      for (int i = 0; i < PT; ++i) km = max(km, key[i]);
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, km);
+      uint32_t cand = 0xFFFFFFFFu;
+#pragma unroll
+      for (int i = PT - 1; i >= 0; --i) cand = key[i] == m ? (uint32_t)(tid + kT * i) : cand;
+      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, cand);
+#pragma unroll
+      for (int i = 0; i < PT; ++i) key[i] = bi == (uint32_t)(tid + kT * i) ? 0u : key[i];
+      if (lane == kk) {
+        ck = m;
+        ci = (int)bi;
+      }
+    }
+    if (lane < K) {
+      S.key[warp * K + lane] = ck;
+      S.idx[warp * K + lane] = (uint32_t)ci;
+    }
+  }
+  if (lane == 0) {
+    S.m[warp] = mw;
+    S.z[warp] = zw;
+  }
+  sync();
+  if (warp != 0) return;
+
+  float mx = -INFINITY;
+#pragma unroll
+  for (int w = 0; w < NW; ++w) mx = fmaxf(mx, S.m[w]);
+  float z = (lane < NW && S.m[lane] > -INFINITY) ? S.z[lane] * __expf(S.m[lane] - mx) : 0.f;
+  z = warp_sum(z);
+  int pick_e = -1;     // lane k (< K) ends up holding pick k
+  float pick_l = 0.f;  // and its logit
+  if (forced) {
+    if (lane < K) {
+      const int bi = forced[lane];
+      const bool okf = bi >= 0 && bi < E;
+      pick_e = okf ? bi : -1;
+      pick_l = okf ? lg[bi] : -INFINITY;
+    }
+  } else {
+    // candidate c = lane + 32 j of the warps' NW * K
+    constexpr int NC = (NW * MOEQ_MAX_K + 31) / 32;
+    const int nc = NW * K;
+    uint32_t ck[NC];
+    uint32_t ci[NC];
+#pragma unroll
+    for (int j = 0; j < NC; ++j) {
+      const int c = lane + 32 * j;
+      ck[j] = c < nc ? S.key[c] : 0u;
+      ci[j] = c < nc ? S.idx[c] : 0xFFFFFFFFu;
+    }
+#pragma unroll 1
+    for (int kk = 0; kk < K; ++kk) {
+      uint32_t km = 0u;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) km = max(km, ck[j]);
+      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, km);
+      uint32_t cand = 0xFFFFFFFFu;
+#pragma unroll
+      for (int j = 0; j < NC; ++j) cand = ck[j] == m ? min(cand, ci[j]) : cand;
+      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, cand);
+#pragma unroll
+      for (int j = 0; j < NC; ++j) ck[j] = (ck[j] == m && ci[j] == bi) ? 0u : ck[j];
+      if (lane == kk) {
+        const bool fin = m > kKeyNegInf;  // no finite logit left: no expert
+        pick_e = fin ? (int)bi : -1;
+        pick_l = fin ? key_logit(m) : -INFINITY;
+      }
+    }
+  }
+  if (lane < K && pick_e < 0) set_error(ctrl, MOE_ERR_INDEX);
+  const float pw = (lane < K && pick_e >= 0) ? __expf(pick_l - mx) / z : 0.f;
+  const float tot = warp_sum(pw);
+  if (lane < K) {
+    sel[lane] = pick_e;
+    wsel[lane] = (renorm && tot > 0.f) ? pw / tot : pw;
+  }
+}
+
+// E <= 512 keeps 16 keys per lane, else 32.
+__device__ __forceinline__ void topk_one_token(const float* lg, int E, int K, int renorm, const int32_t* forced,
+                                               int32_t* idx_out, float* w_out, WsCtrl* ctrl) {
+  if (E <= 512) topk_one_token_nv<16>(lg, E, K, renorm, forced, idx_out, w_out, ctrl);
+  else topk_one_token_nv<kRouterMaxE / 32>(lg, E, K, renorm, forced, idx_out, w_out, ctrl);
 }
 
 // grid (E/kRouterWarps, ceil(B/kRouterTokTile)): CTA (c, j) dots rows of
@@ -213,10 +348,21 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterPara
     }
   }
   __syncthreads();
-  for (int t = warp; t < tb; t += kRouterWarps) {
-    const int b = b0 + t;
-    topk_one_token(lsm + (size_t)t * p.E, p.E, p.K, p.renorm, p.forced ? p.forced + (size_t)b * p.K : nullptr,
-                   p.idx + (size_t)b * p.K, p.w + (size_t)b * p.K, p.ctrl);
+  if (tb == 1) {
+    // one token: all warps select together (a warp alone would walk E/32
+    // keys per lane through K rounds)
+    __shared__ SelScratch<kRouterWarps> S;
+    const int32_t* forced = p.forced ? p.forced + (size_t)b0 * p.K : nullptr;
+    block_select<kRouterWarps, kRouterMaxE / (32 * kRouterWarps)>(lsm, p.E, p.K, p.renorm, forced, S,
+                                                                  [] { __syncthreads(); }, p.idx + (size_t)b0 * p.K,
+                                                                  p.w + (size_t)b0 * p.K, p.ctrl);
+    if (forced && warp == 0 && lane < p.K) p.idx[(size_t)b0 * p.K + lane] = forced[lane];
+  } else {
+    for (int t = warp; t < tb; t += kRouterWarps) {
+      const int b = b0 + t;
+      topk_one_token(lsm + (size_t)t * p.E, p.E, p.K, p.renorm, p.forced ? p.forced + (size_t)b * p.K : nullptr,
+                     p.idx + (size_t)b * p.K, p.w + (size_t)b * p.K, p.ctrl);
+    }
   }
   __syncthreads();
   if (threadIdx.x == 0) p.ctrl->router_ticket[blockIdx.y] = 0u;

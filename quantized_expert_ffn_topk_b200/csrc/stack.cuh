@@ -284,135 +284,6 @@ __device__ bool issue_items(const StackParams& p, const ItemPlan& P, Ring& R, in
 
 // ---- softmax and top-K -------------------------------------------------------
 
-struct TopkScratch {
-  uint32_t key[kCWarps * MOEQ_MAX_K];  // warp w's K best at w*K .. w*K+K-1, in rank order
-  uint32_t idx[kCWarps * MOEQ_MAX_K];
-  float m[kCWarps], z[kCWarps];       // each warp's max logit and sum of exp(v - max)
-};
-
-// Softmax and top-K of layer l's logits `lg` (in shared memory, relayed there
-// by the copy warp) (router gating as the Flash-MoE page
-// gives it in "Metal Compute Shaders": softmax over all experts, the K
-// largest, weights renormalised on request), run by all compute warps of the
-// CTA. Thread t holds logits t and t + kCThreads; a warp takes its K best by
-// K rounds of a warp-wide max over the keys and a warp-wide min over the
-// indices holding it (ties go to the lower expert index), and warp 0 takes
-// the K best of the warps' candidates the same way. The top K of all logits
-// are among the warps' top K, so the picks are those of one global ranking.
-// The normaliser is summed per warp around the warp's own maximum and
-// rescaled to the global one. Warp 0 writes the picks and weights to
-// s_idx/s_w and then raises *ready to l + 1 for the producer warp.
-__device__ void block_topk(const StackParams& p, int l, const float* lg, TopkScratch& S, int* s_idx, float* s_w,
-                           volatile int* ready) {
-  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
-  const int E = p.E, K = p.K;
-  const int t1 = tid + kCThreads;
-  float v0 = -INFINITY, v1 = -INFINITY;
-  if (tid < E) {
-    const float x = lg[tid];
-    v0 = x == x ? x : -INFINITY;
-  }
-  if (t1 < E) {
-    const float x = lg[t1];
-    v1 = x == x ? x : -INFINITY;
-  }
-  uint32_t k0 = tid < E ? logit_key(v0) : 0u, k1 = t1 < E ? logit_key(v1) : 0u;
-  const uint32_t wm = __reduce_max_sync(0xFFFFFFFFu, max(k0, k1));
-  const float mw = wm > kKeyNegInf ? key_logit(wm) : -INFINITY;
-  float zw = 0.f;
-  if (mw > -INFINITY) {  // warp-uniform
-    zw = (tid < E ? __expf(v0 - mw) : 0.f) + (t1 < E ? __expf(v1 - mw) : 0.f);
-    zw = warp_sum(zw);
-  }
-  if (!p.forced) {
-    uint32_t ck = 0u;
-    int ci = -1;
-#pragma unroll 1
-    for (int kk = 0; kk < K; ++kk) {
-      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(k0, k1));
-      const uint32_t cand = k0 == m ? (uint32_t)tid : (k1 == m ? (uint32_t)t1 : 0xFFFFFFFFu);
-      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, cand);
-      if (bi == (uint32_t)tid) {
-        k0 = 0u;
-      } else if (bi == (uint32_t)t1) {
-        k1 = 0u;
-      }
-      if (lane == kk) {
-        ck = m;
-        ci = (int)bi;
-      }
-    }
-    if (lane < K) {
-      S.key[warp * K + lane] = ck;
-      S.idx[warp * K + lane] = (uint32_t)ci;
-    }
-  }
-  if (lane == 0) {
-    S.m[warp] = mw;
-    S.z[warp] = zw;
-  }
-  named_sync(1, kCThreads);
-  if (warp != 0) return;
-
-  float mx = -INFINITY;
-#pragma unroll
-  for (int w = 0; w < kCWarps; ++w) mx = fmaxf(mx, S.m[w]);
-  float z = (lane < kCWarps && S.m[lane] > -INFINITY) ? S.z[lane] * __expf(S.m[lane] - mx) : 0.f;
-  z = warp_sum(z);
-  int pick_e = -1;     // lane k (< K) ends up holding pick k
-  float pick_l = 0.f;  // and its logit
-  const int32_t* forced = p.forced ? p.forced + (size_t)l * K : nullptr;
-  if (forced) {
-    if (lane < K) {
-      const int bi = forced[lane];
-      const bool okf = bi >= 0 && bi < E;
-      pick_e = okf ? bi : -1;
-      pick_l = okf ? lg[bi] : -INFINITY;
-    }
-  } else {
-    // candidate c = lane + 32 j of the warps' kCWarps * K
-    const int nc = kCWarps * K;
-    uint32_t ck[4];
-    uint32_t ci[4];
-#pragma unroll
-    for (int j = 0; j < 4; ++j) {
-      const int c = lane + 32 * j;
-      ck[j] = c < nc ? S.key[c] : 0u;
-      ci[j] = c < nc ? S.idx[c] : 0xFFFFFFFFu;
-    }
-#pragma unroll 1
-    for (int kk = 0; kk < K; ++kk) {
-      const uint32_t m = __reduce_max_sync(0xFFFFFFFFu, max(max(ck[0], ck[1]), max(ck[2], ck[3])));
-      uint32_t cand = 0xFFFFFFFFu;
-#pragma unroll
-      for (int j = 0; j < 4; ++j) cand = ck[j] == m ? min(cand, ci[j]) : cand;
-      const uint32_t bi = __reduce_min_sync(0xFFFFFFFFu, cand);
-#pragma unroll
-      for (int j = 0; j < 4; ++j) ck[j] = (ck[j] == m && ci[j] == bi) ? 0u : ck[j];
-      if (lane == kk) {
-        const bool fin = m > kKeyNegInf;  // no finite logit left: no expert
-        pick_e = fin ? (int)bi : -1;
-        pick_l = fin ? key_logit(m) : -INFINITY;
-      }
-    }
-  }
-  if (lane < K && pick_e < 0) set_error(p.ctrl, MOE_ERR_INDEX);
-  const float pw = (lane < K && pick_e >= 0) ? __expf(pick_l - mx) / z : 0.f;
-  const float tot = warp_sum(pw);
-  if (lane < K) {
-    const float wk = (p.renorm && tot > 0.f) ? pw / tot : pw;
-    s_idx[lane] = pick_e;
-    s_w[lane] = wk;
-    if (blockIdx.x == 0) {
-      if (p.idx_out) p.idx_out[(size_t)l * K + lane] = forced ? forced[lane] : pick_e;
-      if (p.w_out) p.w_out[(size_t)l * K + lane] = wk;
-    }
-  }
-  __syncwarp();
-  __threadfence_block();
-  if (lane == 0) *ready = l + 1;
-}
-
 // Bounded wait until the shared-memory flag reaches target.
 __device__ __forceinline__ bool flag_wait(const volatile int* f, int target, const volatile int* abort,
                                           long long budget) {
@@ -477,7 +348,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
   __shared__ float s_red[2][kCWarps];
   __shared__ unsigned char s_piece_item[kMaxPieces];
   __shared__ ItemPlan P;
-  __shared__ TopkScratch s_topk;
+  __shared__ SelScratch<kCWarps> s_topk;
   __shared__ volatile int s_abort;
   __shared__ volatile int s_topk_ready;
   __shared__ volatile int s_logits_ready;  // layer + 1 once s_logits holds that layer's logits
@@ -794,7 +665,21 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       if (lane == 0 && !flag_wait(&s_logits_ready, l + 1, &s_abort, budget) && !s_abort) fail();
       __syncwarp();
       STACK_MARK(tid == 0, l, 5);
-      block_topk(p, l, s_logits, s_topk, s_idx, s_w, &s_topk_ready);
+      {  // (all compute warps; warp 0 ends with the picks and weights)
+        const int32_t* forced = p.forced ? p.forced + (size_t)l * K : nullptr;
+        block_select<kCWarps, kStackMaxE / kCThreads>(s_logits, p.E, K, p.renorm, forced, s_topk,
+                                                       [] { named_sync(1, kCThreads); }, s_idx, s_w, p.ctrl);
+        if (warp == 0) {
+          __syncwarp();
+          if (blockIdx.x == 0 && lane < K) {
+            if (p.idx_out) p.idx_out[(size_t)l * K + lane] = forced ? forced[lane] : s_idx[lane];
+            if (p.w_out) p.w_out[(size_t)l * K + lane] = s_w[lane];
+          }
+          __syncwarp();
+          __threadfence_block();
+          if (lane == 0) s_topk_ready = l + 1;
+        }
+      }
       STACK_MARK(tid == 0, l, 6);
 
       // ---- the shared expert's down tiles, once every CTA's shared h is out ----
