@@ -25,13 +25,16 @@
 namespace moeq {
 
 constexpr int kGrpWarps = 8;
+// (measured at 32 and 128 tokens per step on the 4-bit layer: 3 CTAs per SM
+// with 4 blocks in flight per warp beat 4 x 2, 4 x 3, 3 x 3, 3 x 5, 2 x 6 and
+// 2 x 8)
 #ifndef MOEQ_GRP_CTAS
-#define MOEQ_GRP_CTAS 4
+#define MOEQ_GRP_CTAS 3
 #endif
 #ifndef MOEQ_GRP_INFLIGHT
-#define MOEQ_GRP_INFLIGHT 2
+#define MOEQ_GRP_INFLIGHT 4
 #endif
-constexpr int kGrpCtasPerSm = MOEQ_GRP_CTAS;        // resident CTAs per SM (64 registers a thread at 4)
+constexpr int kGrpCtasPerSm = MOEQ_GRP_CTAS;        // resident CTAs per SM (85 registers a thread at 3)
 constexpr int kGrpInFlight = MOEQ_GRP_INFLIGHT;     // blocks whose loads a warp keeps in flight
 constexpr int kGrpUnits = kGrpWarps / kFfnPieces;  // units per round (four warps each)
 constexpr int kGrpMaxTok = 64;                      // tokens of one work item at most
@@ -191,19 +194,19 @@ __device__ __forceinline__ void ld_stream_words(const unsigned char* p, uint32_t
 }
 
 // Blocks [0, nblk) of one tile in global memory against groups [g0, g0+nblk)
-// of up to four tokens' images (imgs[c], c < nt; the lanes of column pair c
-// read image c). Lane (gid, t) accumulates token t: acc0 for local row gid,
-// acc1 for row gid+8.
+// of up to four tokens' images: col is the image whose B fragments this lane
+// loads (token gid/2: the mma's column gid carries its hi or lo plane), tok
+// the image of the lane's own token t (its group scales and sums). Lane
+// (gid, t) accumulates token t: acc0 for local row gid, acc1 for row gid+8.
 template <int BITS, int KS>
-__device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int nblk, int g0,
-                                                const unsigned char* const (&imgs)[4], int gs_off, float& acc0,
-                                                float& acc1) {
+__device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int nblk, int g0, const unsigned char* col,
+                                                const unsigned char* tok, int gs_off, float& acc0, float& acc1) {
   using F = TileFmt<BITS, KS>;
   constexpr int P = kGrpInFlight;
   const int lane = threadIdx.x & 31, gid = lane >> 2, t = lane & 3;
-  // B fragments of column gid: token gid/2, plane hi (gid even) or lo
-  const uint2* planes = reinterpret_cast<const uint2*>(imgs[gid >> 1]) + (gid & 1) * 4 + t;
-  const float2* gs = reinterpret_cast<const float2*>(imgs[t] + gs_off);  // this lane's token
+  // B fragments of column gid: token gid/2 (image col), plane hi (gid even) or lo
+  const uint2* planes = reinterpret_cast<const uint2*>(col) + (gid & 1) * 4 + t;
+  const float2* gs = reinterpret_cast<const float2*>(tok + gs_off);  // this lane's token
   for (int b0 = 0; b0 < nblk; b0 += P) {
     uint32_t w[P][F::NW];
     uint2 sb[P], bf[P][KS];
@@ -258,7 +261,10 @@ __device__ __forceinline__ void unit_token(const GrpParams& p, int a, int i, int
 
 // DOWN == false: gate/up tiles against x images, h per (token, slot).
 // DOWN == true: down tiles against h images, y per (token, slot).
-template <bool DOWN>
+// FB, FKS: the one format (bits, k-steps per group) of every expert the
+// instance serves when the routed and shared widths agree, so that only that
+// tile dot is compiled in; FB == 0: any format, chosen per work item.
+template <bool DOWN, int FB, int FKS>
 __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpParams p) {
   __shared__ float part[kGrpUnits][kFfnPieces][kGrpMaxTok][kTileRows];
   __shared__ int s_tok[kGrpUnits][kGrpMaxTok][2];
@@ -293,17 +299,19 @@ __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpPa
       const unsigned char* blk =
           rec + (DOWN ? g.down_off + (size_t)T * g.D : (size_t)T * g.U) + (size_t)g0 * g.blk;
       for (int c0 = 0; c0 < ntok[r]; c0 += 4) {
-        const unsigned char* imgs[4];
-#pragma unroll
-        for (int c = 0; c < 4; ++c) {
-          const int i = min(c0 + c, ntok[r] - 1);
+        auto image = [&](int i) {
+          i = min(c0 + i, ntok[r] - 1);
           const int src = DOWN ? s_tok[r][i][0] * (f.K + 1) + s_tok[r][i][1] : s_tok[r][i][0];
-          imgs[c] = p.img + (size_t)src * p.img_stride;
-        }
+          return p.img + (size_t)src * p.img_stride;
+        };
+        const unsigned char* col = image(lane >> 3);  // token gid/2
+        const unsigned char* tok = image(lane & 3);   // token t
         float acc0 = 0.f, acc1 = 0.f;
-        with_fmt(routed ? f.bits_r : f.bits_s, f.G, [&]<int BITS, int KS>() {
-          tile_dot_tokens<BITS, KS>(blk, g1 - g0, g0, imgs, p.img_gs_off, acc0, acc1);
-        });
+        auto dot = [&]<int BITS, int KS>() {
+          tile_dot_tokens<BITS, KS>(blk, g1 - g0, g0, col, tok, p.img_gs_off, acc0, acc1);
+        };
+        if constexpr (FB == 0) with_fmt(routed ? f.bits_r : f.bits_s, f.G, dot);
+        else dot.template operator()<FB, FKS>();
         const int i = c0 + (lane & 3);
         if (i < ntok[r]) {
           part[r][q][i][lane >> 2] = acc0;

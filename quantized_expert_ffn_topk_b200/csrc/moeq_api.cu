@@ -155,6 +155,28 @@ moe_status check_layer(const moe_layer_q* L) {
 
 bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes);  // below
 
+// The grouped kernels' instances: one format compiled in when the routed and
+// shared widths agree, else the instances that pick the format per item.
+struct GrpKernels {
+  void (*gate_up)(GrpParams);
+  void (*down)(GrpParams);
+};
+GrpKernels grp_kernels(int br, int bs, int G) {
+#define MOEQ_GRP_CASE(B, Gp, KS) \
+  if (br == B && bs == B && G == Gp) return GrpKernels{k_ffn_grp<false, B, KS>, k_ffn_grp<true, B, KS>};
+  MOEQ_GRP_CASE(4, 32, 1)
+  MOEQ_GRP_CASE(4, 64, 2)
+  MOEQ_GRP_CASE(4, 128, 4)
+  MOEQ_GRP_CASE(2, 32, 1)
+  MOEQ_GRP_CASE(2, 64, 2)
+  MOEQ_GRP_CASE(2, 128, 4)
+  MOEQ_GRP_CASE(3, 64, 2)
+  MOEQ_GRP_CASE(3, 128, 4)
+#undef MOEQ_GRP_CASE
+  return GrpKernels{k_ffn_grp<false, 0, 0>, k_ffn_grp<true, 0, 0>};
+}
+
+
 // The one-token FFN kernels' dot: the tensor-core dot, or with
 // MOEQ_BATCH1_DOT=fma in the environment the fp32 CUDA-core dot (a switch
 // for comparing the two on the same kernels; read once).
@@ -447,7 +469,8 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     gp.img_gs_off = wl.ximg_gs;
     gp.tps = p.I / 8;
     gp.max_units = (gp.nsh + max_act) * gp.tps;
-    st = launch_pdl(k_ffn_grp<false>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
+    const GrpKernels gk = grp_kernels(p.bits_r, p.bits_s, p.G);
+    st = launch_pdl(gk.gate_up, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
     if (st != MOE_OK) return st;
     st = launch_pdl(k_stage_batch, dim3(B, p.K + 1), dim3(256), 0, s, (const void*)p.h, 1, p.I, p.G, himg,
                     wl.himg_stride, wl.himg_gs);
@@ -457,7 +480,7 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
     gp.img_gs_off = wl.himg_gs;
     gp.tps = p.H / kTileRows;
     gp.max_units = (gp.nsh + max_act) * gp.tps;
-    return launch_pdl(k_ffn_grp<true>, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
+    return launch_pdl(gk.down, dim3(ctas), dim3(kGrpWarps * 32), 0, s, gp);
   }
 
   // one token: every CTA bulk-copies its share of whole tiles into shared memory
