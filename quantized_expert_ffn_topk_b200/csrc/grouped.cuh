@@ -50,7 +50,7 @@ struct GrpWs {
   int* off;   // [E + 1]
   int* list;  // [B*K]: entries b*K + k grouped by expert, in entry order
   int* act;   // [E + kGrpExtraChunks][3]: (expert, its first entry in list, entries) per chunk, by expert id
-  int* nact;  // [1]: chunks
+  int* nact;  // [3]: chunks, then the next unit of the gate/up and of the down kernel (0 after grouping)
 };
 
 struct GrpParams {
@@ -135,6 +135,8 @@ __global__ void __launch_bounds__(256) k_group(const int32_t* idx, int B, int K,
     }
     g.off[E] = tc;
     g.nact[0] = tk;
+    g.nact[1] = 0;
+    g.nact[2] = 0;
   }
   __syncthreads();
   // each entry's rank among the earlier entries of its expert (a stable
@@ -273,8 +275,18 @@ __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpPa
   pdl_wait();
   const int nunits = min(p.max_units, (p.nsh + p.g.nact[0]) * p.tps);
   const int u_end = nunits;
-  // rounds of kGrpUnits consecutive units, dealt to the CTAs in turn
-  for (int u0 = blockIdx.x * kGrpUnits; u0 < nunits; u0 += gridDim.x * kGrpUnits) {
+  // rounds of kGrpUnits consecutive units, each CTA taking the next round
+  // from the workspace counter when it is free: work items carry different
+  // numbers of tokens (the shared expert's all of them), so a static deal
+  // would leave the CTAs that drew the heavy units last; those come first in
+  // the order and start first
+  __shared__ int s_u0;
+  int* next = p.g.nact + (DOWN ? 2 : 1);
+  while (true) {
+    if (threadIdx.x == 0) s_u0 = atomicAdd(next, kGrpUnits);
+    __syncthreads();
+    const int u0 = s_u0;
+    if (u0 >= nunits) break;
     // the units of this round and their token lists
     int ntok[kGrpUnits];
 #pragma unroll

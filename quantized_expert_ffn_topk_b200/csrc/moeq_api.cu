@@ -126,7 +126,7 @@ inline WsLayout ws_layout(int B, int K, int H, int I, int E) {
   l.act = o;
   o += align_up((size_t)(E + kGrpExtraChunks) * 3 * 4);
   l.nact = o;
-  o += align_up(4);
+  o += align_up(3 * 4);  // chunks, then the two grouped kernels' unit counters
   // images: planes then (scale, sum) per group; the smallest group (32) sizes them
   l.ximg_gs = (int)align_up(qimg_plane_bytes(H), 16);
   l.ximg_stride = (int)align_up(l.ximg_gs + qimg_gs_bytes(H, 32), 256);
