@@ -38,7 +38,14 @@ constexpr int kGrpCtasPerSm = MOEQ_GRP_CTAS;        // resident CTAs per SM (85 
 constexpr int kGrpInFlight = MOEQ_GRP_INFLIGHT;     // blocks whose loads a warp keeps in flight
 constexpr int kGrpUnits = kGrpWarps / kFfnPieces;  // units per round (four warps each)
 constexpr int kGrpMaxTok = 64;                      // tokens of one work item at most
-constexpr int kGrpSharedItems = (MOEQ_MAX_B + kGrpMaxTok - 1) / kGrpMaxTok;  // the shared expert's work items at most
+// (work items of 16 or 8 of the shared expert's tokens measured no faster
+// than 64 at 32 and 128 tokens per step once units are dealt on demand)
+#ifndef MOEQ_GRP_SHARED_TOK
+#define MOEQ_GRP_SHARED_TOK 64
+#endif
+constexpr int kGrpSharedTok = MOEQ_GRP_SHARED_TOK;  // tokens of one of the shared expert's work items
+static_assert(kGrpSharedTok <= kGrpMaxTok, "work items hold kGrpMaxTok tokens at most");
+constexpr int kGrpSharedItems = (MOEQ_MAX_B + kGrpSharedTok - 1) / kGrpSharedTok;  // the shared expert's work items at most
 
 // A routed expert with more than kGrpMaxTok entries (popular experts of a
 // large batch, or forced picks that repeat an expert within a token) is split
@@ -250,7 +257,7 @@ __device__ __forceinline__ void tile_dot_tokens(const unsigned char* blk0, int n
 // routed expert, whose entries b*K + k sit in list from act[1] on.
 __device__ __forceinline__ void unit_token(const GrpParams& p, int a, int i, int& b, int& k) {
   if (a < p.nsh) {
-    b = a * kGrpMaxTok + i;
+    b = a * kGrpSharedTok + i;
     k = p.f.K;
   } else {
     const int ent = p.g.list[p.g.act[3 * (a - p.nsh) + 1] + i];
@@ -295,7 +302,7 @@ __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpPa
       ntok[r] = 0;
       if (u < u_end) {
         const int a = u / p.tps;
-        ntok[r] = a < p.nsh ? min(kGrpMaxTok, f.B - a * kGrpMaxTok) : p.g.act[3 * (a - p.nsh) + 2];
+        ntok[r] = a < p.nsh ? min(kGrpSharedTok, f.B - a * kGrpSharedTok) : p.g.act[3 * (a - p.nsh) + 2];
         for (int i = threadIdx.x; i < ntok[r]; i += blockDim.x) unit_token(p, a, i, s_tok[r][i][0], s_tok[r][i][1]);
       }
     }

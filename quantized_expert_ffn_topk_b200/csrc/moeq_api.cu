@@ -454,7 +454,7 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
                  reinterpret_cast<int*>((char*)ws + wl.nact)};
     const int max_act = std::min(p.E, B * p.K) + kGrpExtraChunks;  // routed work items at most
     const int ctas = kGrpCtasPerSm * num_sms();
-    gp.nsh = (B + kGrpMaxTok - 1) / kGrpMaxTok;
+    gp.nsh = (B + kGrpSharedTok - 1) / kGrpSharedTok;
     st = launch_pdl(k_group, dim3(1), dim3(256), (size_t)std::max(p.E + 1, B * p.K) * 4, s, idx, B, p.K, p.E, p.H, gp.g,
                     y_out,
                     p.ctrl);
