@@ -36,7 +36,18 @@ constexpr int kGrpWarps = 8;
 #endif
 constexpr int kGrpCtasPerSm = MOEQ_GRP_CTAS;        // resident CTAs per SM (85 registers a thread at 3)
 constexpr int kGrpInFlight = MOEQ_GRP_INFLIGHT;     // blocks whose loads a warp keeps in flight
-constexpr int kGrpUnits = kGrpWarps / kFfnPieces;  // units per round (four warps each)
+// Pieces of a tile (warps that share a unit, a part of its groups each): a
+// down tile has a quarter of a gate/up tile's groups, so its units are
+// dealt whole to one warp and a round carries more of them.
+#ifndef MOEQ_GRP_PIECES_GU
+#define MOEQ_GRP_PIECES_GU 4
+#endif
+#ifndef MOEQ_GRP_PIECES_DN
+#define MOEQ_GRP_PIECES_DN 1
+#endif
+constexpr int kGrpPiecesGu = MOEQ_GRP_PIECES_GU;
+constexpr int kGrpPiecesDn = MOEQ_GRP_PIECES_DN;
+static_assert(kGrpWarps % kGrpPiecesGu == 0 && kGrpWarps % kGrpPiecesDn == 0, "whole units per round");
 constexpr int kGrpMaxTok = 64;                      // tokens of one work item at most
 // (work items of 16 or 8 of the shared expert's tokens measured no faster
 // than 64 at 32 and 128 tokens per step once units are dealt on demand)
@@ -275,14 +286,16 @@ __device__ __forceinline__ void unit_token(const GrpParams& p, int a, int i, int
 // tile dot is compiled in; FB == 0: any format, chosen per work item.
 template <bool DOWN, int FB, int FKS>
 __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpParams p) {
-  __shared__ float part[kGrpUnits][kFfnPieces][kGrpMaxTok][kTileRows];
-  __shared__ int s_tok[kGrpUnits][kGrpMaxTok][2];
+  constexpr int NP = DOWN ? kGrpPiecesDn : kGrpPiecesGu;  // warps per unit
+  constexpr int NU = kGrpWarps / NP;                       // units per round
+  __shared__ float part[NU][NP][kGrpMaxTok][kTileRows];
+  __shared__ int s_tok[NU][kGrpMaxTok][2];
   const FfnParams& f = p.f;
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   pdl_wait();
   const int nunits = min(p.max_units, (p.nsh + p.g.nact[0]) * p.tps);
   const int u_end = nunits;
-  // rounds of kGrpUnits consecutive units, each CTA taking the next round
+  // rounds of NU consecutive units, each CTA taking the next round
   // from the workspace counter when it is free: work items carry different
   // numbers of tokens (the shared expert's all of them), so a static deal
   // would leave the CTAs that drew the heavy units last; those come first in
@@ -290,14 +303,14 @@ __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpPa
   __shared__ int s_u0;
   int* next = p.g.nact + (DOWN ? 2 : 1);
   while (true) {
-    if (threadIdx.x == 0) s_u0 = atomicAdd(next, kGrpUnits);
+    if (threadIdx.x == 0) s_u0 = atomicAdd(next, NU);
     __syncthreads();
     const int u0 = s_u0;
     if (u0 >= nunits) break;
     // the units of this round and their token lists
-    int ntok[kGrpUnits];
+    int ntok[NU];
 #pragma unroll
-    for (int r = 0; r < kGrpUnits; ++r) {
+    for (int r = 0; r < NU; ++r) {
       const int u = u0 + r;
       ntok[r] = 0;
       if (u < u_end) {
@@ -307,14 +320,14 @@ __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpPa
       }
     }
     __syncthreads();
-    const int r = warp / kFfnPieces, q = warp % kFfnPieces, u = u0 + r;
+    const int r = warp / NP, q = warp % NP, u = u0 + r;
     if (u < u_end) {
       const int a = u / p.tps, T = u % p.tps;
       const bool routed = a >= p.nsh;
       const RecGeom& g = routed ? f.geo_r : f.geo_s;
       const uint8_t* rec = routed ? f.experts + (size_t)p.g.act[3 * (a - p.nsh)] * f.rec_r : f.shared;
       const int ng = DOWN ? (int)g.ng_i : (int)g.ng_h;
-      const int g0 = piece_lo(q, ng), g1 = piece_lo(q + 1, ng);
+      const int g0 = q * ng / NP, g1 = (q + 1) * ng / NP;
       const unsigned char* blk =
           rec + (DOWN ? g.down_off + (size_t)T * g.D : (size_t)T * g.U) + (size_t)g0 * g.blk;
       for (int c0 = 0; c0 < ntok[r]; c0 += 4) {
@@ -341,7 +354,7 @@ __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpPa
     __syncthreads();
     // finish: gate/up -> h = silu(gate) * up for 8 units; down -> y rows
 #pragma unroll
-    for (int rr = 0; rr < kGrpUnits; ++rr) {
+    for (int rr = 0; rr < NU; ++rr) {
       const int uu = u0 + rr;
       if (uu >= u_end) continue;
       const int T = uu % p.tps;
@@ -351,7 +364,7 @@ __global__ void __launch_bounds__(kGrpWarps * 32, kGrpCtasPerSm) k_ffn_grp(GrpPa
         const int b = s_tok[rr][i][0], k = s_tok[rr][i][1];
         float s0 = 0.f, s1 = 0.f;
 #pragma unroll
-        for (int qq = 0; qq < kFfnPieces; ++qq) {
+        for (int qq = 0; qq < NP; ++qq) {
           s0 += part[rr][qq][i][row];
           if (!DOWN) s1 += part[rr][qq][i][row + 8];
         }
