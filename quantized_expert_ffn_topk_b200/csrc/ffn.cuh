@@ -56,7 +56,8 @@ __device__ __forceinline__ const uint8_t* ffn_slot_rec(const FfnParams& p, int k
 // Issue the bulk copies of tiles [u0, u0 + nt) of the CTA's share (lane j
 // copies tile u0 + j into buffer j; 0 bytes for an invalid expert). `src`
 // gives a tile's record, offset and size; `take(u)` selects which tiles this
-// call issues (the shared expert's before pdl_wait, the routed ones after).
+// call issues (the gate/up kernel: the shared expert's before pdl_wait, the
+// routed ones after).
 template <typename Src, typename Take>
 __device__ __forceinline__ void ffn_issue(unsigned char* tiles, int stride, uint64_t* bar, int u0, int nt, Src src,
                                           Take take) {
@@ -111,7 +112,6 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
     fence_mbar_init();
   }
   __syncthreads();
-  pdl_trigger();
   auto src = [&](int u, const unsigned char** from) -> uint32_t {
     const int k = u / tps, T = u % tps;
     const uint8_t* rec = ffn_slot_rec(p, k);
@@ -126,6 +126,9 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
   // the shared expert's tiles do not depend on the previous kernel
   if (warp == 0 && t_lo < t_hi) ffn_issue(tiles, p.gu_stride, bar, t_lo, min(p.gu_nbuf, t_hi - t_lo), src, is_shared);
   pdl_wait();
+  // the down kernel may start from here on: the router has completed, so it
+  // can read the picks and issue all its tile copies at once
+  pdl_trigger();
   const long long budget = wait_budget(p.ctrl);
   int round = 0, nt = 0;
   for (int r0 = t_lo; r0 < t_hi; r0 += p.gu_nbuf, ++round) {
@@ -218,20 +221,17 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
     *from = rec + g.down_off + (size_t)T * g.D;
     return g.D;
   };
-  auto is_shared = [&](int u) { return u / tpd == p.K; };
-  auto is_routed = [&](int u) { return u / tpd != p.K; };
   auto any = [&](int) { return true; };
-  // the shared expert's tiles do not depend on the previous kernels
-  if (warp == 0 && t_lo < t_hi) ffn_issue(tiles, p.dn_stride, bar, t_lo, min(p.dn_nbuf, t_hi - t_lo), src, is_shared);
+  // the tiles depend only on the weights and the picks: the gate/up kernel
+  // lets this kernel start only after the router has completed, so the
+  // first round's copies go out before the wait for the gate/up kernel's h
+  if (warp == 0 && t_lo < t_hi) ffn_issue(tiles, p.dn_stride, bar, t_lo, min(p.dn_nbuf, t_hi - t_lo), src, any);
   pdl_wait();
   const long long budget = wait_budget(p.ctrl);
   int round = 0, nt = 0;
   for (int r0 = t_lo; r0 < t_hi; r0 += p.dn_nbuf, ++round) {
     nt = min(p.dn_nbuf, t_hi - r0);
-    if (warp == 0) {
-      if (r0 == t_lo) ffn_issue(tiles, p.dn_stride, bar, r0, nt, src, is_routed);
-      else ffn_issue(tiles, p.dn_stride, bar, r0, nt, src, any);
-    }
+    if (warp == 0 && r0 != t_lo) ffn_issue(tiles, p.dn_stride, bar, r0, nt, src, any);
     if (r0 == t_lo) {  // images of the slots this CTA's jobs touch
       for (int k = t_lo / tpd; k <= (t_hi - 1) / tpd; ++k) {
         const float* hk = p.h + (size_t)k * p.I;
