@@ -227,16 +227,25 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, const 
   }
 }
 
-// Bounded wait until *counter >= target (gpu-scope acquire).
+__device__ __forceinline__ unsigned ld_relaxed_gpu(const unsigned* p) {
+  unsigned v;
+  asm volatile("ld.relaxed.gpu.global.u32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
+// Bounded wait until *counter >= target (gpu-scope acquire). The poll reads
+// relaxed; once the target is seen, one acquire read of the counter (the
+// counts only grow) orders the caller's later reads after the arrivals.
 __device__ __forceinline__ bool counter_wait(const unsigned* counter, unsigned target, const volatile int* abort,
                                              long long budget) {
   if (ld_acquire_gpu(counter) >= target) return true;
   const long long t0 = clock64();
-  while (ld_acquire_gpu(counter) < target) {
+  while (ld_relaxed_gpu(counter) < target) {
     if (*abort) return false;
     if (clock64() - t0 > budget) return false;
     __nanosleep(32);
   }
+  (void)ld_acquire_gpu(counter);
   return true;
 }
 
