@@ -169,7 +169,8 @@ def run_reference(args, w, rank: int):
             "n_gpus": args.gpus, "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 / tps,
             "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": workload_config(w, args.layers, args.gpus),
-            "cpu_baseline": {"value": tps, "unit": "layer-tokens/s", "cores": 1, "kind": "oracle",
+            "cpu_baseline": {"value": tps, "unit": "layer-tokens/s", "cores": 1, "host_cores": os.cpu_count(),
+                             "kind": "oracle",
                              "sample": "%d layer-token steps (router, top-K, 5 expert FFNs, combine, RMSNorm) of %s "
                                        "through the single-threaded fp64 C oracle, %.1f s of oracle work"
                                        % (n, w.name, secs)},
@@ -646,7 +647,8 @@ def main():
     line = run_ours(args, w, rank, world, local_rank)
     if rank == 0 and line is not None:
         tps, secs = oracle_tokens_per_s(w, args.cpu_sample)
-        line["cpu_baseline"] = {"value": tps, "unit": "layer-tokens/s", "cores": 1, "kind": "oracle",
+        line["cpu_baseline"] = {"value": tps, "unit": "layer-tokens/s", "cores": 1, "host_cores": os.cpu_count(),
+                                "kind": "oracle",
                                 "sample": "%d layer-token steps of %s through the single-threaded fp64 C oracle "
                                           "(%.1f s of oracle work)" % (args.cpu_sample, w.name, secs)}
         print(json.dumps(line), flush=True)
