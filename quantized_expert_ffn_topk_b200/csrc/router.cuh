@@ -318,16 +318,19 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterPara
       }
     }
   }
-  // The last CTA of this token tile to arrive selects for its tokens.
+  // The last CTA of this token tile to arrive selects for its tokens. The
+  // ticket is one acquire-release add: it publishes this CTA's logits (stored
+  // before the barrier) and, for the last CTA, orders its reads of every
+  // other CTA's logits after their adds.
   __syncthreads();
   if (threadIdx.x == 0) {
-    __threadfence();
-    unsigned t = atomicAdd(&p.ctrl->router_ticket[blockIdx.y], 1u);
+    unsigned t;
+    asm volatile("atom.acq_rel.gpu.global.add.u32 %0, [%1], 1;" : "=r"(t) : "l"(&p.ctrl->router_ticket[blockIdx.y])
+                 : "memory");
     s_last = (t == gridDim.x - 1);
   }
   __syncthreads();
   if (!s_last) return;
-  __threadfence();
   float* lsm = reinterpret_cast<float*>(smem_raw);  // this tile's logits
   {
     // every load of the tile in flight before the stores (the logits come from L2)
