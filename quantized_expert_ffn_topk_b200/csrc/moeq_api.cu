@@ -394,7 +394,10 @@ moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B,
   if (ws_bytes < moe_workspace_bytes(B, K, H, 32, E)) return MOE_ERR_WORKSPACE;
   if (!aligned16(x_bf16) || !aligned16(router_w_bf16) || !aligned16(ws)) return MOE_ERR_ALIGN;
   const size_t smem = std::max((size_t)std::min(B, kRouterTokTile) * H * 2, (size_t)std::min(B, kRouterTokTile) * E * 4);
-  if (ensure_smem(k_router_topk, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;
+  // a single token runs the one-token instance (one accumulator, a whole row's
+  // loads in flight); batches tile eight tokens per CTA
+  auto kern = B == 1 ? k_router_topk<1> : k_router_topk<kRouterTokTile>;
+  if (ensure_smem(kern, smem) != MOE_OK) return MOE_ERR_UNSUPPORTED;
   RouterParams p{};
   p.x = reinterpret_cast<const uint16_t*>(x_bf16);
   p.wr = reinterpret_cast<const uint16_t*>(router_w_bf16);
@@ -412,8 +415,8 @@ moe_status moe_router_topk(const void* x_bf16, const void* router_w_bf16, int B,
   static_assert(MOEQ_MAX_B / kRouterTokTile <= (int)(sizeof(WsCtrl::router_ticket) / sizeof(unsigned)),
                 "one router ticket per token tile");
   const int ctas = (E + kRouterWarps - 1) / kRouterWarps;
-  const dim3 grid(ctas, (B + kRouterTokTile - 1) / kRouterTokTile);
-  return launch_pdl(k_router_topk, grid, dim3(kRouterWarps * 32), smem, (cudaStream_t)stream, p);
+  const dim3 grid(ctas, (B + kRouterTokTile - 1) / kRouterTokTile);  // (B == 1: one tile either way)
+  return launch_pdl(kern, grid, dim3(kRouterWarps * 32), smem, (cudaStream_t)stream, p);
 }
 
 moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, const int32_t* idx, float* y_out,

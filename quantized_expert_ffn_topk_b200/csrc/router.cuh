@@ -256,6 +256,9 @@ __device__ __forceinline__ void topk_one_token(const float* lg, int E, int K, in
 // grid (E/kRouterWarps, ceil(B/kRouterTokTile)): CTA (c, j) dots rows of
 // warps c*kRouterWarps.. with tokens 8j..8j+7; the last CTA of column j to
 // finish selects for those tokens.
+// TT: tokens of a CTA's tile (kRouterTokTile, or 1 for a single token: then
+// one accumulator, and all of a row's 16-byte loads in flight at once).
+template <int TT>
 __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterParams p) {
   extern __shared__ __align__(16) unsigned char smem_raw[];
   uint16_t* xs = reinterpret_cast<uint16_t*>(smem_raw);  // [tok_tile, H]
@@ -264,7 +267,8 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterPara
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   const int gwarp = blockIdx.x * kRouterWarps + warp, nwarps = gridDim.x * kRouterWarps;
   const int nvec = p.H / 8;  // 16-byte words per row
-  const int b0 = blockIdx.y * kRouterTokTile, tb = min(kRouterTokTile, p.B - b0);
+  const int b0 = blockIdx.y * TT, tb = min(TT, p.B - b0);
+  constexpr int UNR = TT == 1 ? 2 * kRouterUnroll : kRouterUnroll;  // loads of a row in flight per lane
 
   if (threadIdx.x == 0) {
     mbar_init(&s_bar, 1);
@@ -292,26 +296,26 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterPara
   __syncthreads();
   for (int e = gwarp; e < p.E; e += nwarps) {
     const uint16_t* row = p.wr + (size_t)e * p.H;
-    float acc[kRouterTokTile];
+    float acc[TT];
 #pragma unroll
-    for (int t = 0; t < kRouterTokTile; ++t) acc[t] = 0.f;
-    for (int v0 = lane; v0 < nvec; v0 += 32 * kRouterUnroll) {
-      uint4 wv[kRouterUnroll];
+    for (int t = 0; t < TT; ++t) acc[t] = 0.f;
+    for (int v0 = lane; v0 < nvec; v0 += 32 * UNR) {
+      uint4 wv[UNR];
 #pragma unroll
-      for (int u = 0; u < kRouterUnroll; ++u)
+      for (int u = 0; u < UNR; ++u)
         if (v0 + 32 * u < nvec) wv[u] = ld_stream16(row + (size_t)(v0 + 32 * u) * 8);
 #pragma unroll
-      for (int u = 0; u < kRouterUnroll; ++u) {
+      for (int u = 0; u < UNR; ++u) {
         const int v = v0 + 32 * u;
         if (v < nvec) {
 #pragma unroll
-          for (int t = 0; t < kRouterTokTile; ++t)
+          for (int t = 0; t < TT; ++t)
             if (t < tb) acc[t] = dot8_bf16(wv[u], reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
         }
       }
     }
 #pragma unroll
-    for (int t = 0; t < kRouterTokTile; ++t) {
+    for (int t = 0; t < TT; ++t) {
       if (t < tb) {
         float sum = warp_sum(acc[t]);
         if (lane == 0) p.logits[(size_t)(b0 + t) * p.E + e] = sum;
