@@ -280,37 +280,46 @@ __global__ void __launch_bounds__(kRouterWarps * 32, 1) k_router_topk(RouterPara
     for (int e = gwarp; e < p.E; e += nwarps) prefetch_l2(p.wr + (size_t)e * p.H, (uint32_t)p.H * 2);
   __syncthreads();
   pdl_wait();
-  // the token tile's x rows (contiguous) in one bulk copy; bounded wait
-  if (threadIdx.x == 0) {
-    const uint32_t bytes = (uint32_t)tb * (uint32_t)p.H * 2u;
-    mbar_arrive_expect_tx(&s_bar, bytes);
-    bulk_g2s(xs, p.x + (size_t)b0 * p.H, bytes, &s_bar);
-  }
-  {
+  // the token tile's x rows (contiguous) in one bulk copy; bounded wait (one
+  // token reads its x at L2 beside each row's loads instead: no wait first)
+  if (TT > 1) {
+    if (threadIdx.x == 0) {
+      const uint32_t bytes = (uint32_t)tb * (uint32_t)p.H * 2u;
+      mbar_arrive_expect_tx(&s_bar, bytes);
+      bulk_g2s(xs, p.x + (size_t)b0 * p.H, bytes, &s_bar);
+    }
     const long long budget = wait_budget(p.ctrl);
     const long long t0 = clock64();
     bool ok;
     while (!(ok = mbar_try_wait(&s_bar, 0u)) && clock64() - t0 < budget) __nanosleep(32);
     if (!ok && threadIdx.x == 0) set_error(p.ctrl, MOE_ERR_TIMEOUT);
+    __syncthreads();
   }
-  __syncthreads();
+  const uint4* x1 = reinterpret_cast<const uint4*>(p.x + (size_t)b0 * p.H);
   for (int e = gwarp; e < p.E; e += nwarps) {
     const uint16_t* row = p.wr + (size_t)e * p.H;
     float acc[TT];
 #pragma unroll
     for (int t = 0; t < TT; ++t) acc[t] = 0.f;
     for (int v0 = lane; v0 < nvec; v0 += 32 * UNR) {
-      uint4 wv[UNR];
+      uint4 wv[UNR], xv[TT == 1 ? UNR : 1];
 #pragma unroll
       for (int u = 0; u < UNR; ++u)
-        if (v0 + 32 * u < nvec) wv[u] = ld_stream16(row + (size_t)(v0 + 32 * u) * 8);
+        if (v0 + 32 * u < nvec) {
+          wv[u] = ld_stream16(row + (size_t)(v0 + 32 * u) * 8);
+          if constexpr (TT == 1) xv[u] = __ldcg(x1 + v0 + 32 * u);
+        }
 #pragma unroll
       for (int u = 0; u < UNR; ++u) {
         const int v = v0 + 32 * u;
         if (v < nvec) {
+          if constexpr (TT == 1) {
+            acc[0] = dot8_bf16(wv[u], xv[u], acc[0]);
+          } else {
 #pragma unroll
-          for (int t = 0; t < TT; ++t)
-            if (t < tb) acc[t] = dot8_bf16(wv[u], reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
+            for (int t = 0; t < TT; ++t)
+              if (t < tb) acc[t] = dot8_bf16(wv[u], reinterpret_cast<const uint4*>(xs + (size_t)t * p.H)[v], acc[t]);
+          }
         }
       }
     }
