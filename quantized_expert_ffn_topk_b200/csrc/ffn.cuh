@@ -18,7 +18,17 @@
 namespace moeq {
 
 constexpr int kFfnWarps = 16;
-constexpr int kFfnPieces = 4;     // pieces of a tile: each takes a quarter of its groups
+// Pieces of a tile (each a contiguous part of its groups, one warp each): a
+// CTA's share of 4 or 5 gate/up tiles in 3 pieces is one wave of the 16 warps
+// (in 4, five tiles took two); down jobs stay in 4 (5 or 8 measured no faster)
+#ifndef MOEQ_FFN_PIECES_GU
+#define MOEQ_FFN_PIECES_GU 3
+#endif
+#ifndef MOEQ_FFN_PIECES_DN
+#define MOEQ_FFN_PIECES_DN 4
+#endif
+constexpr int kFfnPiecesGu = MOEQ_FFN_PIECES_GU;
+constexpr int kFfnPiecesDn = MOEQ_FFN_PIECES_DN;
 constexpr int kFfnMaxBuf = 32;    // tile buffers (mbarriers) per CTA
 
 struct FfnParams {
@@ -42,8 +52,9 @@ struct FfnParams {
   int dot_fma, gu_xf, dn_img_xf;
 };
 
-// Groups [lo, hi) of piece q of a tile with ng groups.
-__host__ __device__ inline int piece_lo(int q, int ng) { return q * ng / kFfnPieces; }
+// Groups [lo, hi) of piece q of NP of a tile with ng groups.
+template <int NP>
+__host__ __device__ inline int piece_lo(int q, int ng) { return q * ng / NP; }
 
 // Record of slot k of the token (routed expert idx[k], or the shared expert
 // for k == K); null for an invalid expert index.
@@ -151,13 +162,13 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
           p.H, p.G, X, tid, blockDim.x);
       __syncthreads();
     }
-    for (int pc = warp; pc < nt * kFfnPieces; pc += kFfnWarps) {
-      const int j = pc / kFfnPieces, q = pc % kFfnPieces, k = (r0 + j) / tps;
+    for (int pc = warp; pc < nt * kFfnPiecesGu; pc += kFfnWarps) {
+      const int j = pc / kFfnPiecesGu, q = pc % kFfnPiecesGu, k = (r0 + j) / tps;
       const bool routed = k < p.K;
       float acc0 = 0.f, acc1 = 0.f;
       if (ffn_wait(bar, j, round, p.ctrl, &s_abort, budget) && ffn_slot_rec(p, k)) {
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
-        const int g0 = piece_lo(q, (int)g.ng_h), g1 = piece_lo(q + 1, (int)g.ng_h);
+        const int g0 = piece_lo<kFfnPiecesGu>(q, (int)g.ng_h), g1 = piece_lo<kFfnPiecesGu>(q + 1, (int)g.ng_h);
         const unsigned char* blk = tiles + (size_t)j * p.gu_stride + (size_t)g0 * g.blk;
         const float* xf = reinterpret_cast<const float*>(smem + p.gu_xf);
         with_fmt(routed ? p.bits_r : p.bits_s, p.G, [&]<int BITS, int KS>() {
@@ -166,7 +177,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
         });
       }
       if ((lane & 3) == 0) {
-        float* pp = part + ((size_t)j * kFfnPieces + q) * kTileRows;
+        float* pp = part + ((size_t)j * kFfnPiecesGu + q) * kTileRows;
         pp[lane >> 2] = acc0;
         pp[(lane >> 2) + 8] = acc1;
       }
@@ -176,9 +187,9 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_gate_up(const __grid_cons
       const int j = i / 8, unit = i % 8, u = r0 + j, k = u / tps, T = u % tps;
       float gate = 0.f, up = 0.f;
 #pragma unroll
-      for (int q = 0; q < kFfnPieces; ++q) {
-        gate += part[((size_t)j * kFfnPieces + q) * kTileRows + unit];
-        up += part[((size_t)j * kFfnPieces + q) * kTileRows + 8 + unit];
+      for (int q = 0; q < kFfnPiecesGu; ++q) {
+        gate += part[((size_t)j * kFfnPiecesGu + q) * kTileRows + unit];
+        up += part[((size_t)j * kFfnPiecesGu + q) * kTileRows + 8 + unit];
       }
       const bool ok = ffn_slot_rec(p, k) != nullptr;
       if (!ok && unit == 0) set_error(p.ctrl, MOE_ERR_INDEX);
@@ -248,13 +259,13 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
       }
       __syncthreads();
     }
-    for (int pc = warp; pc < nt * kFfnPieces; pc += kFfnWarps) {
-      const int j = pc / kFfnPieces, q = pc % kFfnPieces, k = (r0 + j) / tpd;
+    for (int pc = warp; pc < nt * kFfnPiecesDn; pc += kFfnWarps) {
+      const int j = pc / kFfnPiecesDn, q = pc % kFfnPiecesDn, k = (r0 + j) / tpd;
       const bool routed = k < p.K;
       float acc0 = 0.f, acc1 = 0.f;
       if (ffn_wait(bar, j, round, p.ctrl, &s_abort, budget) && ffn_slot_rec(p, k)) {
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
-        const int g0 = piece_lo(q, (int)g.ng_i), g1 = piece_lo(q + 1, (int)g.ng_i);
+        const int g0 = piece_lo<kFfnPiecesDn>(q, (int)g.ng_i), g1 = piece_lo<kFfnPiecesDn>(q + 1, (int)g.ng_i);
         const unsigned char* blk = tiles + (size_t)j * p.dn_stride + (size_t)g0 * g.blk;
         const QImg Hk = img(k);
         const float* hf = reinterpret_cast<const float*>(smem + (size_t)k * p.dn_img_stride + p.dn_img_xf);
@@ -264,7 +275,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
         });
       }
       if ((lane & 3) == 0) {
-        float* pp = part + ((size_t)j * kFfnPieces + q) * kTileRows;
+        float* pp = part + ((size_t)j * kFfnPiecesDn + q) * kTileRows;
         pp[lane >> 2] = acc0;
         pp[(lane >> 2) + 8] = acc1;
       }
@@ -274,7 +285,7 @@ __global__ void __launch_bounds__(kFfnWarps * 32, 1) k_down(const __grid_constan
       const int j = i / kTileRows, rho = i % kTileRows, u = r0 + j, k = u / tpd, T = u % tpd;
       float y = 0.f;
 #pragma unroll
-      for (int q = 0; q < kFfnPieces; ++q) y += part[((size_t)j * kFfnPieces + q) * kTileRows + rho];
+      for (int q = 0; q < kFfnPiecesDn; ++q) y += part[((size_t)j * kFfnPiecesDn + q) * kTileRows + rho];
       p.y[(size_t)k * p.H + (size_t)T * kTileRows + rho] = y;
     }
     __syncthreads();

@@ -560,7 +560,7 @@ bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes) {
   if (p.dot_fma) o += align_up((size_t)p.H * 4, 128);
   const int gu_want = std::min(kFfnMaxBuf, cdiv(gu_total, std::min(G, gu_total)));
   p.gu_part = (int)o;
-  o += align_up((size_t)gu_want * kFfnPieces * kTileRows * 4, 128);
+  o += align_up((size_t)gu_want * kFfnPiecesGu * kTileRows * 4, 128);
   p.gu_tiles = (int)o;
   p.gu_stride = (int)align_up(std::max(p.geo_r.U, p.geo_s.U), 128);
   if (o + (size_t)p.gu_stride > budget) return false;
@@ -573,7 +573,7 @@ bool ffn_plan(FfnParams& p, int G, size_t& gu_bytes, size_t& dn_bytes) {
   o = (size_t)p.dn_img_stride * (p.K + 1);
   const int dn_want = std::min(kFfnMaxBuf, cdiv(dn_total, std::min(G, dn_total)));
   p.dn_part = (int)o;
-  o += align_up((size_t)dn_want * kFfnPieces * kTileRows * 4, 128);
+  o += align_up((size_t)dn_want * kFfnPiecesDn * kTileRows * 4, 128);
   p.dn_tiles = (int)o;
   p.dn_stride = (int)align_up(std::max(p.geo_r.D, p.geo_s.D), 128);
   if (o + (size_t)p.dn_stride > budget) return false;
