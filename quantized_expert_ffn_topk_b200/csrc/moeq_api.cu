@@ -633,7 +633,8 @@ bool stack_plan(StackParams& p, int G, size_t static_smem) {
   const int ntiles_max = cdiv(I / 8, G) + cdiv(K * (I / 8), G) + 1;
   const int nd_max = cdiv(H / kTileRows, G);
   if (ntiles_max > kMaxTiles || nd_max > kMaxDnTiles) return false;
-  p.sm_gpart = take((size_t)ntiles_max * kGuPieces * kTileRows * 4);
+  p.sm_gpart = take(((size_t)cdiv(I / 8, G) * kGuPiecesShared + (size_t)(cdiv(K * (I / 8), G) + 1) * kGuPieces) *
+                    kTileRows * 4);
   p.sm_dpart = take((size_t)nd_max * (K + 1) * kDnPieces * kTileRows * 4);
   // a ring slot holds two router rows, half of a gate/up tile or the CTA's
   // down tiles of one slot

@@ -42,13 +42,24 @@ constexpr int kStackMaxLayers = 64;
 constexpr int kCWarps = 16;                      // compute warps
 constexpr int kCThreads = kCWarps * 32;
 constexpr int kStackThreads = kCThreads + 32;    // + producer warp
+// The compute warp that publishes a phase's results (the release-add of a
+// grid exchange waits until the CTA's writes are acknowledged, so it falls to
+// the last warp, which takes a piece of the next phase last or not at all).
+constexpr int kSigWarp = kCWarps - 1;
 constexpr int kMaxSlots = 16;
 constexpr int kMaxRouterRowsPerCta = 8;
 constexpr int kRouterPieces = 4;                 // a router row is dotted in quarters
-constexpr int kGuPieces = 4;                     // pieces of a gate/up tile (2 per ring item)
+constexpr int kGuPieces = 4;                     // pieces of a routed gate/up tile (2 per ring item)
+// pieces of a shared-expert gate/up tile: a CTA holds at most one or two of
+// them, so four pieces would leave most warps idle before the top-K
+#ifndef MOEQ_STACK_SHARED_PIECES
+#define MOEQ_STACK_SHARED_PIECES 8
+#endif
+constexpr int kGuPiecesShared = MOEQ_STACK_SHARED_PIECES;
 constexpr int kDnPieces = 4;                     // pieces of a (down tile, slot) job
 constexpr int kMaxDnTiles = 4;                   // down tiles per CTA
 constexpr int kItemPieces = kDnPieces * kMaxDnTiles;  // pieces of the largest item (a down item)
+static_assert(kGuPiecesShared % 2 == 0 && kGuPiecesShared / 2 <= kItemPieces, "a ring item holds half of a tile's pieces");
 constexpr int kMaxItems = 32;
 constexpr int kMaxPieces = kMaxItems * kItemPieces;
 constexpr int kMaxTiles = 16;                    // gate/up tiles per CTA per layer
@@ -139,6 +150,7 @@ struct ItemPlan {
   int half[kMaxItems];                     // which half of the tile's groups
   int npieces[kMaxItems];
   int piece0[kMaxItems];
+  int nst;                                 // shared gate/up tiles (CTA-local tiles 0..nst-1)
   int r0, nr;                              // router rows [r0, r0+nr)
   int d0, nd;                              // down tiles [d0, d0+nd)
   int ntiles;
@@ -171,9 +183,9 @@ __device__ void make_plan(const StackParams& p, ItemPlan& P) {
       P.tile[n] = T;
       P.tl[n] = tl;
       P.half[n] = h;
-      P.npieces[n] = 2;
+      P.npieces[n] = k == p.K ? kGuPiecesShared / 2 : kGuPieces / 2;
       P.piece0[n] = pc;
-      pc += 2;
+      pc += P.npieces[n];
       ++n;
     }
     ++tl;
@@ -194,6 +206,7 @@ __device__ void make_plan(const StackParams& p, ItemPlan& P) {
   const int tps = p.I / 8;  // gate/up tiles per slot
 #pragma unroll 1
   for (int T = share_lo(c, G, tps); T < share_lo(c + 1, G, tps); ++T) add_tile(p.K, T);
+  P.nst = tl;
   P.n_sgu_items = n;
   if (P.nd > 0) add_down(p.K);
   P.n_pre_items = n;
@@ -500,19 +513,24 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
           dp[(lane >> 2) + 8] = acc1;
         }
       } else {
-        const int k = P.k[it], tl = P.tl[it], q = 2 * P.half[it] + pos;
+        const int k = P.k[it], tl = P.tl[it], npi = P.npieces[it], npt = 2 * npi, q = npi * P.half[it] + pos;
         const bool routed = k < K;
         const bool valid = ok && (!routed || s_idx[k] >= 0);
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
-        const int ga = quarter_lo(2 * P.half[it], (int)g.ng_h);
-        const int g0 = quarter_lo(q, (int)g.ng_h), g1 = quarter_lo(q + 1, (int)g.ng_h);
+        const int ng = (int)g.ng_h;
+        const int ga = quarter_lo(2 * P.half[it], ng);
+        const int g0 = q * ng / npt, g1 = (q + 1) * ng / npt;
+        // the tile's partial sums: shared tiles (first) hold kGuPiecesShared pieces, routed ones kGuPieces
+        float* g4 = gpart + (tl < P.nst ? (size_t)tl * kGuPiecesShared
+                                        : (size_t)P.nst * kGuPiecesShared + (size_t)(tl - P.nst) * kGuPieces) *
+                                kTileRows;
         float acc0 = 0.f, acc1 = 0.f;
         if (valid) {
           const unsigned char* blk = sl + (size_t)(g0 - ga) * g.blk;
           with_fixed_fmt<BR, BS, KS>(
               routed, [&]<int BITS, int KS_>() { tile_dot<BITS, KS_>(blk, g1 - g0, g0, X, acc0, acc1); });
         }
-        float* gp = gpart + ((size_t)tl * kGuPieces + q) * kTileRows;
+        float* gp = g4 + (size_t)q * kTileRows;
         if ((lane & 3) == 0) {
           gp[lane >> 2] = acc0;
           gp[(lane >> 2) + 8] = acc1;
@@ -522,13 +540,11 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         int prev = 0;
         if (lane == 0) prev = atomicAdd(&s_gcnt[tl], 1);
         prev = __shfl_sync(0xFFFFFFFFu, prev, 0);
-        if (prev == kGuPieces - 1) {  // the tile's last piece: finish its 8 units
+        if (prev == npt - 1) {  // the tile's last piece: finish its 8 units
           __threadfence_block();
           if (lane < 8) {
-            const float* g4 = gpart + (size_t)tl * kGuPieces * kTileRows;
             float gate = 0.f, up = 0.f;
-#pragma unroll
-            for (int qq = 0; qq < kGuPieces; ++qq) {
+            for (int qq = 0; qq < npt; ++qq) {
               gate += g4[qq * kTileRows + lane];
               up += g4[qq * kTileRows + 8 + lane];
             }
@@ -645,7 +661,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       // ---- router pieces, then the shared expert's gate/up pieces ----
       run_items(l, 0, P.n_router_items);
       named_sync(1, kCThreads);
-      if (warp == 0) {
+      if (warp == kSigWarp) {
         if (lane < P.nr) {
           float lg = 0.f;
 #pragma unroll
@@ -658,7 +674,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       STACK_MARK(tid == 0, l, 3);
       run_items(l, P.n_router_items, P.n_sgu_items);
       named_sync(1, kCThreads);
-      if (tid == 0) arrive_release_gpu(p.sync + kSyncSharedH);
+      if (tid == kSigWarp * 32) arrive_release_gpu(p.sync + kSyncSharedH);
       STACK_MARK(tid == 0, l, 4);
 
       // ---- softmax / top-K over every CTA's logits (the producer waits for it) ----
@@ -692,7 +708,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       // ---- routed gate/up pieces ----
       run_items(l, P.n_pre_items, P.n_rgu_items);
       named_sync(1, kCThreads);
-      if (tid == 0) arrive_release_gpu(p.sync + kSyncRoutedH);
+      if (tid == kSigWarp * 32) arrive_release_gpu(p.sync + kSyncRoutedH);
       STACK_MARK(tid == 0, l, 9);
 #ifdef MOEQ_STACK_TRACE
       if (tid == 0 && p.trace) {
@@ -735,7 +751,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         if (lane == 0) s_red[0][warp] = sq;
       }
       named_sync(1, kCThreads);
-      if (tid == 0) {
+      if (tid == kSigWarp * 32) {
         float t = 0.f;
         for (int w = 0; w < kCWarps; ++w) t += s_red[0][w];
         __stcg(p.ss_part + blockIdx.x, t);
