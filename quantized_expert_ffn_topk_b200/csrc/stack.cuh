@@ -49,7 +49,12 @@ constexpr int kSigWarp = kCWarps - 1;
 constexpr int kMaxSlots = 16;
 constexpr int kMaxRouterRowsPerCta = 8;
 constexpr int kRouterPieces = 4;                 // a router row is dotted in quarters
-constexpr int kGuPieces = 4;                     // pieces of a routed gate/up tile (2 per ring item)
+// (a CTA holds 3 or 4 routed gate/up tiles: 4 pieces each fill the 16 warps;
+// 8 pieces, a shorter tail after the last tile lands, measured no faster)
+#ifndef MOEQ_STACK_ROUTED_PIECES
+#define MOEQ_STACK_ROUTED_PIECES 4
+#endif
+constexpr int kGuPieces = MOEQ_STACK_ROUTED_PIECES;  // pieces of a routed gate/up tile (half per ring item)
 // pieces of a shared-expert gate/up tile: a CTA holds at most one or two of
 // them, so four pieces would leave most warps idle before the top-K
 #ifndef MOEQ_STACK_SHARED_PIECES
@@ -59,7 +64,9 @@ constexpr int kGuPiecesShared = MOEQ_STACK_SHARED_PIECES;
 constexpr int kDnPieces = 4;                     // pieces of a (down tile, slot) job
 constexpr int kMaxDnTiles = 4;                   // down tiles per CTA
 constexpr int kItemPieces = kDnPieces * kMaxDnTiles;  // pieces of the largest item (a down item)
-static_assert(kGuPiecesShared % 2 == 0 && kGuPiecesShared / 2 <= kItemPieces, "a ring item holds half of a tile's pieces");
+static_assert(kGuPiecesShared % 2 == 0 && kGuPiecesShared / 2 <= kItemPieces && kGuPieces % 2 == 0 &&
+                  kGuPieces / 2 <= kItemPieces,
+              "a ring item holds half of a tile's pieces");
 constexpr int kMaxItems = 32;
 constexpr int kMaxPieces = kMaxItems * kItemPieces;
 constexpr int kMaxTiles = 16;                    // gate/up tiles per CTA per layer
