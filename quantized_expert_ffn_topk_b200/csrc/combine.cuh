@@ -25,22 +25,80 @@ struct CombineParams {
   float eps;
 };
 
+// Cluster shared-memory helpers: the address of the same variable in CTA
+// `rank` of the cluster, a 4-byte store into it that completes `bytes` on
+// that CTA's mbarrier, and a bounded wait on a local mbarrier phase whose
+// data came from the cluster's CTAs.
+__device__ __forceinline__ uint32_t cluster_addr(const void* p, uint32_t rank) {
+  uint32_t r;
+  asm volatile("mapa.shared::cluster.u32 %0, %1, %2;" : "=r"(r) : "r"(smem_u32(p)), "r"(rank));
+  return r;
+}
+__device__ __forceinline__ void st_async_f32(uint32_t dst, float v, uint32_t bar) {
+  asm volatile("st.async.shared::cluster.mbarrier::complete_tx::bytes.b32 [%0], %1, [%2];" ::"r"(dst),
+               "r"(__float_as_uint(v)), "r"(bar)
+               : "memory");
+}
+__device__ __forceinline__ bool mbar_wait_cluster(uint64_t* bar, uint32_t parity, long long budget) {
+  const long long t0 = clock64();
+  while (true) {
+    uint32_t ok;
+    asm volatile(
+        "{ .reg .pred p;\n\t mbarrier.try_wait.parity.acquire.cluster.shared::cta.b64 p, [%1], %2;\n\t selp.u32 %0, 1, "
+        "0, p; }"
+        : "=r"(ok)
+        : "r"(smem_u32(bar)), "r"(parity)
+        : "memory");
+    if (ok) return true;
+    if (clock64() - t0 > budget) return false;
+  }
+}
+
 // grid: B clusters of kCombineCluster CTAs, one cluster per token; CTA rank
 // q of a cluster owns elements [q*per, (q+1)*per) of its token (per =
 // ceil(H / kCombineCluster)), one or a few per thread. The RMSNorm'd copy
-// needs the token's whole sum of squares: each CTA reduces its part in
-// shared memory and reads its cluster peers' parts through distributed
-// shared memory (two cluster barriers; every CTA reaches both).
+// needs the token's whole sum of squares: each CTA reduces its part and
+// stores it into every cluster peer's shared memory (st.async, counted on
+// the peer's mbarrier), then adds the parts in rank order once its own
+// barrier has them all. The only cluster barrier comes first (the peers'
+// mbarriers armed, nothing stored yet), so no fence waits on the global
+// stores of r; a CTA leaves only after every peer's part has landed in it.
+// The first element of each thread has its inputs loaded before the gate's
+// reduction. A part that never lands (after about a second) leaves the
+// CTA's share of the bf16 copy NaN.
 __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombineThreads)
     k_combine(CombineParams p) {
   __shared__ float red[32];
-  __shared__ float s_part;
+  __shared__ float s_parts[kCombineCluster];
+  __shared__ __align__(8) uint64_t s_bar;
   namespace cg = cooperative_groups;
   cg::cluster_group cluster = cg::this_cluster();
   const int b = blockIdx.x / kCombineCluster, q = (int)cluster.block_rank();
+  if (p.xnorm) {
+    if (threadIdx.x == 0) {
+      mbar_init(&s_bar, 1);
+      fence_mbar_init();
+      mbar_arrive_expect_tx(&s_bar, kCombineCluster * (uint32_t)sizeof(float));
+    }
+    cluster.sync();  // every peer's barrier is armed before any part is sent
+  }
   pdl_trigger();
   pdl_wait();
   const uint16_t* xb = p.x + (size_t)b * p.H;
+  const float* yb = p.y + (size_t)b * (p.K + 1) * p.H;
+  float* rb = p.resid_out + (size_t)b * p.H;
+  const int per = (p.H + kCombineCluster - 1) / kCombineCluster;
+  const int j0 = q * per, j1 = min(p.H, j0 + per);
+  const int ja = j0 + (int)threadIdx.x;
+  float ra = 0.f, ya[MOEQ_MAX_K + 1];
+#pragma unroll
+  for (int k = 0; k <= MOEQ_MAX_K; ++k) ya[k] = 0.f;
+  if (ja < j1) {
+    ra = p.resid_in ? p.resid_in[(size_t)b * p.H + ja] : bf16_bits_to_f32(xb[ja]);
+#pragma unroll
+    for (int k = 0; k <= MOEQ_MAX_K; ++k)
+      if (k <= p.K) ya[k] = yb[(size_t)k * p.H + ja];
+  }
   float gamma = 1.f;
   if (p.gate_w) {
     float a = 0.f;
@@ -53,34 +111,36 @@ __global__ void __cluster_dims__(kCombineCluster, 1, 1) __launch_bounds__(kCombi
   float wk[MOEQ_MAX_K + 1];
 #pragma unroll
   for (int k = 0; k <= MOEQ_MAX_K; ++k) wk[k] = k < p.K ? p.w[(size_t)b * p.K + k] : (k == p.K ? gamma : 0.f);
-  const float* yb = p.y + (size_t)b * (p.K + 1) * p.H;
-  float* rb = p.resid_out + (size_t)b * p.H;
-  const int per = (p.H + kCombineCluster - 1) / kCombineCluster;
-  const int j0 = q * per, j1 = min(p.H, j0 + per);
   float ss = 0.f, keep = 0.f;
-  for (int j = j0 + (int)threadIdx.x; j < j1; j += blockDim.x) {
+  if (ja < j1) {
+    float acc = ra;
+#pragma unroll
+    for (int k = 0; k <= MOEQ_MAX_K; ++k)
+      if (k <= p.K) acc += wk[k] * ya[k];
+    keep = acc;
+    rb[ja] = acc;
+    ss += acc * acc;
+  }
+  for (int j = ja + (int)blockDim.x; j < j1; j += blockDim.x) {
     float acc = p.resid_in ? p.resid_in[(size_t)b * p.H + j] : bf16_bits_to_f32(xb[j]);
 #pragma unroll
     for (int k = 0; k <= MOEQ_MAX_K; ++k)
       if (k <= p.K) acc += wk[k] * yb[(size_t)k * p.H + j];
-    if (j == j0 + (int)threadIdx.x) keep = acc;
     rb[j] = acc;
     ss += acc * acc;
   }
   if (p.xnorm) {
     ss = block_sum(ss, red);
-    if (threadIdx.x == 0) s_part = ss;
-  }
-  cluster.sync();  // every CTA's part is in its shared memory
-  if (p.xnorm) {
+    if (threadIdx.x < kCombineCluster)  // thread r sends this CTA's part to rank r
+      st_async_f32(cluster_addr(&s_parts[q], threadIdx.x), ss, cluster_addr(&s_bar, threadIdx.x));
+    const bool ok = mbar_wait_cluster(&s_bar, 0, kWaitBudgetCycles);
     float tot = 0.f;
-    for (int r = 0; r < kCombineCluster; ++r) tot += *cluster.map_shared_rank(&s_part, r);
-    const float inv = rsqrtf(tot / (float)p.H + p.eps);
+#pragma unroll
+    for (int r = 0; r < kCombineCluster; ++r) tot += s_parts[r];
+    const float inv = ok ? rsqrtf(tot / (float)p.H + p.eps) : __int_as_float(0x7FC00000);
     uint16_t* xn = p.xnorm + (size_t)b * p.H;
-    for (int j = j0 + (int)threadIdx.x; j < j1; j += blockDim.x)
-      xn[j] = f32_to_bf16_bits((j == j0 + (int)threadIdx.x ? keep : rb[j]) * inv);
+    for (int j = ja; j < j1; j += blockDim.x) xn[j] = f32_to_bf16_bits((j == ja ? keep : rb[j]) * inv);
   }
-  cluster.sync();  // peers' reads of this CTA's shared memory are done before it leaves
 }
 
 // moe_rmsnorm: grid B, one token per CTA. xn = bf16(r * rsqrt(mean(r^2) +

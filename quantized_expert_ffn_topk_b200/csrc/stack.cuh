@@ -117,9 +117,12 @@ struct StackParams {
 // thread per CTA stamps %globaltimer at phase ends into
 // trace[(layer * kTracePhases + phase) * G + cta]. Off in the library build.
 // 14, 15: first/last routed gate/up item landed; 16: longest such piece (ns);
-// 19, 20: x staging loads back / image written; 22, 23: the copy warp done
-// issuing layer l's routed items / the next layer's items
-constexpr int kTracePhases = 24;
+// 17, 18: routed h counter seen / its loads back; 19, 20: x staging loads
+// back / image written; 21: the routed h arrival made; 22, 23: the copy
+// warp done issuing layer l's routed items / the next layer's items;
+// 24, 25: first routed down piece started / last one done; 26: longest such
+// piece (ns)
+constexpr int kTracePhases = 27;
 #ifdef MOEQ_STACK_TRACE
 #define STACK_MARK(cond, l, ph)                                                                    \
   do {                                                                                             \
@@ -372,12 +375,12 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
   __shared__ volatile int s_abort;
   __shared__ volatile int s_topk_ready;
   __shared__ volatile int s_logits_ready;  // layer + 1 once s_logits holds that layer's logits
+  __shared__ volatile int s_rh_arrived;    // layer + 1 once this CTA's routed h arrival is made
 #ifdef MOEQ_STACK_TRACE
-  __shared__ unsigned long long s_tr[3];
+  __shared__ unsigned long long s_tr[6];
   if (threadIdx.x == 0) {
-    s_tr[0] = ~0ull;
-    s_tr[1] = 0ull;
-    s_tr[2] = 0ull;
+    s_tr[0] = s_tr[3] = ~0ull;
+    s_tr[1] = s_tr[2] = s_tr[4] = s_tr[5] = 0ull;
   }
 #endif
   __shared__ __align__(16) float s_logits[kStackMaxE];
@@ -404,6 +407,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     s_abort = 0;
     s_topk_ready = 0;
     s_logits_ready = 0;
+    s_rh_arrived = 0;
     fence_mbar_init();
   }
   __syncthreads();
@@ -437,10 +441,25 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       STACK_MARK(lane == 0, l, 13);
       // routed gate/up items (they gate the h exchange), the routed down
       // items (needed only after it), then the next layer's router, shared
-      // gate/up and shared down items
+      // gate/up and shared down items. What follows the gate/up items waits
+      // for this CTA's routed h arrival: a gpu-scope release waits for the
+      // CTA's bulk copies in flight, so copies issued before it would hold
+      // up the arrival that every CTA waits for.
       const uint32_t seq_l = (uint32_t)(l * n_items);
+#if MOEQ_STACK_HOLD_DOWN
+      bool ok = !s_abort && issue_items(p, P, R, l, P.n_pre_items, P.n_rgu_items, seq_l + P.n_pre_items, s_idx,
+                                        &s_abort, budget);
+      if (ok && lane == 0 && !flag_wait(&s_rh_arrived, l + 1, &s_abort, budget) && !s_abort) fail();
+      __syncwarp();
+      ok = ok && !s_abort &&
+           issue_items(p, P, R, l, P.n_rgu_items, n_items, seq_l + P.n_rgu_items, s_idx, &s_abort, budget);
+      STACK_MARK(lane == 0, l, 22);
+#else
       bool ok = !s_abort && issue_items(p, P, R, l, P.n_pre_items, n_items, seq_l + P.n_pre_items, s_idx, &s_abort, budget);
       STACK_MARK(lane == 0, l, 22);
+      if (ok && l + 1 < p.n_layers && lane == 0 && !flag_wait(&s_rh_arrived, l + 1, &s_abort, budget) && !s_abort) fail();
+      __syncwarp();
+#endif
       if (ok && l + 1 < p.n_layers)
         ok = issue_items(p, P, R, l + 1, 0, P.n_pre_items, (uint32_t)((l + 1) * n_items), s_idx, &s_abort, budget);
       STACK_MARK(lane == 0, l, 23);
@@ -503,6 +522,10 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         acc = warp_sum(acc);
         if (lane == 0) s_rpart[P.tile[it] + row][qr] = acc;
       } else if (P.kind[it] == kItemDown) {
+#ifdef MOEQ_STACK_TRACE
+        unsigned long long t_dn0 = 0;
+        if (P.k[it] < K && lane == 0) asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_dn0));
+#endif
         const int k = P.k[it], q = pos % kDnPieces, j = pos / kDnPieces;
         const bool routed = k < K;
         const RecGeom& g = routed ? p.geo_r : p.geo_s;
@@ -519,6 +542,15 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
           dp[lane >> 2] = acc0;
           dp[(lane >> 2) + 8] = acc1;
         }
+#ifdef MOEQ_STACK_TRACE
+        if (routed && lane == 0) {
+          unsigned long long t_dn1;
+          asm volatile("mov.u64 %0, %%globaltimer;" : "=l"(t_dn1));
+          atomicMin(&s_tr[3], t_dn0);
+          atomicMax(&s_tr[4], t_dn1);
+          atomicMax(&s_tr[5], t_dn1 - t_dn0);
+        }
+#endif
       } else {
         const int k = P.k[it], tl = P.tl[it], npi = P.npieces[it], npt = 2 * npi, q = npi * P.half[it] + pos;
         const bool routed = k < K;
@@ -586,8 +618,9 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
     // part of them out (counter `c` at `target`). Each lane stages its own
     // segment into its own slot's image; a group's lanes are adjacent and
     // share a slot (I is a multiple of G).
-    auto stage_h = [&](int k0, int k1, int c, unsigned target) {
+    auto stage_h = [&](int l, int k0, int k1, int c, unsigned target) {
       if (tid == 0 && !counter_wait(p.sync + c, target, &s_abort, budget) && !s_abort) fail();
+      STACK_MARK(tid == 0 && k0 == 0, l, 17);
       named_sync(1, kCThreads);
       const int spk = I / 16;  // segments per slot
       for (int s0 = tid - lane; s0 < (k1 - k0) * spk; s0 += kCThreads) {
@@ -597,6 +630,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
         float v[16];
         if (active) {
           load_f32_16_cg(p.h + (size_t)k * I + (size_t)sk * 16, v);
+          STACK_MARK(tid == 0 && k0 == 0 && s0 == 0 && v[0] == v[0], l, 18);
         } else {
 #pragma unroll
           for (int j = 0; j < 16; ++j) v[j] = 0.f;
@@ -706,7 +740,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       STACK_MARK(tid == 0, l, 6);
 
       // ---- the shared expert's down tiles, once every CTA's shared h is out ----
-      stage_h(K, K + 1, kSyncSharedH, (unsigned)(l + 1) * G1);
+      stage_h(l, K, K + 1, kSyncSharedH, (unsigned)(l + 1) * G1);
       named_sync(1, kCThreads);
       STACK_MARK(tid == 0, l, 7);
       run_items(l, P.n_sgu_items, P.n_pre_items);
@@ -715,7 +749,11 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       // ---- routed gate/up pieces ----
       run_items(l, P.n_pre_items, P.n_rgu_items);
       named_sync(1, kCThreads);
-      if (tid == kSigWarp * 32) arrive_release_gpu(p.sync + kSyncRoutedH);
+      if (tid == kSigWarp * 32) {
+        arrive_release_gpu(p.sync + kSyncRoutedH);
+        s_rh_arrived = l + 1;
+      }
+      STACK_MARK(tid == kSigWarp * 32, l, 21);
       STACK_MARK(tid == 0, l, 9);
 #ifdef MOEQ_STACK_TRACE
       if (tid == 0 && p.trace) {
@@ -730,12 +768,23 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
 #endif
 
       // ---- routed down tiles ----
-      stage_h(0, K, kSyncRoutedH, (unsigned)(l + 1) * G1);
+      stage_h(l, 0, K, kSyncRoutedH, (unsigned)(l + 1) * G1);
       named_sync(1, kCThreads);
       STACK_MARK(tid == 0, l, 10);
       run_items(l, P.n_rgu_items, n_items);
       named_sync(1, kCThreads);
       STACK_MARK(tid == 0, l, 11);
+#ifdef MOEQ_STACK_TRACE
+      if (tid == 0 && p.trace) {
+        const size_t at = (size_t)l * kTracePhases * gridDim.x + blockIdx.x;
+        p.trace[at + (size_t)24 * gridDim.x] = s_tr[3];
+        p.trace[at + (size_t)25 * gridDim.x] = s_tr[4];
+        p.trace[at + (size_t)26 * gridDim.x] = s_tr[5];
+        s_tr[3] = ~0ull;
+        s_tr[4] = 0ull;
+        s_tr[5] = 0ull;
+      }
+#endif
 
       // ---- combine: r_{l+1} = r_l + sum_k w_k y_k + gamma y_shared ----
       if (my_row >= 0) {
