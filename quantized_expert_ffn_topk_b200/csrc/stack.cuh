@@ -319,10 +319,10 @@ __device__ __forceinline__ bool flag_wait(const volatile int* f, int target, con
   return true;
 }
 
-// The sum of the G CTAs' published partial sums of squares, in one fixed
-// order (lane j adds entries j, j+32, ... then a butterfly over the lanes), so
-// every warp of every CTA gets the same value. The loads are all issued
-// before the first add (one L2 round trip for G <= 256).
+// The sum of the G CTAs' published partial sums of squares by one warp, in
+// one fixed order (lane j adds entries j, j+32, ... then a butterfly over the
+// lanes), so every CTA gets the same value. The loads are all issued before
+// the first add (one L2 round trip for G <= 256).
 __device__ __forceinline__ float sum_partials(const float* part, int G) {
   const int lane = threadIdx.x & 31;
   float v[8];
@@ -376,6 +376,7 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
   __shared__ volatile int s_topk_ready;
   __shared__ volatile int s_logits_ready;  // layer + 1 once s_logits holds that layer's logits
   __shared__ volatile int s_rh_arrived;    // layer + 1 once this CTA's routed h arrival is made
+  __shared__ float s_inv_norm;             // 1 / RMS of r_l (x staging)
 #ifdef MOEQ_STACK_TRACE
   __shared__ unsigned long long s_tr[6];
   if (threadIdx.x == 0) {
@@ -653,10 +654,16 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
           STACK_MARK(tid == 0, l, 1);
           named_sync(1, kCThreads);
           // the RMS norm's sum of squares from the CTAs' published partial
-          // sums, in one fixed order (every warp of every CTA gets the same
-          // value), read in the same round trip as r
+          // sums, in one fixed order (every CTA gets the same value), read by
+          // one warp in the same round trip as r (one reader per CTA of those
+          // few lines instead of sixteen)
           if (active) load_f32_16_cg(p.r + (size_t)tid * 16, v);
-          const float inv_norm = rsqrtf(sum_partials(p.ss_part, G) / (float)H + p.eps);
+          if (warp == 0) {
+            const float t = sum_partials(p.ss_part, G);
+            if (lane == 0) s_inv_norm = rsqrtf(t / (float)H + p.eps);
+          }
+          named_sync(1, kCThreads);
+          const float inv_norm = s_inv_norm;
           STACK_MARK(tid == 0 && v[0] == v[0], l, 19);
           if (active) {
 #pragma unroll
@@ -824,7 +831,12 @@ __global__ void __launch_bounds__(kStackThreads, 1) k_decode_layers(const __grid
       named_sync(1, kCThreads);
       (void)nseg;
       (void)ss;
-      const float inv = rsqrtf(sum_partials(p.ss_part, G) / (float)H + p.eps);
+      if (warp == 0) {
+        const float t = sum_partials(p.ss_part, G);
+        if (lane == 0) s_inv_norm = rsqrtf(t / (float)H + p.eps);
+      }
+      named_sync(1, kCThreads);
+      const float inv = s_inv_norm;
       if (my_row >= 0) p.xnorm_out[my_row] = f32_to_bf16_bits(my_r * inv);
     }
   }
