@@ -357,6 +357,39 @@ def test_combine_residual(with_gate, with_resid):
         assert (np.abs(xg - rn) <= np.abs(rn) * 2.0 ** -8 + 1e-30).all()
 
 
+@pytest.mark.parametrize("H,with_norm", [(4096, True), (4096, False), (16448, True)])
+def test_combine_residual_shapes(H, with_norm):
+    """The combine at the layer width (one row per thread of each cluster
+    CTA), without the normalised copy, and at a width where a thread owns
+    several rows (the partial sums of squares still meet across the cluster)."""
+    K, B = 4, 2
+    L = moeq.moe_layer_q(H=H, I=1024, E=64, K=K, group=64, bits_routed=4, bits_shared=4, experts=0x10000,
+                         shared=0x10000, router_w=0x10000, shared_gate_w=None)
+    rng = np.random.default_rng(H + with_norm)
+    y = torch.from_numpy(rng.normal(size=(B, K + 1, H)).astype(np.float32)).cuda()
+    wt = torch.from_numpy(rng.uniform(size=(B, K)).astype(np.float32)).cuda()
+    x = torch.from_numpy(rng.normal(size=(B, H)).astype(np.float32)).to(torch.bfloat16).cuda()
+    resid = torch.from_numpy(rng.normal(size=(B, H)).astype(np.float32)).cuda()
+    out = torch.empty((B, H), dtype=torch.float32, device="cuda")
+    xn = torch.empty((B, H), dtype=torch.bfloat16, device="cuda") if with_norm else None
+    moeq.moe_combine_residual(L, y, wt, x, resid, B, out, xn, 1e-6)
+    torch.cuda.synchronize()
+    for b in range(B):
+        yb, wb, rb = (t[b].cpu().numpy().astype(np.float64) for t in (y, wt, resid))
+        ro = ref.combine(yb, wb, 1.0, rb)
+        assert hz.max_rel_err(out[b].cpu().numpy(), ro) <= 1e-6
+        if with_norm:
+            rn = ref.rmsnorm(ro, 1e-6)
+            xg = hz.bf16_to_f64(hz.bf16_bits(xn[b]))
+            # one bf16 rounding, plus the fp32 error of r itself carried
+            # through 1/RMS: r = r_in + sum_k w_k y_k in fp32 is off by up to
+            # (K + 2) * 2^-23 * (|r_in| + sum_k |w_k y_k|) per element, which
+            # matters where the terms cancel
+            inv = np.abs(rn).sum() / np.abs(ro).sum()
+            mag = np.abs(rb) + (np.abs(wb[:, None] * yb[:K]).sum(axis=0)) + np.abs(yb[K])
+            assert (np.abs(xg - rn) <= np.abs(rn) * 2.0 ** -8 + inv * (K + 2) * 2.0 ** -23 * mag + 1e-30).all()
+
+
 # ---- A1..A6 whole layer -----------------------------------------------------------
 
 @pytest.mark.parametrize("name,B", [("tiny", 1), ("tiny", 4), ("layer4", 1), ("layer2", 1), ("layer4", 3),
