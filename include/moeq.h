@@ -321,8 +321,9 @@ moe_status moe_get_device_error(void* ws, void* stream);
  * such call; it is a convenience of this library.)
  *   L, x_bf16, B, idx, y_out, stream  as in moe_expert_ffn_q
  *   error_out  int32 device word, or NULL: receives the call's device error
- *              (0, or MOE_ERR_INDEX when an index was outside [0,E) and its
- *              slot was zeroed) in stream order
+ *              in stream order: 0, MOE_ERR_INDEX when an index was outside
+ *              [0,E) and its slot was zeroed, or MOE_ERR_TIMEOUT when a
+ *              bounded wait for a tile copy ran out (about one second)
  * Scratch is a MOEQ_STATIC_SCRATCH_BYTES array inside the library, held by
  * every GPU that loads it until the process exits. A shape whose
  * moe_workspace_bytes(B, K, H, I, E) exceeds that size is rejected with
