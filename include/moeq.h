@@ -256,7 +256,10 @@ moe_status moe_expert_ffn_q(const moe_layer_q* L, const void* x_bf16, int B, con
  *   gamma_b    1 when L->shared_gate_w is NULL, else sigmoid(w_sg . x[b])
  *   resid_out  fp32 [B, H] (may alias resid_in)
  *   xnorm_bf16_out  bf16 [B, H] or NULL: RMSNorm(out[b]) with unit weight
- *              and epsilon eps, rounded to nearest-even bf16
+ *              and epsilon eps, rounded to nearest-even bf16 (each token's
+ *              sum of squares is gathered across a cluster of 8 CTAs; a part
+ *              that has not arrived after about a second leaves that CTA's
+ *              eighth of the row NaN instead of waiting on)
  * Source: "Metal Compute Shaders" (MoE combine + residual + gate, RMS norm)
  * and "Deferred GPU Expert Compute" (combine + norm + residual feed the next
  * layer).
