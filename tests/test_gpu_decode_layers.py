@@ -83,6 +83,24 @@ def test_one_layer_matches_oracle(name):
     assert (np.abs(xg - rn) <= np.abs(rn) * 2.0 ** -8 + FFN_TOL * np.abs(rn).max()).all()
 
 
+@pytest.mark.parametrize("over", [dict(E=1024, K=8, group=128), dict(bits_routed=2, bits_shared=2),
+                                  dict(bits_routed=3, bits_shared=3, group=128)],
+                         ids=["E1024-K8-g128", "2bit-both", "3bit-both-g128"])
+def test_one_layer_other_shapes(over):
+    """The fused kernel at the most experts and picks it takes (its largest
+    item plan), at group 128 (four k-steps per group) and with the shared
+    expert at the routed width, one layer against the oracle."""
+    w, Ls = layers_for("layer4", 1, **over)
+    toks, skipped = hz.decided_tokens(w, 0, 1, 321, ref.router_logits)
+    x = hz.x_tokens_device(w, toks)[0]
+    ws, idx, wt, out, xn = run(w, Ls, x)
+    assert moeq.moe_get_device_error(ws.buf) == moeq.MOE_OK
+    ro = oracle_chain(w, 1, synth.x_host(w, toks[0])[0])[0]
+    assert list(idx[0]) == list(ro["idx"])
+    assert np.abs(wt[0] - ro["w"]).max() <= W_TOL
+    assert hz.max_rel_err(out, ro["out"]) <= FFN_TOL
+
+
 # ---- the 24-layer stack (87 GB resident) ------------------------------------------
 
 N_STACK = 24

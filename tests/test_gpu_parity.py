@@ -413,6 +413,29 @@ def test_layer_end_to_end(name, B):
     print("near-tie tokens skipped:", skipped)
 
 
+@pytest.mark.parametrize("over,B", [(dict(E=1024, K=8, group=128), 1), (dict(E=1024, K=8, group=128), 5),
+                                    (dict(bits_routed=2, bits_shared=2), 1), (dict(bits_routed=3, bits_shared=3,
+                                                                                   group=128), 3)],
+                         ids=["E1024-K8-g128-B1", "E1024-K8-g128-B5", "2bit-both-B1", "3bit-both-g128-B3"])
+def test_layer_end_to_end_other_shapes(over, B):
+    """The three per-token calls at the most experts and picks (E 1024, K 8),
+    at group 128 and with the shared expert at the routed width, for one token
+    and for a grouped batch: indices, weights, every slot and the residual."""
+    w, L = get_layer("layer4", **over)
+    toks, skipped = hz.decided_tokens(w, 0, B, 500, ref.router_logits)
+    x = hz.x_tokens_device(w, toks)
+    out = run_layer(w, L, x, eps=1e-6)
+    for b, t in enumerate(toks):
+        ro = oracle_token(w, 0, synth.x_host(w, t)[0], eps=1e-6)
+        assert list(out["idx"][b].cpu().numpy()) == list(ro["idx"]), (t, out["idx"][b].tolist(), list(ro["idx"]))
+        assert np.abs(out["w"][b].cpu().numpy() - ro["w"]).max() <= W_TOL
+        yg = out["y"][b].cpu().numpy()
+        for k in range(w.K + 1):
+            assert hz.max_rel_err(yg[k], ro["y"][k]) <= FFN_TOL
+        assert hz.max_rel_err(out["resid"][b].cpu().numpy(), ro["out"]) <= FFN_TOL
+    print("near-tie tokens skipped:", skipped)
+
+
 @pytest.mark.parametrize("B", [64, 128])
 def test_batched_zipf_larger_batches(B):
     """Batches of 64 and 128 tokens on the layer4 arena (Zipf(1.1) picks, so
